@@ -1,0 +1,188 @@
+/*
+ * int8row -- LLM.int8() mixed-precision linear layer for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every pointer argument is a DEVICE pointer unless stated otherwise;
+ * the caller owns every buffer, and no entry point allocates device memory.
+ * Every compute entry point is asynchronous on the given stream and returns
+ * as soon as its kernels are enqueued.  Matrices are row-major and contiguous
+ * (leading dimension = number of columns).  fp16 data is IEEE binary16,
+ * passed as `const void *` / `void *`.
+ *
+ * The method (web pages on LLM.int8()):
+ *   "LLM.int8()" abstract, taxoreview.com/v/2/lake/expert/dblp:280/8696;
+ *   "LLM.int8(): A Procedure for Int8 Matrix Multiplication in Transformer
+ *   Language Models", summarizepaper.com/en/paper/2208.07339v1, sections
+ *   "The LLM.int8() Methodology" and the summary bullets.
+ * A linear layer Y = X W is computed in two parts.  Vector-wise quantisation:
+ * every row of X and every output column of W gets its own absmax scale, so
+ * each inner product has its own pair of normalisation constants.
+ * Mixed-precision decomposition: the feature dimensions (columns of X) that
+ * hold an outlier are multiplied in 16-bit together with the matching rows
+ * of W; all other values are multiplied in int8 with int32 accumulation,
+ * dequantised by the outer product of the two scale vectors and added to
+ * the 16-bit partial result.
+ *
+ * Fixed choices where the pages give no number (one rule for all callers):
+ *   - column k of X is an outlier when any |X[t,k]| >= alpha;
+ *   - a scale is the absmax; a code is clamp(rhaz(v * fl32(127 / absmax)),
+ *     -127, 127) with rhaz = round half away from zero, one fp32 division
+ *     per row/column and one fp32 multiply per element; absmax 0 gives codes 0;
+ *   - row scales of X are taken over the non-outlier columns only, and the
+ *     outlier columns are 0 in the int8 operand;
+ *   - column scales of W are taken over all K rows;
+ *   - the 16-bit part uses the fp16 rows W16[k,:] for k in the outlier set,
+ *     with fp32 accumulation; the result is rounded to fp16 (nearest-even).
+ *
+ * Shape rules shared by the entry points: T >= 0 (T == 0 is a no-op that
+ * returns I8R_OK), 16 <= K <= 133144 (int32 accumulation is exact while
+ * K * 127^2 < 2^31), K % 16 == 0, 16 <= N, N % 16 == 0, and every pointer
+ * 16-byte aligned.  A violated rule is reported before anything is
+ * enqueued, and nothing is written.
+ *
+ * Device-side anomalies (a pipeline wait that exceeded its time limit) do
+ * not trap: the kernel records a code in a per-device status word and
+ * returns early.  Read it with int8_read_and_clear_device_status().
+ */
+#ifndef INT8ROW_H
+#define INT8ROW_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    I8R_OK = 0,
+    I8R_EINVAL = 1,      /* null pointer, negative size, NaN or negative alpha */
+    I8R_EALIGN = 2,      /* pointer not 16-byte aligned, K or N not a multiple of 16 */
+    I8R_ERANGE = 3,      /* K > 133144, K < 16, N < 16, or a size beyond the library's limits */
+    I8R_EWORKSPACE = 4,  /* workspace pointer null or smaller than the queried size */
+    I8R_ECUDA = 5,       /* a CUDA runtime/driver call failed (see int8_last_cuda_error) */
+    I8R_EDEVICE = 6,     /* the device status word holds a kernel-reported anomaly */
+    I8R_EARCH = 7        /* the current device is not sm_100 (B200) */
+} i8r_status;
+
+/* Device status codes written by kernels (returned by
+ * int8_read_and_clear_device_status). */
+#define I8R_DEV_OK 0
+#define I8R_DEV_PIPELINE_TIMEOUT 1   /* a shared-memory pipeline wait gave up */
+#define I8R_DEV_TMEM_TIMEOUT 2       /* a tensor-memory hand-off wait gave up */
+
+/* ---------------------------------------------------------------------------
+ * Weight conversion.  The pages describe a 16/32-bit checkpoint converted to
+ * Int8 at load time and used straight away, with one normalisation constant
+ * per output column of W (LLM.int8() abstract; "The LLM.int8() Methodology").
+ *
+ *   W16 [K,N] fp16   input weight
+ *   Wq  [K,N] int8   output codes, Wq[k,n] = clamp(rhaz(W16[k,n] * fl32(127/sW[n])), +-127)
+ *   sW  [N]   fp32   output column absmax, sW[n] = max_k |W16[k,n]|
+ * Enqueues two HBM-bound kernels; needs no workspace.
+ * ------------------------------------------------------------------------- */
+i8r_status int8_quantize_weight_colwise(const void *W16, int K, int N,
+                                        int8_t *Wq, float *sW, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The mixed-precision linear layer (LLM.int8() abstract; "The LLM.int8()
+ * Methodology"; the summary's bullets on vector-wise quantisation and the
+ * mixed-precision decomposition).
+ *
+ *   X   [T,K] fp16   activation
+ *   Wq  [K,N] int8   and sW [N] fp32: from int8_quantize_weight_colwise
+ *   W16 [K,N] fp16   the fp16 weight; only its rows in the outlier set are read
+ *   alpha            outlier threshold (>= 0; +inf disables the 16-bit part)
+ *   Y   [T,N] fp16   output, Y = fp16( acc*sX[t]*sW[n]/127^2 + X[:,O] W16[O,:] )
+ *                    with acc the exact int32 product of the int8 codes
+ *   workspace        device scratch of at least
+ *                    int8_mixed_linear_workspace_size(T, K, N) bytes, 256-byte
+ *                    aligned; its contents on entry are ignored and on return
+ *                    are unspecified (it holds the quantised activation)
+ * Two calls that share a workspace must not overlap on the GPU.
+ * T <= 128 runs the decode-shaped kernel (weight streaming, split over K);
+ * larger T runs the prefill kernel (tensor-core bound).
+ * ------------------------------------------------------------------------- */
+size_t int8_mixed_linear_workspace_size(int T, int K, int N);
+
+i8r_status int8_mixed_linear(const void *X, int T, int K,
+                             const int8_t *Wq, const float *sW, const void *W16, int N,
+                             float alpha, void *Y,
+                             void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Outlier statistics: the outlier feature dimensions of X and the share of
+ * values that go through the 8-bit product (the pages report that share as
+ * above 99.9% on large models; LLM.int8() abstract).
+ *
+ *   num_outlier_cols [1] int32   |O|
+ *   col_idx          [K] int32   O in ascending order in [0, |O|); the rest untouched
+ *   col_hit_count    [K] int32   rows t with |X[t,k]| >= alpha, per column (nullable)
+ *   frac_8bit        [1] fp32    1 - |O|/K, computed in double and rounded to fp32
+ *   workspace        at least int8_outlier_stats_workspace_size(K) bytes
+ * ------------------------------------------------------------------------- */
+size_t int8_outlier_stats_workspace_size(int K);
+
+i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha,
+                              int32_t *num_outlier_cols, int32_t *col_idx,
+                              int32_t *col_hit_count, float *frac_8bit,
+                              void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Intermediate results, for checking the pipeline stage by stage.
+ *
+ * int8_quantize_activation: the activation side of int8_mixed_linear
+ *   mask  [ceil(K/32)] uint32   bit k%32 of word k/32 set when column k is an outlier
+ *   idx   [K] int32             O ascending in [0, count)
+ *   count [1] int32             |O|
+ *   sX    [T] fp32              row absmax over the non-outlier columns
+ *   Xq    [T,K] int8            row codes, 0 in outlier columns
+ *   Xo    [T,K] fp16 (nullable) Xo[t,j] = X[t, idx[j]] for j < |O|, 0 for
+ *                               |O| <= j < 64*ceil(|O|/64); later columns untouched
+ *
+ * int8_gemm_i8_s32: acc [T,N] int32 = Xq [T,K] int8 x Wq [K,N] int8, exact,
+ *   by the same tensor-core kernels int8_mixed_linear uses (decode-shaped for
+ *   T <= 128, prefill otherwise).  Needs workspace of at least
+ *   int8_gemm_i8_s32_workspace_size(T, K, N) bytes (may be 0; pass NULL then).
+ * ------------------------------------------------------------------------- */
+i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha,
+                                    uint32_t *mask, int32_t *idx, int32_t *count,
+                                    float *sX, int8_t *Xq, void *Xo,
+                                    cudaStream_t stream);
+
+size_t int8_gemm_i8_s32_workspace_size(int T, int K, int N);
+
+i8r_status int8_gemm_i8_s32(const int8_t *Xq, int T, int K, const int8_t *Wq, int N,
+                            int32_t *acc, void *workspace, size_t workspace_bytes,
+                            cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Status, errors and measurement.
+ * ------------------------------------------------------------------------- */
+
+/* Synchronises `stream`, then returns in *code (HOST pointer) the current
+ * device's status word (I8R_DEV_*) and resets it to I8R_DEV_OK. */
+i8r_status int8_read_and_clear_device_status(int *code, cudaStream_t stream);
+
+/* Static description of a status code. */
+const char *int8_status_string(i8r_status status);
+
+/* The last CUDA error seen by an entry point on this host thread (cudaError_t). */
+int int8_last_cuda_error(void);
+
+/* Measurement hook: the next int8_mixed_linear or int8_gemm_i8_s32 call made
+ * by this host thread records `before` (a cudaEvent_t) on its stream right
+ * before its tensor-core GEMM kernel and `after` right after it, then forgets
+ * both.  Pass NULL, NULL to cancel. */
+void int8_time_next_gemm(cudaEvent_t before, cudaEvent_t after);
+
+/* Number of kernels this library has enqueued in this process (all threads,
+ * all devices), for launch accounting. */
+uint64_t int8_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* INT8ROW_H */

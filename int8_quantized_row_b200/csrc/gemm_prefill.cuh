@@ -1,0 +1,310 @@
+// Prefill-shaped LLM.int8() GEMM on sm_100a tensor cores.
+//
+// One persistent CTA per SM walks 128 x 256 output tiles (rows of X x columns
+// of W).  Per tile:
+//   8-bit part:  acc_i32[128x256] (TMEM cols 0..255)  = sum_k Xq[t,k] Wq[k,n]
+//                tcgen05.mma kind::i8, A = Xq tile K-major, B = Wq tile MN-major
+//   16-bit part: acc_f32[128x256] (TMEM cols 256..511) = sum_j Xo[t,j] W16[O_j,n]
+//                tcgen05.mma kind::f16 over ceil(|O|/16) K-steps; |O| is read
+//                from device memory, so no host round trip
+//   epilogue:    Y = fp16(acc_i32 * sX[t] * sW[n] / 127^2 + acc_f32)
+// (vector-wise scales + mixed-precision decomposition: LLM.int8() abstract;
+// "The LLM.int8() Methodology".)
+//
+// Warp roles (192 threads):
+//   warp 0  producer: TMA loads of Xq / Wq / Xo tiles into a 4-stage ring; the
+//           W16 outlier rows are fetched by index with cp.async (all 32 lanes),
+//           then fenced into the async proxy before the stage is published
+//   warp 1  TMEM allocation + MMA issue (one lane)
+//   warps 2-5 epilogue: tcgen05.ld of their 32-lane quadrant, scale, store
+// Shared-memory stage: A 128 rows x 128 B (16 KB) + B 256 x 128 B (32 KB).  An
+// outlier stage reuses the same bytes: A = 128 rows x 64 fp16, B = 64 outlier
+// rows x 256 fp16 (4 MN-major chunks of 64 columns).
+#pragma once
+
+#include "device_common.cuh"
+
+namespace i8r {
+namespace prefill {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 128;                    // int8 K per stage (bytes)
+constexpr int OBK = 64;                    // fp16 K (outlier columns) per outlier stage
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK;           // 16 KB
+constexpr int B_BYTES = BN * BK;           // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int B_CHUNK_I8 = 128 * BK;       // 128 columns x 128 k-rows
+constexpr int B_CHUNK_F16 = 64 * OBK * 2;  // 64 columns x 64 rows of fp16 = 8 KB
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC16_COL = 256;
+constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+
+struct Params {
+    int T, K, N;
+    int num_m, num_tiles, KB;
+    const int32_t *count;      // |O| (device); nullptr => no 16-bit part
+    const int32_t *idx;        // O, ascending
+    const __half *W16;         // [K,N] fp16, rows read by index
+    const float *sX;           // [T]
+    const float *sW;           // [N]
+    __half *Y;                 // [T,N] fp16 (mode Y)
+    int32_t *acc_out;          // [T,N] int32 (mode S32)
+};
+
+struct Barriers {
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t tmem_full;
+    uint64_t tmem_empty;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+template <bool kS32>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_prefill_kernel(const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
+                        const __grid_constant__ CUtensorMap map_xo, const Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Barriers *bars = reinterpret_cast<Barriers *>(smem + STAGES * STAGE_BYTES);
+    volatile int *abort = &bars->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int count = (!kS32 && p.count) ? *p.count : 0;
+    const int nob = (count + OBK - 1) / OBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], 1);
+        }
+        mbar_init(&bars->tmem_full, 1);
+        mbar_init(&bars->tmem_empty, 4);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        fence_mbar_init();
+        tma_prefetch_map(&map_xq);
+        tma_prefetch_map(&map_wq);
+        if (nob) tma_prefetch_map(&map_xo);
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars->tmem_base, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int stage = 0;
+        uint32_t phase = 0;
+        int pending[STAGES];
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) pending[s] = -1;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+            const int m0 = (tile % p.num_m) * BM;
+            const int n0 = (tile / p.num_m) * BN;
+            for (int kb = 0; kb < p.KB; ++kb) {
+                if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
+                if (lane == 0) {
+                    uint8_t *a = smem + stage * STAGE_BYTES;
+                    uint8_t *b = a + A_BYTES;
+                    mbar_arrive_expect_tx(&bars->full[stage], STAGE_BYTES);
+                    tma_load_2d(a, &map_xq, &bars->full[stage], kb * BK, m0);
+                    tma_load_2d(b, &map_wq, &bars->full[stage], n0, kb * BK);
+                    tma_load_2d(b + B_CHUNK_I8, &map_wq, &bars->full[stage], n0 + 128, kb * BK);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int s = 0; s < STAGES; ++s) if (s == stage) pending[s] = static_cast<int>(phase);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            for (int ob = 0; ok && ob < nob; ++ob) {
+                if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
+                uint8_t *a = smem + stage * STAGE_BYTES;
+                const uint32_t b = smem_u32(a + A_BYTES);
+                // rows of W16 for outliers ob*64 .. ob*64+63, zero past |O| (rounded to 16)
+                const int rows = min(OBK, (count - ob * OBK + 15) / 16 * 16);
+                const int g0 = ob * OBK + lane, g1 = ob * OBK + 32 + lane;
+                const int k0 = g0 < count ? p.idx[g0] : -1;
+                const int k1 = g1 < count ? p.idx[g1] : -1;
+                const int n = n0 + lane * 8;       // this lane's 8 columns
+                const uint32_t chunk = b + (lane >> 3) * B_CHUNK_F16;
+                const uint32_t unit = lane & 7;
+                for (int j = 0; j < rows; ++j) {
+                    const int k = __shfl_sync(0xFFFFFFFFu, j < 32 ? k0 : k1, j & 31);
+                    const bool have = (k >= 0) && (n < p.N);
+                    const __half *src = have ? p.W16 + static_cast<size_t>(k) * p.N + n : p.W16;
+                    const uint32_t dst = chunk + j * 128 + ((unit ^ (j & 7)) << 4);   // 128-B swizzle
+                    cp_async_16(dst, src, have ? 16u : 0u);
+                }
+                // make the rows visible to the tensor core (async proxy) before
+                // the stage is published
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&bars->full[stage], A_BYTES);
+                    tma_load_2d(a, &map_xo, &bars->full[stage], ob * OBK, m0);
+                }
+                __syncwarp();
+#pragma unroll
+                for (int s = 0; s < STAGES; ++s) if (s == stage) pending[s] = static_cast<int>(phase);
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+        }
+        // Before leaving, make sure nothing this warp issued is still landing in
+        // shared memory (only matters after an abort).
+        if (!ok && lane == 0) {
+            volatile int never = 0;
+#pragma unroll
+            for (int s = 0; s < STAGES; ++s)
+                if (pending[s] >= 0) mbar_wait(&bars->full[s], static_cast<uint32_t>(pending[s]), &never, 0);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        const uint32_t id_i8 = idesc_i8(BM, BN, false, true);
+        const uint32_t id_f16 = idesc_f16(BM, BN, false, true);
+        int stage = 0;
+        uint32_t phase = 0, tphase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+            if (!warp_wait(&bars->tmem_empty, tphase ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) { ok = false; break; }
+            tc_fence_after_sync();
+            for (int kb = 0; kb < p.KB; ++kb) {
+                if (!warp_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
+                tc_fence_after_sync();
+                if (lane == 0) {
+                    const uint32_t a = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t b = a + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 32; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(a + kk * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(b + kk * 32 * 128, B_CHUNK_I8, 1024);
+                        mma_i8(tmem, ad, bd, id_i8, (kb | kk) != 0);
+                    }
+                    mma_commit(&bars->empty[stage]);
+                }
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            for (int ob = 0; ok && ob < nob; ++ob) {
+                if (!warp_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
+                tc_fence_after_sync();
+                fence_proxy_async_smem();   // cp.async (generic proxy) data -> tensor core reads
+                if (lane == 0) {
+                    const uint32_t a = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t b = a + A_BYTES;
+                    const int nk = min(OBK / 16, (count - ob * OBK + 15) / 16);
+                    for (int kk = 0; kk < nk; ++kk) {
+                        const uint64_t ad = smem_desc_sw128(a + kk * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(b + kk * 16 * 128, B_CHUNK_F16, 1024);
+                        mma_f16(tmem + ACC16_COL, ad, bd, id_f16, (ob | kk) != 0);
+                    }
+                    mma_commit(&bars->empty[stage]);
+                }
+                __syncwarp();
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok) break;
+            if (lane == 0) mma_commit(&bars->tmem_full);
+            __syncwarp();
+            tphase ^= 1u;
+        }
+        // Drain: every MMA this thread issued has completed before TMEM is freed.
+        if (lane == 0) {
+            volatile int never = 0;
+            mma_commit(&bars->drain);
+            mbar_wait(&bars->drain, 0, &never, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
+        const int row = quad * 32 + lane;
+        uint32_t tphase = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+            if (!warp_wait(&bars->tmem_full, tphase, abort, I8R_DEV_TMEM_TIMEOUT)) break;
+            tc_fence_after_sync();
+            const int m0 = (tile % p.num_m) * BM;
+            const int n0 = (tile / p.num_m) * BN;
+            const int t = m0 + row;
+            const bool row_ok = t < p.T;
+            const float rs = (!kS32 && row_ok) ? p.sX[t] * (1.0f / 16129.0f) : 0.0f;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int nc = n0 + c * 32;
+                uint32_t r[32];
+                tmem_ld32(taddr + c * 32, r);
+                uint32_t f[32];
+                if (!kS32 && nob) tmem_ld32(taddr + ACC16_COL + c * 32, f);
+                tmem_wait_ld();
+                if (kS32) {
+                    if (row_ok) {
+                        int4 *dst = reinterpret_cast<int4 *>(p.acc_out + static_cast<size_t>(t) * p.N + nc);
+#pragma unroll
+                        for (int g = 0; g < 8; ++g)
+                            if (nc + g * 4 < p.N)
+                                dst[g] = make_int4(static_cast<int>(r[4 * g]), static_cast<int>(r[4 * g + 1]),
+                                                   static_cast<int>(r[4 * g + 2]), static_cast<int>(r[4 * g + 3]));
+                    }
+                } else {
+                    uint4 out[4];
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        float sw[8];
+                        if (nc + g * 8 < p.N) {
+                            const float4 s0 = __ldg(reinterpret_cast<const float4 *>(p.sW + nc + g * 8));
+                            const float4 s1 = __ldg(reinterpret_cast<const float4 *>(p.sW + nc + g * 8 + 4));
+                            sw[0] = s0.x; sw[1] = s0.y; sw[2] = s0.z; sw[3] = s0.w;
+                            sw[4] = s1.x; sw[5] = s1.y; sw[6] = s1.z; sw[7] = s1.w;
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) sw[e] = 0.0f;
+                        }
+                        __half2 h[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int i0 = g * 8 + 2 * e, i1 = i0 + 1;
+                            const float y0 = fmaf(static_cast<float>(static_cast<int>(r[i0])), rs * sw[2 * e],
+                                                  nob ? __uint_as_float(f[i0]) : 0.0f);
+                            const float y1 = fmaf(static_cast<float>(static_cast<int>(r[i1])), rs * sw[2 * e + 1],
+                                                  nob ? __uint_as_float(f[i1]) : 0.0f);
+                            h[e] = __floats2half2_rn(y0, y1);
+                        }
+                        out[g] = *reinterpret_cast<uint4 *>(h);
+                    }
+                    if (row_ok) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.Y + static_cast<size_t>(t) * p.N + nc);
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            if (nc + g * 8 < p.N) dst[g] = out[g];
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tmem_empty);
+            tphase ^= 1u;
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace prefill
+}  // namespace i8r

@@ -1,0 +1,456 @@
+// int8row C ABI: argument checks, workspace layout, tensor maps, launches.
+// The declarations and their contracts are in include/int8row.h.
+//
+// Pipeline of int8_mixed_linear (all on the caller's stream, no host sync):
+//   outlier_mask_kernel     X -> outlier column bitmask              (a1)
+//   outlier_index_kernel    bitmask -> ascending index list, |O|      (a1)
+//   quantize_rows_kernel    X -> sX, Xq (outliers zeroed), Xo gather  (a2, a3)
+//   T > 128:  gemm_prefill_kernel  int8 + fp16 tensor-core MMA, epilogue -> Y
+//   T <= 128: gemm_decode_kernel   split-K int8 MMA -> int32 partial sums,
+//             finalize_kernel      scales + fp16 outlier part -> Y
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "int8row.h"
+#include "device_common.cuh"
+#include "quant_kernels.cuh"
+#include "gemm_prefill.cuh"
+#include "gemm_decode.cuh"
+
+namespace {
+
+using namespace i8r;
+
+constexpr int kMaxK = 133144;          // K * 127^2 < 2^31
+constexpr int kMaxDevices = 64;
+constexpr size_t kAlign = 256;
+
+std::atomic<uint64_t> g_launches{0};
+thread_local int tl_last_cuda_error = 0;
+thread_local cudaEvent_t tl_ev_before = nullptr;
+thread_local cudaEvent_t tl_ev_after = nullptr;
+
+struct DeviceInfo {
+    bool ready = false;
+    bool sm100 = false;
+    int sms = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+#define I8R_CUDA(call)                                             \
+    do {                                                           \
+        cudaError_t e_ = (call);                                   \
+        if (e_ != cudaSuccess) {                                   \
+            tl_last_cuda_error = static_cast<int>(e_);             \
+            return I8R_ECUDA;                                      \
+        }                                                          \
+    } while (0)
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device one-time setup: architecture check, SM count, kernel attributes,
+// the driver's tensor-map encoder.
+i8r_status device_setup(const DeviceInfo **out) {
+    int dev = 0;
+    I8R_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return I8R_ERANGE;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        I8R_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+        I8R_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+        I8R_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+        d.sm100 = (major == 10 && minor == 0);
+        if (d.sm100) {
+            I8R_CUDA(cudaFuncSetAttribute(prefill::gemm_prefill_kernel<false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(prefill::SMEM_BYTES)));
+            I8R_CUDA(cudaFuncSetAttribute(prefill::gemm_prefill_kernel<true>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(prefill::SMEM_BYTES)));
+            I8R_CUDA(cudaFuncSetAttribute(decode::gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(decode::SMEM_BUDGET + 4096)));
+        }
+        if (!g_encode) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            I8R_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+            if (q != cudaDriverEntryPointSuccess || !fn) return I8R_ECUDA;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        d.ready = true;
+    }
+    if (!d.sm100) return I8R_EARCH;
+    *out = &d;
+    return I8R_OK;
+}
+
+// 2-D row-major tensor [rows, cols] of `elem` bytes, box [box_rows, box_cols],
+// 128-byte swizzle, zero fill out of bounds.
+i8r_status make_map(CUtensorMap *map, const void *base, CUtensorMapDataType type, int elem, uint64_t rows,
+                    uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem)};
+    const cuuint32_t box[2] = {box_cols, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        tl_last_cuda_error = static_cast<int>(r);
+        return I8R_ECUDA;
+    }
+    return I8R_OK;
+}
+
+i8r_status check_launch() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = static_cast<int>(e);
+        return I8R_ECUDA;
+    }
+    return I8R_OK;
+}
+
+#define I8R_LAUNCHED()                        \
+    do {                                      \
+        i8r_status s_ = check_launch();       \
+        if (s_ != I8R_OK) return s_;          \
+    } while (0)
+
+i8r_status check_shape(int T, int K, int N, bool need_n) {
+    if (T < 0 || K < 0 || (need_n && N < 0)) return I8R_EINVAL;
+    if (K < 16 || K > kMaxK) return I8R_ERANGE;
+    if (K % 16) return I8R_EALIGN;
+    if (need_n) {
+        if (N < 16) return I8R_ERANGE;
+        if (N % 16) return I8R_EALIGN;
+    }
+    return I8R_OK;
+}
+
+i8r_status check_ptr(const void *p) {
+    if (!p) return I8R_EINVAL;
+    if (!aligned16(p)) return I8R_EALIGN;
+    return I8R_OK;
+}
+
+#define I8R_TRY(expr)                         \
+    do {                                      \
+        i8r_status s_ = (expr);               \
+        if (s_ != I8R_OK) return s_;          \
+    } while (0)
+
+// Workspace of int8_mixed_linear.
+struct Workspace {
+    size_t count, mask, idx, sX, Xq, Xo, acc32, total;
+};
+
+Workspace ws_layout(int T, int K, int N) {
+    Workspace w{};
+    size_t off = 0;
+    w.count = off; off = align_up(off + sizeof(int32_t));
+    w.mask = off;  off = align_up(off + static_cast<size_t>((K + 31) / 32) * 4);
+    w.idx = off;   off = align_up(off + static_cast<size_t>(K) * 4);
+    w.sX = off;    off = align_up(off + static_cast<size_t>(T) * 4);
+    w.Xq = off;    off = align_up(off + static_cast<size_t>(T) * K);
+    w.Xo = off;    off = align_up(off + static_cast<size_t>(T) * K * 2);
+    w.acc32 = off;
+    if (T <= decode::MAX_T) off = align_up(off + static_cast<size_t>(T) * N * 4);
+    w.total = off;
+    return w;
+}
+
+// a1-a3 on the stream: mask, index list, row quantisation and gather.
+i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_t *mask, int32_t *idx,
+                             int32_t *count, float *sX, int8_t *Xq, __half *Xo, int32_t *acc32, int N,
+                             cudaStream_t s) {
+    outlier_mask_kernel<false><<<(K + kStripCols - 1) / kStripCols, kStripThreads, 0, s>>>(X, T, K, alpha, mask,
+                                                                                          nullptr);
+    I8R_LAUNCHED();
+    outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(mask, K, idx, count, nullptr);
+    I8R_LAUNCHED();
+    if (T > 0) {
+        quantize_rows_kernel<<<T, kRowThreads, 0, s>>>(X, T, K, mask, idx, count, sX, Xq, Xo, acc32, N);
+        I8R_LAUNCHED();
+    }
+    return I8R_OK;
+}
+
+void record_before(cudaStream_t s) {
+    if (tl_ev_before) cudaEventRecord(tl_ev_before, s);
+}
+void record_after(cudaStream_t s) {
+    if (tl_ev_after) cudaEventRecord(tl_ev_after, s);
+    tl_ev_before = nullptr;
+    tl_ev_after = nullptr;
+}
+
+// Prefill GEMM (T > 128): Y mode when Y != nullptr, else int32 accumulators.
+i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
+                          const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
+                          const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
+    CUtensorMap map_xq, map_wq, map_xo;
+    I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, prefill::BM, prefill::BK));
+    I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, prefill::BK, 128));
+    if (Xo) {
+        I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, prefill::BM, prefill::OBK));
+    } else {
+        map_xo = map_xq;   // unused: no 16-bit part
+    }
+    prefill::Params p{};
+    p.T = T;
+    p.K = K;
+    p.N = N;
+    p.num_m = (T + prefill::BM - 1) / prefill::BM;
+    const int num_n = (N + prefill::BN - 1) / prefill::BN;
+    p.num_tiles = p.num_m * num_n;
+    p.KB = (K + prefill::BK - 1) / prefill::BK;
+    p.count = Y ? count : nullptr;
+    p.idx = idx;
+    p.W16 = W16;
+    p.sX = sX;
+    p.sW = sW;
+    p.Y = Y;
+    p.acc_out = acc_out;
+    const int grid = p.num_tiles < dev->sms ? p.num_tiles : dev->sms;
+    record_before(s);
+    if (Y)
+        prefill::gemm_prefill_kernel<false><<<grid, prefill::THREADS, prefill::SMEM_BYTES, s>>>(map_xq, map_wq,
+                                                                                              map_xo, p);
+    else
+        prefill::gemm_prefill_kernel<true><<<grid, prefill::THREADS, prefill::SMEM_BYTES, s>>>(map_xq, map_wq,
+                                                                                             map_xo, p);
+    I8R_LAUNCHED();
+    record_after(s);
+    return I8R_OK;
+}
+
+// Decode GEMM (T <= 128): int32 partial sums added into acc32, which must be
+// zero on entry.
+i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, const int8_t *Wq, int N,
+                         int32_t *acc32, cudaStream_t s) {
+    decode::Params p{};
+    p.T = T;
+    p.TP = (T + 15) / 16 * 16;
+    p.K = K;
+    p.N = N;
+    p.KB = (K + decode::BK - 1) / decode::BK;
+    p.num_tiles = (N + decode::BM - 1) / decode::BM;
+    p.total_units = static_cast<long long>(p.num_tiles) * p.KB;
+    p.stage_bytes = decode::A_BYTES + p.TP * decode::BK;
+    p.stages = static_cast<int>(decode::SMEM_BUDGET / p.stage_bytes);
+    if (p.stages > decode::MAX_STAGES) p.stages = decode::MAX_STAGES;
+    uint32_t cols = 32;
+    while (cols < static_cast<uint32_t>(2 * p.TP)) cols <<= 1;
+    p.tmem_cols = cols;
+    p.acc32 = acc32;
+    CUtensorMap map_wq, map_xq;
+    I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BM));
+    I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, p.TP, decode::BK));
+    const long long g = p.total_units < dev->sms ? p.total_units : dev->sms;
+    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes);
+    record_before(s);
+    decode::gemm_decode_kernel<<<static_cast<int>(g), decode::THREADS, smem, s>>>(map_wq, map_xq, p);
+    I8R_LAUNCHED();
+    record_after(s);
+    return I8R_OK;
+}
+
+__global__ void zero_kernel(int4 *p, size_t n16) {
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n16;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x)
+        p[i] = make_int4(0, 0, 0, 0);
+}
+
+}  // namespace
+
+extern "C" {
+
+i8r_status int8_quantize_weight_colwise(const void *W16, int K, int N, int8_t *Wq, float *sW, cudaStream_t stream) {
+    I8R_TRY(check_shape(0, K, N, true));
+    I8R_TRY(check_ptr(W16));
+    I8R_TRY(check_ptr(Wq));
+    I8R_TRY(check_ptr(sW));
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+    const __half *w = static_cast<const __half *>(W16);
+    weight_absmax_kernel<<<(N + kStripCols - 1) / kStripCols, kStripThreads, 0, stream>>>(w, K, N, sW);
+    I8R_LAUNCHED();
+    const size_t groups = static_cast<size_t>(K) * (N / 8);
+    size_t blocks = (groups + 255) / 256;
+    const size_t cap = static_cast<size_t>(dev->sms) * 16;
+    if (blocks > cap) blocks = cap;
+    weight_codes_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(w, K, N, sW, Wq);
+    I8R_LAUNCHED();
+    return I8R_OK;
+}
+
+size_t int8_mixed_linear_workspace_size(int T, int K, int N) {
+    if (T < 0 || K < 0 || N < 0) return 0;
+    return ws_layout(T, K, N).total;
+}
+
+i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, const float *sW, const void *W16, int N,
+                             float alpha, void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    I8R_TRY(check_shape(T, K, N, true));
+    if (std::isnan(alpha) || alpha < 0.0f) return I8R_EINVAL;
+    if (T == 0) return I8R_OK;
+    I8R_TRY(check_ptr(X));
+    I8R_TRY(check_ptr(Wq));
+    I8R_TRY(check_ptr(sW));
+    I8R_TRY(check_ptr(W16));
+    I8R_TRY(check_ptr(Y));
+    const Workspace w = ws_layout(T, K, N);
+    if (!workspace || workspace_bytes < w.total) return I8R_EWORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return I8R_EALIGN;
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    int32_t *count = reinterpret_cast<int32_t *>(ws + w.count);
+    uint32_t *mask = reinterpret_cast<uint32_t *>(ws + w.mask);
+    int32_t *idx = reinterpret_cast<int32_t *>(ws + w.idx);
+    float *sX = reinterpret_cast<float *>(ws + w.sX);
+    int8_t *Xq = reinterpret_cast<int8_t *>(ws + w.Xq);
+    __half *Xo = reinterpret_cast<__half *>(ws + w.Xo);
+    const bool small_t = T <= decode::MAX_T;
+    int32_t *acc32 = small_t ? reinterpret_cast<int32_t *>(ws + w.acc32) : nullptr;
+    const __half *x = static_cast<const __half *>(X);
+    const __half *w16 = static_cast<const __half *>(W16);
+    __half *y = static_cast<__half *>(Y);
+
+    I8R_TRY(launch_activation(x, T, K, alpha, mask, idx, count, sX, Xq, Xo, acc32, N, stream));
+    if (!small_t)
+        return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream);
+
+    I8R_TRY(launch_decode(dev, Xq, T, K, Wq, N, acc32, stream));
+    dim3 grid((N / 8 + decode::FIN_THREADS - 1) / decode::FIN_THREADS, (T + decode::FIN_ROWS - 1) / decode::FIN_ROWS);
+    decode::finalize_kernel<<<grid, decode::FIN_THREADS, 0, stream>>>(acc32, T, K, N, sX, sW, Xo, idx, count, w16, y);
+    I8R_LAUNCHED();
+    return I8R_OK;
+}
+
+size_t int8_outlier_stats_workspace_size(int K) {
+    if (K < 0) return 0;
+    return align_up(static_cast<size_t>((K + 31) / 32) * 4);
+}
+
+i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha, int32_t *num_outlier_cols, int32_t *col_idx,
+                              int32_t *col_hit_count, float *frac_8bit, void *workspace, size_t workspace_bytes,
+                              cudaStream_t stream) {
+    I8R_TRY(check_shape(T, K, 0, false));
+    if (std::isnan(alpha) || alpha < 0.0f) return I8R_EINVAL;
+    if (T > 0) I8R_TRY(check_ptr(X));
+    if (!num_outlier_cols || !col_idx || !frac_8bit) return I8R_EINVAL;
+    if (col_hit_count && !aligned16(col_hit_count)) return I8R_EALIGN;
+    if (!workspace || workspace_bytes < int8_outlier_stats_workspace_size(K)) return I8R_EWORKSPACE;
+    if (!aligned16(workspace)) return I8R_EALIGN;
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+    uint32_t *mask = static_cast<uint32_t *>(workspace);
+    const int blocks = (K + kStripCols - 1) / kStripCols;
+    const __half *x = static_cast<const __half *>(X);
+    if (col_hit_count)
+        outlier_mask_kernel<true><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, mask, col_hit_count);
+    else
+        outlier_mask_kernel<false><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, mask, nullptr);
+    I8R_LAUNCHED();
+    outlier_index_kernel<<<1, kIndexThreads, 0, stream>>>(mask, K, col_idx, num_outlier_cols, frac_8bit);
+    I8R_LAUNCHED();
+    return I8R_OK;
+}
+
+i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha, uint32_t *mask, int32_t *idx,
+                                    int32_t *count, float *sX, int8_t *Xq, void *Xo, cudaStream_t stream) {
+    I8R_TRY(check_shape(T, K, 0, false));
+    if (std::isnan(alpha) || alpha < 0.0f) return I8R_EINVAL;
+    if (T > 0) {
+        I8R_TRY(check_ptr(X));
+        I8R_TRY(check_ptr(sX));
+        I8R_TRY(check_ptr(Xq));
+        if (Xo) I8R_TRY(check_ptr(Xo));
+    }
+    I8R_TRY(check_ptr(mask));
+    I8R_TRY(check_ptr(idx));
+    if (!count) return I8R_EINVAL;
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+    return launch_activation(static_cast<const __half *>(X), T, K, alpha, mask, idx, count, sX, Xq,
+                             static_cast<__half *>(Xo), nullptr, 0, stream);
+}
+
+size_t int8_gemm_i8_s32_workspace_size(int T, int K, int N) {
+    (void)T;
+    (void)K;
+    (void)N;
+    return 0;
+}
+
+i8r_status int8_gemm_i8_s32(const int8_t *Xq, int T, int K, const int8_t *Wq, int N, int32_t *acc, void *workspace,
+                            size_t workspace_bytes, cudaStream_t stream) {
+    (void)workspace;
+    (void)workspace_bytes;
+    I8R_TRY(check_shape(T, K, N, true));
+    if (T == 0) return I8R_OK;
+    I8R_TRY(check_ptr(Xq));
+    I8R_TRY(check_ptr(Wq));
+    I8R_TRY(check_ptr(acc));
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+    if (T > decode::MAX_T)
+        return launch_prefill(dev, Xq, nullptr, T, K, Wq, nullptr, nullptr, N, nullptr, nullptr, nullptr, nullptr,
+                              acc, stream);
+    const size_t n16 = static_cast<size_t>(T) * N / 4;
+    zero_kernel<<<dev->sms * 4, 256, 0, stream>>>(reinterpret_cast<int4 *>(acc), n16);
+    I8R_LAUNCHED();
+    return launch_decode(dev, Xq, T, K, Wq, N, acc, stream);
+}
+
+i8r_status int8_read_and_clear_device_status(int *code, cudaStream_t stream) {
+    if (!code) return I8R_EINVAL;
+    I8R_CUDA(cudaStreamSynchronize(stream));
+    int v = 0;
+    I8R_CUDA(cudaMemcpyFromSymbol(&v, i8r::g_device_status, sizeof(int)));
+    const int zero = 0;
+    I8R_CUDA(cudaMemcpyToSymbol(i8r::g_device_status, &zero, sizeof(int)));
+    *code = v;
+    return I8R_OK;
+}
+
+const char *int8_status_string(i8r_status status) {
+    switch (status) {
+        case I8R_OK: return "ok";
+        case I8R_EINVAL: return "invalid argument (null pointer, negative size, NaN or negative alpha)";
+        case I8R_EALIGN: return "misaligned pointer, or K / N not a multiple of 16";
+        case I8R_ERANGE: return "size out of range (16 <= K <= 133144, N >= 16)";
+        case I8R_EWORKSPACE: return "workspace missing or too small";
+        case I8R_ECUDA: return "CUDA error (see int8_last_cuda_error)";
+        case I8R_EDEVICE: return "a kernel reported an anomaly in the device status word";
+        case I8R_EARCH: return "current device is not sm_100 (B200)";
+    }
+    return "unknown status";
+}
+
+int int8_last_cuda_error(void) { return tl_last_cuda_error; }
+
+void int8_time_next_gemm(cudaEvent_t before, cudaEvent_t after) {
+    tl_ev_before = before;
+    tl_ev_after = after;
+}
+
+uint64_t int8_kernel_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

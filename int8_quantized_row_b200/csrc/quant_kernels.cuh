@@ -1,0 +1,274 @@
+// HBM-bound kernels of the LLM.int8() linear: weight conversion (column
+// absmax + codes), outlier-column detection, the outlier index list, and the
+// activation's row quantisation with the outlier gather.  All loads and stores
+// are 16-byte vectors; every kernel owns its outputs (no zero-initialised
+// accumulators, no atomics), so repeated runs are bit-identical.
+#pragma once
+
+#include "device_common.cuh"
+
+namespace i8r {
+
+constexpr int kStripCols = 64;        // columns owned by one block in the column scans
+constexpr int kStripThreads = 256;    // 8 warps; a warp covers 4 rows x 64 columns per step
+
+union Vec16 {
+    uint4 u;
+    __half2 h2[4];
+    __half h[8];
+};
+
+// ---------------------------------------------------------------------------
+// Weight conversion, pass 1: sW[n] = max_k |W16[k,n]| ("one normalisation
+// constant per output column", LLM.int8() abstract).  Block b owns columns
+// [64b, 64b+64) and scans every row; lane l reads the 16-byte group
+// (l % 8) of row 4w + l/8 (+ 32 i).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kStripThreads) weight_absmax_kernel(const __half *__restrict__ W16, int K, int N,
+                                                                     float *__restrict__ sW) {
+    __shared__ float part[kStripThreads / 8][kStripCols];
+    const int tid = threadIdx.x;
+    const int grp = tid & 7, sub = tid >> 3;                // 8 column groups x 32 row slots
+    const int col = blockIdx.x * kStripCols + grp * 8;
+    float m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (col < N) {
+        for (int k = sub; k < K; k += kStripThreads / 8) {
+            Vec16 v;
+            v.u = __ldg(reinterpret_cast<const uint4 *>(W16 + static_cast<size_t>(k) * N + col));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(__half2float(v.h[i])));
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[sub][grp * 8 + i] = m[i];
+    __syncthreads();
+    if (tid < kStripCols) {
+        float r = 0.0f;
+        for (int s = 0; s < kStripThreads / 8; ++s) r = fmaxf(r, part[s][tid]);
+        const int c = blockIdx.x * kStripCols + tid;
+        if (c < N) sW[c] = r;
+    }
+}
+
+// Weight conversion, pass 2: Wq[k,n] = clamp(rhaz(W16[k,n] * fl32(127/sW[n])), +-127).
+__global__ void __launch_bounds__(256) weight_codes_kernel(const __half *__restrict__ W16, int K, int N,
+                                                          const float *__restrict__ sW, int8_t *__restrict__ Wq) {
+    const size_t groups = static_cast<size_t>(K) * (N / 8);
+    const int gpr = N / 8;
+    for (size_t g = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; g < groups;
+         g += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        const size_t k = g / gpr;
+        const int n = static_cast<int>(g - k * gpr) * 8;
+        Vec16 v;
+        v.u = __ldg(reinterpret_cast<const uint4 *>(W16 + k * N + n));
+        const float4 s0 = __ldg(reinterpret_cast<const float4 *>(sW + n));
+        const float4 s1 = __ldg(reinterpret_cast<const float4 *>(sW + n + 4));
+        const float s[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t b = static_cast<uint32_t>(quant_code(__half2float(v.h[i]), recip127(s[i]))) & 0xFFu;
+            if (i < 4) lo |= b << (8 * i); else hi |= b << (8 * (i - 4));
+        }
+        *reinterpret_cast<uint2 *>(Wq + k * N + n) = make_uint2(lo, hi);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Outlier feature dimensions: mask bit k set when any |X[t,k]| >= alpha
+// (outliers defined by magnitude; "The LLM.int8() Methodology").  Optional
+// per-column hit counts for the statistics entry point.  Block b owns mask
+// words 2b and 2b+1 (columns [64b, 64b+64)).
+// ---------------------------------------------------------------------------
+template <bool kHits>
+__global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __half *__restrict__ X, int T, int K,
+                                                                    float alpha, uint32_t *__restrict__ mask,
+                                                                    int32_t *__restrict__ hits) {
+    __shared__ uint32_t flags[kStripThreads];
+    __shared__ int32_t cnt[kHits ? kStripThreads / 8 : 1][kHits ? kStripCols : 1];
+    const int tid = threadIdx.x;
+    const int grp = tid & 7, sub = tid >> 3;
+    const int col = blockIdx.x * kStripCols + grp * 8;
+    uint32_t f = 0;
+    int32_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (col < K) {
+        for (int t = sub; t < T; t += kStripThreads / 8) {
+            Vec16 v;
+            v.u = __ldg(reinterpret_cast<const uint4 *>(X + static_cast<size_t>(t) * K + col));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const bool hit = fabsf(__half2float(v.h[i])) >= alpha;
+                f |= static_cast<uint32_t>(hit) << i;
+                if (kHits) h[i] += hit;
+            }
+        }
+    }
+    flags[tid] = f;
+    if (kHits) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cnt[sub][grp * 8 + i] = h[i];
+    }
+    __syncthreads();
+    if (tid < 2) {
+        // word tid covers groups 4*tid .. 4*tid+3 (8 columns each)
+        uint32_t w = 0;
+        for (int g = 0; g < 4; ++g) {
+            uint32_t byte = 0;
+            for (int s = 0; s < kStripThreads / 8; ++s) byte |= flags[s * 8 + tid * 4 + g];
+            w |= byte << (8 * g);
+        }
+        const int word = blockIdx.x * 2 + tid;
+        if (word * 32 < K) mask[word] = w;
+    }
+    if (kHits && tid < kStripCols) {
+        int32_t r = 0;
+        for (int s = 0; s < kStripThreads / 8; ++s) r += cnt[s][tid];
+        const int c = blockIdx.x * kStripCols + tid;
+        if (c < K) hits[c] = r;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// The outlier set O as an ascending index list, by prefix popcount of the
+// mask (one block).  Also |O| and, when asked, 1 - |O|/K rounded from double.
+// ---------------------------------------------------------------------------
+constexpr int kIndexThreads = 1024;
+
+__global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint32_t *__restrict__ mask, int K,
+                                                                     int32_t *__restrict__ idx,
+                                                                     int32_t *__restrict__ count,
+                                                                     float *__restrict__ frac_8bit) {
+    __shared__ int32_t warp_sums[kIndexThreads / 32];
+    const int nwords = (K + 31) / 32;
+    const int per = (nwords + kIndexThreads - 1) / kIndexThreads;
+    const int w0 = threadIdx.x * per;
+    const int w1 = min(w0 + per, nwords);
+    int local = 0;
+    for (int w = w0; w < w1; ++w) local += __popc(mask[w]);
+    // block-wide exclusive scan of `local`
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int s = warp_sums[lane];
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, s, d);
+            if (lane >= d) s += y;
+        }
+        warp_sums[lane] = s;   // inclusive over warps
+    }
+    __syncthreads();
+    int pos = incl - local + (warp > 0 ? warp_sums[warp - 1] : 0);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t m = mask[w];
+        while (m) {
+            const int b = __ffs(m) - 1;
+            idx[pos++] = w * 32 + b;
+            m &= m - 1;
+        }
+    }
+    if (threadIdx.x == kIndexThreads - 1) {
+        const int total = warp_sums[kIndexThreads / 32 - 1];
+        *count = total;
+        if (frac_8bit) *frac_8bit = static_cast<float>(1.0 - static_cast<double>(total) / static_cast<double>(K));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Row quantisation of the non-outlier part plus the outlier gather (one
+// block per row of X):
+//   sX[t]   = max over k not in O of |X[t,k]|
+//   Xq[t,k] = 0 for k in O, else clamp(rhaz(X[t,k] * fl32(127/sX[t])), +-127)
+//   Xo[t,j] = X[t, idx[j]] for j < |O|, 0 up to the next multiple of 64
+// and, when acc32 is given, zeroes row t of the int32 accumulator [T,N] that
+// the decode-shaped GEMM adds its split-K partial sums into.
+// ---------------------------------------------------------------------------
+constexpr int kRowThreads = 256;
+constexpr int kRowRegChunks = 8;     // 16-byte chunks kept in registers (K <= 16384)
+
+__global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
+    const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ mask, const int32_t *__restrict__ idx,
+    const int32_t *__restrict__ count_ptr, float *__restrict__ sX, int8_t *__restrict__ Xq, __half *__restrict__ Xo,
+    int32_t *__restrict__ acc32, int N) {
+    __shared__ float red[kRowThreads / 32];
+    const int t = blockIdx.x;
+    const int tid = threadIdx.x;
+    const __half *xrow = X + static_cast<size_t>(t) * K;
+    const int chunks = K / 8;
+    const uint8_t *mbytes = reinterpret_cast<const uint8_t *>(mask);
+
+    Vec16 keep[kRowRegChunks];
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < kRowRegChunks; ++c) {
+        const int i = tid + c * kRowThreads;
+        if (i < chunks) {
+            keep[c].u = __ldg(reinterpret_cast<const uint4 *>(xrow) + i);
+            const uint32_t mb = mbytes[i];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (!((mb >> e) & 1u)) amax = fmaxf(amax, fabsf(__half2float(keep[c].h[e])));
+        }
+    }
+    for (int i = tid + kRowRegChunks * kRowThreads; i < chunks; i += kRowThreads) {
+        Vec16 v;
+        v.u = __ldg(reinterpret_cast<const uint4 *>(xrow) + i);
+        const uint32_t mb = mbytes[i];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (!((mb >> e) & 1u)) amax = fmaxf(amax, fabsf(__half2float(v.h[e])));
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
+    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    __syncthreads();
+    float s = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kRowThreads / 32; ++w) s = fmaxf(s, red[w]);
+    const float inv = recip127(s);
+    if (tid == 0) sX[t] = s;
+
+    int8_t *qrow = Xq + static_cast<size_t>(t) * K;
+    auto emit = [&](int i, const Vec16 &v) {
+        const uint32_t mb = mbytes[i];
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int q = ((mb >> e) & 1u) ? 0 : quant_code(__half2float(v.h[e]), inv);
+            const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
+            if (e < 4) lo |= b << (8 * e); else hi |= b << (8 * (e - 4));
+        }
+        reinterpret_cast<uint2 *>(qrow)[i] = make_uint2(lo, hi);
+    };
+#pragma unroll
+    for (int c = 0; c < kRowRegChunks; ++c) {
+        const int i = tid + c * kRowThreads;
+        if (i < chunks) emit(i, keep[c]);
+    }
+    for (int i = tid + kRowRegChunks * kRowThreads; i < chunks; i += kRowThreads) {
+        Vec16 v;
+        v.u = __ldg(reinterpret_cast<const uint4 *>(xrow) + i);
+        emit(i, v);
+    }
+
+    if (Xo) {
+        const int count = *count_ptr;
+        const int padded = (count + 63) / 64 * 64;
+        __half *orow = Xo + static_cast<size_t>(t) * K;
+        for (int j = tid; j < padded; j += kRowThreads)
+            orow[j] = j < count ? xrow[idx[j]] : __float2half_rn(0.0f);
+    }
+    if (acc32) {
+        int4 *arow = reinterpret_cast<int4 *>(acc32 + static_cast<size_t>(t) * N);
+        for (int i = tid; i < N / 4; i += kRowThreads) arow[i] = make_int4(0, 0, 0, 0);
+    }
+}
+
+}  // namespace i8r

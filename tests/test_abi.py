@@ -1,0 +1,102 @@
+"""The C-ABI library: it loads, exports every entry point the header declares,
+and rejects bad arguments on the host before touching the device (CPU only:
+no compute call is made)."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "int8row.h")
+
+
+@pytest.fixture(scope="module")
+def so():
+    from int8_quantized_row_b200 import build
+    build.build()
+    import int8_quantized_row_b200 as m
+    return m.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(int8_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("int8_quantize_weight_colwise", "int8_mixed_linear", "int8_outlier_stats",
+                     "int8_mixed_linear_workspace_size", "int8_quantize_activation", "int8_gemm_i8_s32",
+                     "int8_read_and_clear_device_status", "int8_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(so):
+    for name in declared_functions():
+        assert hasattr(so, name), name
+
+
+def test_library_exports_no_oracle_symbols(so):
+    for name in ("orc_mixed_linear", "orc_quantize_rows", "orc_int8_gemm", "orc_half_to_float"):
+        assert not hasattr(so, name)
+
+
+def test_status_strings(so):
+    for code in range(8):
+        assert len(so.int8_status_string(code)) >= 2
+    assert so.int8_status_string(99) == b"unknown status"
+
+
+def _null():
+    return ctypes.c_void_p(0)
+
+
+def _p(addr=4096):
+    return ctypes.c_void_p(addr)
+
+
+def test_host_rejects_bad_shapes_before_any_launch(so):
+    f = so.int8_mixed_linear
+    ws = so.int8_mixed_linear_workspace_size(16, 1024, 1024)
+    args = lambda T, K, N, alpha=6.0, x=_p(), y=_p(), wsp=_p(), wsb=ws: (
+        x, T, K, _p(), _p(), _p(), N, alpha, y, wsp, wsb, _null())
+    assert f(*args(16, 1000, 1024)) == 2          # K % 16
+    assert f(*args(16, 1024, 1000)) == 2          # N % 16
+    assert f(*args(16, 133152, 1024)) == 3        # K too large for exact int32 accumulation
+    assert f(*args(16, 0, 1024)) == 3
+    assert f(*args(-1, 1024, 1024)) == 1
+    assert f(*args(16, 1024, 1024, alpha=float("nan"))) == 1
+    assert f(*args(16, 1024, 1024, alpha=-1.0)) == 1
+    assert f(*args(16, 1024, 1024, x=_null())) == 1
+    assert f(*args(16, 1024, 1024, x=_p(4097))) == 2     # misaligned
+    assert f(*args(16, 1024, 1024, wsb=ws - 1)) == 4     # workspace too small
+    assert f(*args(16, 1024, 1024, wsp=_null())) == 4
+    assert f(*args(0, 1024, 1024)) == 0           # T == 0: a no-op
+
+
+def test_host_rejects_bad_weight_conversion(so):
+    f = so.int8_quantize_weight_colwise
+    assert f(_p(), 1024, 1000, _p(), _p(), _null()) == 2
+    assert f(_null(), 1024, 1024, _p(), _p(), _null()) == 1
+    assert f(_p(), 8, 1024, _p(), _p(), _null()) == 3
+
+
+def test_host_rejects_bad_stats_args(so):
+    f = so.int8_outlier_stats
+    wsb = so.int8_outlier_stats_workspace_size(1024)
+    assert f(_p(), 4, 1024, 6.0, _null(), _p(), _null(), _p(), _p(), wsb, _null()) == 1
+    assert f(_p(), 4, 1024, 6.0, _p(), _p(), _null(), _p(), _p(), wsb - 1, _null()) == 4
+
+
+def test_workspace_size_grows_with_shape(so):
+    a = so.int8_mixed_linear_workspace_size(16, 1024, 1024)
+    b = so.int8_mixed_linear_workspace_size(32, 1024, 1024)
+    c = so.int8_mixed_linear_workspace_size(256, 1024, 1024)
+    assert 0 < a < b
+    # it covers Xq (T*K) and the fp16 outlier capacity (2*T*K) at least
+    assert c >= 3 * 256 * 1024
+    assert so.int8_mixed_linear_workspace_size(-1, 1024, 1024) == 0

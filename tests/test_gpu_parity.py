@@ -1,0 +1,229 @@
+"""CUDA path vs the CPU oracle, element by element, on small and ragged shapes.
+
+Bit-exact: weight codes and scales, outlier mask / index list / count, row
+scales and codes, the gathered outlier columns, int32 accumulators.
+Tolerance on Y: relative L2 <= 1e-3 and max abs <= 2^-8 max|Y_oracle|.
+Shapes span several 128 x 256 tiles and ragged tails in T, K and N, both
+GEMM variants (decode-shaped for T <= 128, prefill above), and the
+degenerate cases of the method (no outliers, every column an outlier,
+all-zero rows and columns, T = 0).
+"""
+import numpy as np
+import pytest
+import torch
+
+import int8_quantized_row_b200 as i8
+from gpu_helpers import assert_y_close, device_status_clean, outlier_x, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+# ------------------------------------------------------------------ weights
+
+@pytest.mark.parametrize("K,N", [(16, 16), (96, 48), (1024, 272), (160, 1040), (5120, 256)])
+def test_weight_conversion_bit_exact(orc, K, N):
+    rng = np.random.default_rng(K * 7 + N)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    W[:, 3] = 0                                    # all-zero column -> sW = 0, codes 0
+    W[5, 7] = np.float16(-0.5)                     # a clear column maximum
+    Wq_o, sW_o = orc.quantize_weight_colwise(W)
+    Wq, sW = i8.int8_quantize_weight_colwise(to_dev(W))
+    torch.cuda.synchronize()
+    assert np.array_equal(to_host(sW), sW_o)
+    assert np.array_equal(to_host(Wq), Wq_o)
+    assert device_status_clean()
+
+
+def test_weight_conversion_all_fp16_codes(orc):
+    """Every finite fp16 value passes through the column quantiser."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    vals = bits[np.isfinite(bits)]
+    N = 64
+    K = (len(vals) + N - 1) // N // 16 * 16 + 16
+    W = np.zeros(K * N, np.float16)
+    W[:len(vals)] = vals
+    W = W.reshape(K, N)
+    Wq_o, sW_o = orc.quantize_weight_colwise(W)
+    Wq, sW = i8.int8_quantize_weight_colwise(to_dev(W))
+    assert np.array_equal(to_host(sW), sW_o)
+    assert np.array_equal(to_host(Wq), Wq_o)
+
+
+# ------------------------------------------------------------------ activation side
+
+ACT_CASES = [
+    # T, K, outlier columns, alpha
+    (1, 64, [5], 6.0),
+    (3, 96, [0, 95], 6.0),
+    (16, 1024, [171, 918], 6.0),
+    (127, 1024, list(range(0, 1024, 61)), 6.0),
+    (129, 1040, [], 6.0),
+    (300, 4096, [1, 2, 3, 4000], 2.5),
+    (17, 256, [], 0.0),                      # every column is an outlier
+    (17, 256, [10, 20], float("inf")),       # none is
+    (5, 12288, [7, 12287], 6.0),
+]
+
+
+@pytest.mark.parametrize("T,K,cols,alpha", ACT_CASES)
+def test_activation_quantisation_bit_exact(orc, T, K, cols, alpha):
+    rng = np.random.default_rng(T * 1000 + K)
+    X = outlier_x(rng, T, K, cols)
+    if T > 2:
+        X[2] = 0                                   # an all-zero row
+    out = i8.int8_quantize_activation(to_dev(X), alpha)
+    torch.cuda.synchronize()
+    mask_o, idx_o = orc.outlier_columns(X, alpha)
+    Xq_o, sX_o = orc.quantize_rows(X, mask_o)
+    cnt = int(to_host(out["count"])[0])
+    assert cnt == len(idx_o)
+    assert np.array_equal(to_host(out["idx"])[:cnt], idx_o)
+    words = to_host(out["mask"]).view(np.uint32)
+    bits = np.array([(words[k // 32] >> (k % 32)) & 1 for k in range(K)], bool)
+    assert np.array_equal(bits, mask_o)
+    assert np.array_equal(to_host(out["sX"])[:T], sX_o)
+    assert np.array_equal(to_host(out["Xq"])[:T], Xq_o)
+    Xo = to_host(out["Xo"])[:T]
+    pad = (cnt + 63) // 64 * 64
+    assert np.array_equal(Xo[:, :cnt].view(np.uint16), X[:, idx_o].view(np.uint16))
+    assert np.all(Xo[:, cnt:pad] == 0)
+    assert device_status_clean()
+
+
+def test_activation_t0_is_noop():
+    X = torch.zeros((0, 64), dtype=torch.float16, device="cuda")
+    out = i8.int8_quantize_activation(X, 6.0)
+    torch.cuda.synchronize()
+    assert int(out["count"][0]) == 0
+
+
+# ------------------------------------------------------------------ int8 product
+
+GEMM_CASES = [
+    # T, K, N  (T <= 128: decode-shaped kernel; T > 128: prefill kernel)
+    (1, 64, 16), (3, 96, 48), (16, 1024, 1024), (100, 160, 272), (128, 1024, 256),
+    (129, 1024, 256), (256, 512, 512), (300, 1040, 272), (513, 256, 528), (200, 12288, 64),
+    (8, 12288, 1024), (2, 4096, 12288),
+]
+
+
+@pytest.mark.parametrize("T,K,N", GEMM_CASES)
+def test_int8_gemm_bit_exact(T, K, N):
+    rng = np.random.default_rng(T + 3 * K + 7 * N)
+    A = rng.integers(-127, 128, (T, K)).astype(np.int8)
+    B = rng.integers(-127, 128, (K, N)).astype(np.int8)
+    A[0, :] = 127
+    B[:, 0] = 127                                 # the largest accumulator, K * 127^2
+    acc = i8.int8_gemm_i8_s32(to_dev(A), to_dev(B))
+    torch.cuda.synchronize()
+    ref = A.astype(np.int64) @ B.astype(np.int64)
+    assert np.array_equal(to_host(acc).astype(np.int64), ref)
+    assert device_status_clean()
+
+
+def test_int8_gemm_against_oracle_accumulators(orc):
+    rng = np.random.default_rng(99)
+    X = outlier_x(rng, 200, 1024, [3, 500])
+    W = (rng.standard_normal((1024, 384)) * 0.02).astype(np.float16)
+    Wq_o, _ = orc.quantize_weight_colwise(W)
+    mask, _ = orc.outlier_columns(X, 6.0)
+    Xq_o, _ = orc.quantize_rows(X, mask)
+    acc_o = orc.int8_gemm(Xq_o, Wq_o)
+    for T in (200, 64):
+        acc = i8.int8_gemm_i8_s32(to_dev(Xq_o[:T]), to_dev(Wq_o))
+        assert np.array_equal(to_host(acc), acc_o[:T])
+
+
+# ------------------------------------------------------------------ whole layer
+
+LINEAR_CASES = [
+    # T, K, N, outlier columns, alpha, row_prob
+    (1, 64, 16, [5], 6.0, 1.0),
+    (3, 96, 48, [], 6.0, 1.0),
+    (16, 1024, 1024, [171, 918], 6.0, 1.0),          # the single-linear shape
+    (16, 1024, 1024, [171, 918], float("inf"), 1.0),
+    (128, 1024, 272, list(range(15)), 6.0, 1.0),      # |O| = 15
+    (129, 1024, 272, list(range(16)), 6.0, 1.0),      # |O| = 16
+    (200, 1040, 528, list(range(0, 1040, 61)), 6.0, 1.0),   # |O| = 18
+    (300, 2048, 256, list(range(0, 2048, 31)), 6.0, 0.25),  # |O| = 67 > 64: two outlier blocks
+    (257, 512, 1024, [0, 511], 6.0, 0.25),
+    (64, 256, 256, [], 0.0, 1.0),                     # alpha = 0: every column in 16-bit
+    (200, 256, 256, [], 0.0, 1.0),
+    (7, 12288, 1024, [1, 100, 12000], 6.0, 1.0),
+]
+
+
+@pytest.mark.parametrize("T,K,N,cols,alpha,row_prob", LINEAR_CASES)
+def test_mixed_linear_matches_oracle(orc, T, K, N, cols, alpha, row_prob):
+    rng = np.random.default_rng(T * 31 + K + N)
+    X = outlier_x(rng, T, K, cols, row_prob=row_prob)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    Wq_o, sW_o = orc.quantize_weight_colwise(W)
+    Wq, sW = i8.int8_quantize_weight_colwise(to_dev(W))
+    assert np.array_equal(to_host(Wq), Wq_o) and np.array_equal(to_host(sW), sW_o)
+    Y = i8.int8_mixed_linear(to_dev(X), Wq, sW, to_dev(W), alpha)
+    torch.cuda.synchronize()
+    Y_o, Ypre_o, _, cnt = orc.mixed_linear(X, Wq_o, sW_o, W, alpha)
+    assert_y_close(to_host(Y), Y_o, f"T={T} K={K} N={N} |O|={cnt}")
+    assert device_status_clean()
+
+
+def test_exact_integer_case_is_exact(orc):
+    """alpha = +inf with integer inputs whose row / column absmax is 127: the
+    codes are the inputs, and Y is the exact integer product (kept within
+    +-2048, where fp16 holds every integer)."""
+    rng = np.random.default_rng(5)
+    for T in (16, 200):
+        K, N = 128, 272
+        X = rng.integers(-3, 4, (T, K)).astype(np.float16)
+        X[:, 0] = 127                                 # row absmax 127 ...
+        X[:, 1] = 0
+        W = rng.integers(-3, 4, (K, N)).astype(np.float16)
+        W[1, :] = -127                                # ... column absmax 127, and the two
+        W[0, :] = 0                                   # 127s only ever meet zeros
+        Wq, sW = i8.int8_quantize_weight_colwise(to_dev(W))
+        assert np.array_equal(to_host(Wq), W.astype(np.int8))
+        Y = i8.int8_mixed_linear(to_dev(X), Wq, sW, to_dev(W), float("inf"))
+        exact = X.astype(np.int64) @ W.astype(np.int64)
+        assert np.abs(exact).max() <= 2048
+        Y_o, _, _, _ = orc.mixed_linear(X, to_host(Wq), to_host(sW), W, float("inf"))
+        assert np.array_equal(to_host(Y).astype(np.int64), exact)
+        assert np.array_equal(Y_o.astype(np.int64), exact)
+
+
+def test_repeat_runs_are_bit_identical():
+    rng = np.random.default_rng(17)
+    for T in (16, 300):
+        X = outlier_x(rng, T, 1024, [9, 77])
+        W = (rng.standard_normal((1024, 512)) * 0.02).astype(np.float16)
+        Wq, sW = i8.int8_quantize_weight_colwise(to_dev(W))
+        Xd, Wd = to_dev(X), to_dev(W)
+        ws = i8.workspace(T, 1024, 512)
+        a = to_host(i8.int8_mixed_linear(Xd, Wq, sW, Wd, 6.0, workspace_buf=ws))
+        ws.fill_(0xAB)                              # stale workspace contents must not matter
+        b = to_host(i8.int8_mixed_linear(Xd, Wq, sW, Wd, 6.0, workspace_buf=ws))
+        assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+def test_mixed_linear_t0_is_noop():
+    Wq = torch.zeros((64, 16), dtype=torch.int8, device="cuda")
+    sW = torch.zeros(16, dtype=torch.float32, device="cuda")
+    W16 = torch.zeros((64, 16), dtype=torch.float16, device="cuda")
+    Y = i8.int8_mixed_linear(torch.zeros((0, 64), dtype=torch.float16, device="cuda"), Wq, sW, W16, 6.0)
+    assert Y.shape == (0, 16)
+
+
+# ------------------------------------------------------------------ statistics
+
+@pytest.mark.parametrize("T,K,cols,alpha", ACT_CASES[:6])
+def test_outlier_stats_match_oracle(orc, T, K, cols, alpha):
+    rng = np.random.default_rng(T + K)
+    X = outlier_x(rng, T, K, cols, row_prob=0.5)
+    count, idx, hits, frac = i8.int8_outlier_stats(to_dev(X), alpha)
+    torch.cuda.synchronize()
+    _, idx_o = orc.outlier_columns(X, alpha)
+    c = int(to_host(count)[0])
+    assert c == len(idx_o)
+    assert np.array_equal(to_host(idx)[:c], idx_o)
+    assert np.array_equal(to_host(hits), orc.outlier_hits(X, alpha))
+    assert to_host(frac)[0] == np.float32(orc.frac_8bit(c, K))

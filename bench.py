@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--rotate", type=int, default=ROTATE,
+                    help="input sets rotated between steps (default 3: operands not in L2)")
     return ap.parse_args()
 
 
@@ -124,22 +126,28 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.f.seek(0)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.f.read().splitlines():
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        return parse_clock_csv(self.f.read())
+
+
+def parse_clock_csv(text):
+    """Median SM clock, max SM clock and the throttle reasons seen, from
+    `nvidia-smi --query-gpu=<ClockSampler.FIELDS> --format=csv,noheader,nounits` lines."""
+    sm, smax, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in text.splitlines():
+        parts = [x.strip() for x in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            smax = float(parts[2])
+        except ValueError:
+            continue
+        for nm, v in zip(names, parts[5:9]):
+            if v.lower().startswith("active"):
+                reasons.add(nm)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+            "samples": len(sm), "reasons": sorted(reasons)}
 
 
 # ------------------------------------------------------------------ distributed
@@ -265,7 +273,8 @@ def run_ours(args, cfg, world, rank, local, pg):
     sets = []
     host_x = []
     X0 = W0 = None
-    for r in range(ROTATE):
+    nrot = max(1, args.rotate)
+    for r in range(nrot):
         c = dict(cfg, seed=cfg["seed"] + 1000 * rank + r)
         X, W = wl.generate(c)
         if r == 0:
@@ -286,7 +295,7 @@ def run_ours(args, cfg, world, rank, local, pg):
     ops, wbytes = work(cfg, n_out)
 
     def step(i):
-        Xd, Wq, sW, Wd = sets[i % ROTATE]
+        Xd, Wq, sW, Wd = sets[i % nrot]
         i8.int8_mixed_linear(Xd, Wq, sW, Wd, alpha, Y=Y, workspace_buf=ws)
 
     for i in range(args.warmup):
@@ -327,8 +336,8 @@ def run_ours(args, cfg, world, rank, local, pg):
     # end to end through the public API with host buffers: H2D of X, the call,
     # D2H of Y, every step, all inside the timed region
     for i in range(min(args.warmup, 3)):
-        Xd = sets[i % ROTATE][0]
-        Xd.copy_(host_x[i % ROTATE], non_blocking=True)
+        Xd = sets[i % nrot][0]
+        Xd.copy_(host_x[i % nrot], non_blocking=True)
         step(i)
         Y_host.copy_(Y, non_blocking=True)
     torch.cuda.synchronize()
@@ -337,8 +346,8 @@ def run_ours(args, cfg, world, rank, local, pg):
     torch.cuda.synchronize()
     start.record(stream)
     for i in range(e_steps):
-        Xd = sets[i % ROTATE][0]
-        Xd.copy_(host_x[i % ROTATE], non_blocking=True)
+        Xd = sets[i % nrot][0]
+        Xd.copy_(host_x[i % nrot], non_blocking=True)
         step(i)
         Y_host.copy_(Y, non_blocking=True)
     end.record(stream)
@@ -370,7 +379,8 @@ def run_ours(args, cfg, world, rank, local, pg):
         "columns, N(0,sigma) weights); no datasets or trained weights",
         "config": {"workload": args.workload, "T": T, "K": K, "N": N, "alpha": alpha, "outlier_cols": n_out,
                    "frac_8bit": frac8, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": f"{ROTATE} rotating input sets (each step's operands not in L2)"},
+                   "l2": f"{nrot} rotating input sets" + (" (each step's operands not in L2)" if nrot >= 3 else
+                                                          " (operands may be partly L2-resident)")},
         "weight_gbs": world * wbytes / (ms_step * 1e-3) / 1e9,
         "roofline": roof,
         "e2e": {"value": e_value, "unit": "TOPS", "h2d_bytes_per_step": 2 * T * K,

@@ -141,15 +141,20 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha,
  *   Xq    [T,K] int8            row codes, 0 in outlier columns
  *   Xo    [T,K] fp16 (nullable) Xo[t,j] = X[t, idx[j]] for j < |O|, 0 for
  *                               |O| <= j < 64*ceil(|O|/64); later columns untouched
+ *   workspace  at least int8_quantize_activation_workspace_size(T, K) bytes
+ *              (partial outlier masks of 128-row chunks; 0 bytes when T <= 128)
  *
  * int8_gemm_i8_s32: acc [T,N] int32 = Xq [T,K] int8 x Wq [K,N] int8, exact,
  *   by the same tensor-core kernels int8_mixed_linear uses (decode-shaped for
  *   T <= 128, prefill otherwise).  Needs workspace of at least
  *   int8_gemm_i8_s32_workspace_size(T, K, N) bytes (may be 0; pass NULL then).
  * ------------------------------------------------------------------------- */
+size_t int8_quantize_activation_workspace_size(int T, int K);
+
 i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha,
                                     uint32_t *mask, int32_t *idx, int32_t *count,
                                     float *sX, int8_t *Xq, void *Xo,
+                                    void *workspace, size_t workspace_bytes,
                                     cudaStream_t stream);
 
 size_t int8_gemm_i8_s32_workspace_size(int T, int K, int N);
@@ -165,6 +170,15 @@ i8r_status int8_gemm_i8_s32(const int8_t *Xq, int T, int K, const int8_t *Wq, in
 /* Synchronises `stream`, then returns in *code (HOST pointer) the current
  * device's status word (I8R_DEV_*) and resets it to I8R_DEV_OK. */
 i8r_status int8_read_and_clear_device_status(int *code, cudaStream_t stream);
+
+/* Failure-detection self-test: enqueues one kernel whose single thread waits
+ * on a shared-memory barrier that nothing ever completes.  The bounded wait
+ * gives up after limit_us microseconds (1 .. 1e6), records
+ * I8R_DEV_PIPELINE_TIMEOUT in the device status word and returns, exactly as
+ * a pipeline wait in the GEMM kernels would.  The GPU is not faulted and the
+ * context stays usable; read the code with
+ * int8_read_and_clear_device_status(). */
+i8r_status int8_selftest_wait_timeout(int limit_us, cudaStream_t stream);
 
 /* Static description of a status code. */
 const char *int8_status_string(i8r_status status);

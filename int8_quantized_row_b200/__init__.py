@@ -15,6 +15,7 @@ __all__ = [
     "int8_quantize_weight_colwise", "int8_mixed_linear_workspace_size", "int8_mixed_linear",
     "int8_outlier_stats_workspace_size", "int8_outlier_stats", "int8_quantize_activation",
     "int8_gemm_i8_s32", "int8_read_and_clear_device_status", "int8_status_string",
+    "int8_selftest_wait_timeout",
     "int8_time_next_gemm", "int8_kernel_launch_count", "LIB_PATH",
 ]
 
@@ -54,11 +55,15 @@ def lib():
     so.int8_outlier_stats_workspace_size.argtypes = [_I]
     so.int8_outlier_stats_workspace_size.restype = _Z
     so.int8_outlier_stats.argtypes = [_P, _I, _I, _F, _P, _P, _P, _P, _P, _Z, _P]
-    so.int8_quantize_activation.argtypes = [_P, _I, _I, _F, _P, _P, _P, _P, _P, _P, _P]
+    so.int8_quantize_activation_workspace_size.argtypes = [_I, _I]
+    so.int8_quantize_activation_workspace_size.restype = _Z
+    so.int8_quantize_activation.argtypes = [_P, _I, _I, _F, _P, _P, _P, _P, _P, _P, _P, _Z, _P]
     so.int8_gemm_i8_s32_workspace_size.argtypes = [_I, _I, _I]
     so.int8_gemm_i8_s32_workspace_size.restype = _Z
     so.int8_gemm_i8_s32.argtypes = [_P, _I, _I, _P, _I, _P, _P, _Z, _P]
     so.int8_read_and_clear_device_status.argtypes = [ctypes.POINTER(ctypes.c_int), _P]
+    so.int8_selftest_wait_timeout.argtypes = [_I, _P]
+    so.int8_selftest_wait_timeout.restype = _I
     so.int8_status_string.argtypes = [_I]
     so.int8_status_string.restype = ctypes.c_char_p
     so.int8_last_cuda_error.restype = _I
@@ -166,11 +171,14 @@ def int8_quantize_activation(X, alpha=6.0, with_xo=True, stream=None):
         Xq=torch.empty((max(T, 1), K), dtype=torch.int8, device=dev),
         Xo=torch.full((max(T, 1), K), float("nan"), dtype=torch.float16, device=dev) if with_xo else None,
     )
+    wsb = int(lib().int8_quantize_activation_workspace_size(T, K))
+    ws = torch.empty(max(1, wsb), dtype=torch.uint8, device=dev)
     _check("int8_quantize_activation", lib().int8_quantize_activation(
         _dev(X, torch.float16, "X", 2), T, K, float(alpha), _dev(out["mask"], torch.int32, "mask"),
         _dev(out["idx"], torch.int32, "idx"), _dev(out["count"], torch.int32, "count"),
         _dev(out["sX"], torch.float32, "sX"), _dev(out["Xq"], torch.int8, "Xq"),
-        _dev(out["Xo"], torch.float16, "Xo") if with_xo else None, _stream(stream)))
+        _dev(out["Xo"], torch.float16, "Xo") if with_xo else None, ctypes.c_void_p(ws.data_ptr()), wsb,
+        _stream(stream)))
     out["mask"] = out["mask"][:(K + 31) // 32]
     out["count"] = out["count"][:1]
     return out
@@ -193,6 +201,11 @@ def int8_read_and_clear_device_status(stream=None):
     _check("int8_read_and_clear_device_status", lib().int8_read_and_clear_device_status(
         ctypes.byref(code), _stream(stream)))
     return code.value
+
+
+def int8_selftest_wait_timeout(limit_us=1000, stream=None):
+    """Enqueue the bounded-wait self-test kernel (see include/int8row.h)."""
+    _check("int8_selftest_wait_timeout", lib().int8_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def int8_status_string(status):

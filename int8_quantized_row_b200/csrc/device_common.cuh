@@ -67,14 +67,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed.  Bounded: gives
 // up after kWaitLimitNs (or when another warp of the CTA raised `abort`),
 // records `code` in the device status word, raises `abort`, returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int code) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int code,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31u) == 0) {
             if (*abort) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs || it > kWaitLimitIters) {
+            if (global_timer_ns() - t0 > limit_ns || it > kWaitLimitIters) {
                 report_status(code);
                 *abort = 1;
                 return false;

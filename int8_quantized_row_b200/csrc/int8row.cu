@@ -98,15 +98,18 @@ i8r_status device_setup(const DeviceInfo **out) {
 
 // 2-D row-major tensor [rows, cols] of `elem` bytes, box [box_rows, box_cols],
 // 128-byte swizzle, zero fill out of bounds.
+// `promote` widens the L2 fetch of each box row (256 B helps when the next
+// 128 B are read soon by the same CTA; it doubles DRAM reads when they are not).
 i8r_status make_map(CUtensorMap *map, const void *base, CUtensorMapDataType type, int elem, uint64_t rows,
-                    uint64_t cols, uint32_t box_rows, uint32_t box_cols) {
+                    uint64_t cols, uint32_t box_rows, uint32_t box_cols,
+                    CUtensorMapL2promotion promote = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem)};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promote,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         tl_last_cuda_error = static_cast<int>(r);
         return I8R_ECUDA;
@@ -155,14 +158,24 @@ i8r_status check_ptr(const void *p) {
 
 // Workspace of int8_mixed_linear.
 struct Workspace {
-    size_t count, mask, idx, sX, Xq, Xo, acc32, total;
+    size_t count, mask, parts, idx, sX, Xq, Xo, acc32, total;
 };
+
+// Row chunks of the outlier scan; each writes one partial mask.
+inline int mask_parts(int T) { return T <= kMaskRowsPerPart ? 1 : (T + kMaskRowsPerPart - 1) / kMaskRowsPerPart; }
+
+// Scratch for the partial masks when there is more than one (else none).
+inline size_t parts_bytes(int T, int K) {
+    const int np = mask_parts(T);
+    return np > 1 ? align_up(static_cast<size_t>(np) * ((K + 31) / 32) * 4) : 0;
+}
 
 Workspace ws_layout(int T, int K, int N) {
     Workspace w{};
     size_t off = 0;
     w.count = off; off = align_up(off + sizeof(int32_t));
     w.mask = off;  off = align_up(off + static_cast<size_t>((K + 31) / 32) * 4);
+    w.parts = off; off += parts_bytes(T, K);
     w.idx = off;   off = align_up(off + static_cast<size_t>(K) * 4);
     w.sX = off;    off = align_up(off + static_cast<size_t>(T) * 4);
     w.Xq = off;    off = align_up(off + static_cast<size_t>(T) * K);
@@ -174,16 +187,25 @@ Workspace ws_layout(int T, int K, int N) {
 }
 
 // a1-a3 on the stream: mask, index list, row quantisation and gather.
-i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_t *mask, int32_t *idx,
-                             int32_t *count, float *sX, int8_t *Xq, __half *Xo, int32_t *acc32, int N,
-                             cudaStream_t s) {
-    outlier_mask_kernel<false><<<(K + kStripCols - 1) / kStripCols, kStripThreads, 0, s>>>(X, T, K, alpha, mask,
-                                                                                          nullptr);
+// `parts` holds mask_parts(T) partial masks when there is more than one.
+i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_t *mask, uint32_t *parts,
+                             int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, int32_t *acc32,
+                             int N, cudaStream_t s) {
+    const int np = mask_parts(T);
+    uint32_t *pm = np > 1 ? parts : mask;
+    dim3 grid((K + kStripCols - 1) / kStripCols, np);
+    outlier_mask_kernel<false><<<grid, kStripThreads, 0, s>>>(X, T, K, alpha, kMaskRowsPerPart, pm, nullptr);
     I8R_LAUNCHED();
-    outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(mask, K, idx, count, nullptr);
+    outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(pm, np, K, mask, idx, count, nullptr);
     I8R_LAUNCHED();
     if (T > 0) {
-        quantize_rows_kernel<<<T, kRowThreads, 0, s>>>(X, T, K, mask, idx, count, sX, Xq, Xo, acc32, N);
+        const int rt = row_threads(K);
+        if (rt == 64)
+            quantize_rows_kernel<64><<<T, 64, 0, s>>>(X, T, K, mask, idx, count, sX, Xq, Xo, acc32, N);
+        else if (rt == 128)
+            quantize_rows_kernel<128><<<T, 128, 0, s>>>(X, T, K, mask, idx, count, sX, Xq, Xo, acc32, N);
+        else
+            quantize_rows_kernel<256><<<T, 256, 0, s>>>(X, T, K, mask, idx, count, sX, Xq, Xo, acc32, N);
         I8R_LAUNCHED();
     }
     return I8R_OK;
@@ -258,7 +280,10 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.tmem_cols = cols;
     p.acc32 = acc32;
     CUtensorMap map_wq, map_xq;
-    I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BM));
+    // each 128-B weight row is streamed exactly once: no L2 promotion, or the
+    // neighbouring tile's half of every 256-B line is fetched and thrown away
+    I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BM,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE));
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, p.TP, decode::BK));
     const long long g = p.total_units < dev->sms ? p.total_units : dev->sms;
     const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes);
@@ -267,6 +292,19 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     I8R_LAUNCHED();
     record_after(s);
     return I8R_OK;
+}
+
+// Failure-detection self-test: one thread waits on an mbarrier that nothing
+// ever arrives on.  The bounded wait gives up after `limit_ns`, records
+// I8R_DEV_PIPELINE_TIMEOUT in the device status word and the kernel returns.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, &abort_flag, I8R_DEV_PIPELINE_TIMEOUT, limit_ns);
 }
 
 __global__ void zero_kernel(int4 *p, size_t n16) {
@@ -322,6 +360,7 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int32_t *count = reinterpret_cast<int32_t *>(ws + w.count);
     uint32_t *mask = reinterpret_cast<uint32_t *>(ws + w.mask);
+    uint32_t *parts = reinterpret_cast<uint32_t *>(ws + w.parts);
     int32_t *idx = reinterpret_cast<int32_t *>(ws + w.idx);
     float *sX = reinterpret_cast<float *>(ws + w.sX);
     int8_t *Xq = reinterpret_cast<int8_t *>(ws + w.Xq);
@@ -332,7 +371,7 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
     const __half *w16 = static_cast<const __half *>(W16);
     __half *y = static_cast<__half *>(Y);
 
-    I8R_TRY(launch_activation(x, T, K, alpha, mask, idx, count, sX, Xq, Xo, acc32, N, stream));
+    I8R_TRY(launch_activation(x, T, K, alpha, mask, parts, idx, count, sX, Xq, Xo, acc32, N, stream));
     if (!small_t)
         return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream);
 
@@ -363,18 +402,26 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha, int32_t 
     uint32_t *mask = static_cast<uint32_t *>(workspace);
     const int blocks = (K + kStripCols - 1) / kStripCols;
     const __half *x = static_cast<const __half *>(X);
+    // one row part: every block scans all rows of its columns, so the hit counts are complete
+    const int rows = T > 0 ? T : 1;
     if (col_hit_count)
-        outlier_mask_kernel<true><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, mask, col_hit_count);
+        outlier_mask_kernel<true><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, rows, mask, col_hit_count);
     else
-        outlier_mask_kernel<false><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, mask, nullptr);
+        outlier_mask_kernel<false><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, rows, mask, nullptr);
     I8R_LAUNCHED();
-    outlier_index_kernel<<<1, kIndexThreads, 0, stream>>>(mask, K, col_idx, num_outlier_cols, frac_8bit);
+    outlier_index_kernel<<<1, kIndexThreads, 0, stream>>>(mask, 1, K, mask, col_idx, num_outlier_cols, frac_8bit);
     I8R_LAUNCHED();
     return I8R_OK;
 }
 
+size_t int8_quantize_activation_workspace_size(int T, int K) {
+    if (T < 0 || K < 0) return 0;
+    return parts_bytes(T, K);
+}
+
 i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha, uint32_t *mask, int32_t *idx,
-                                    int32_t *count, float *sX, int8_t *Xq, void *Xo, cudaStream_t stream) {
+                                    int32_t *count, float *sX, int8_t *Xq, void *Xo, void *workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
     I8R_TRY(check_shape(T, K, 0, false));
     if (std::isnan(alpha) || alpha < 0.0f) return I8R_EINVAL;
     if (T > 0) {
@@ -386,10 +433,13 @@ i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha, ui
     I8R_TRY(check_ptr(mask));
     I8R_TRY(check_ptr(idx));
     if (!count) return I8R_EINVAL;
+    const size_t need = parts_bytes(T, K);
+    if (need && (!workspace || workspace_bytes < need)) return I8R_EWORKSPACE;
+    if (need && !aligned16(workspace)) return I8R_EALIGN;
     const DeviceInfo *dev = nullptr;
     I8R_TRY(device_setup(&dev));
-    return launch_activation(static_cast<const __half *>(X), T, K, alpha, mask, idx, count, sX, Xq,
-                             static_cast<__half *>(Xo), nullptr, 0, stream);
+    return launch_activation(static_cast<const __half *>(X), T, K, alpha, mask, static_cast<uint32_t *>(workspace),
+                             idx, count, sX, Xq, static_cast<__half *>(Xo), nullptr, 0, stream);
 }
 
 size_t int8_gemm_i8_s32_workspace_size(int T, int K, int N) {
@@ -442,6 +492,15 @@ const char *int8_status_string(i8r_status status) {
         case I8R_EARCH: return "current device is not sm_100 (B200)";
     }
     return "unknown status";
+}
+
+i8r_status int8_selftest_wait_timeout(int limit_us, cudaStream_t stream) {
+    if (limit_us < 1 || limit_us > 1000000) return I8R_ERANGE;
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+    wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000u);
+    I8R_LAUNCHED();
+    return I8R_OK;
 }
 
 int int8_last_cuda_error(void) { return tl_last_cuda_error; }

@@ -76,30 +76,48 @@ __global__ void __launch_bounds__(256) weight_codes_kernel(const __half *__restr
 
 // ---------------------------------------------------------------------------
 // Outlier feature dimensions: mask bit k set when any |X[t,k]| >= alpha
-// (outliers defined by magnitude; "The LLM.int8() Methodology").  Optional
-// per-column hit counts for the statistics entry point.  Block b owns mask
-// words 2b and 2b+1 (columns [64b, 64b+64)).
+// (outliers defined by magnitude; "The LLM.int8() Methodology").
+// Block (x, y) owns columns [64x, 64x+64) of rows [y*rows_per_part,
+// (y+1)*rows_per_part) and writes the two partial mask words
+// part_masks[y*words + 2x + {0,1}]; outlier_index_kernel ORs the parts.  With
+// one part (gridDim.y == 1) the partial words are the mask, and the optional
+// per-column hit counts are exact.  A thread keeps 4 row loads in flight.
 // ---------------------------------------------------------------------------
+constexpr int kMaskRowsPerPart = 128;
+
 template <bool kHits>
 __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __half *__restrict__ X, int T, int K,
-                                                                    float alpha, uint32_t *__restrict__ mask,
+                                                                    float alpha, int rows_per_part,
+                                                                    uint32_t *__restrict__ part_masks,
                                                                     int32_t *__restrict__ hits) {
     __shared__ uint32_t flags[kStripThreads];
     __shared__ int32_t cnt[kHits ? kStripThreads / 8 : 1][kHits ? kStripCols : 1];
+    constexpr int kSlots = kStripThreads / 8;          // 32 row slots per step
     const int tid = threadIdx.x;
     const int grp = tid & 7, sub = tid >> 3;
     const int col = blockIdx.x * kStripCols + grp * 8;
+    const int r0 = blockIdx.y * rows_per_part;
+    const int r1 = min(T, r0 + rows_per_part);
     uint32_t f = 0;
     int32_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (col < K) {
-        for (int t = sub; t < T; t += kStripThreads / 8) {
-            Vec16 v;
-            v.u = __ldg(reinterpret_cast<const uint4 *>(X + static_cast<size_t>(t) * K + col));
+        for (int t = r0 + sub; t < r1; t += 4 * kSlots) {
+            Vec16 v[4];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const bool hit = fabsf(__half2float(v.h[i])) >= alpha;
-                f |= static_cast<uint32_t>(hit) << i;
-                if (kHits) h[i] += hit;
+            for (int u = 0; u < 4; ++u) {
+                const int tt = t + u * kSlots;
+                v[u].u = tt < r1 ? __ldg(reinterpret_cast<const uint4 *>(X + static_cast<size_t>(tt) * K + col))
+                                 : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const bool live = t + u * kSlots < r1;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const bool hit = live && fabsf(__half2float(v[u].h[i])) >= alpha;
+                    f |= static_cast<uint32_t>(hit) << i;
+                    if (kHits) h[i] += hit;
+                }
             }
         }
     }
@@ -109,20 +127,21 @@ __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __hal
         for (int i = 0; i < 8; ++i) cnt[sub][grp * 8 + i] = h[i];
     }
     __syncthreads();
+    const int words = (K + 31) / 32;
     if (tid < 2) {
-        // word tid covers groups 4*tid .. 4*tid+3 (8 columns each)
+        // word tid covers column groups 4*tid .. 4*tid+3 (8 columns each)
         uint32_t w = 0;
         for (int g = 0; g < 4; ++g) {
             uint32_t byte = 0;
-            for (int s = 0; s < kStripThreads / 8; ++s) byte |= flags[s * 8 + tid * 4 + g];
+            for (int s = 0; s < kSlots; ++s) byte |= flags[s * 8 + tid * 4 + g];
             w |= byte << (8 * g);
         }
         const int word = blockIdx.x * 2 + tid;
-        if (word * 32 < K) mask[word] = w;
+        if (word < words) part_masks[static_cast<size_t>(blockIdx.y) * words + word] = w;
     }
     if (kHits && tid < kStripCols) {
         int32_t r = 0;
-        for (int s = 0; s < kStripThreads / 8; ++s) r += cnt[s][tid];
+        for (int s = 0; s < kSlots; ++s) r += cnt[s][tid];
         const int c = blockIdx.x * kStripCols + tid;
         if (c < K) hits[c] = r;
     }
@@ -134,8 +153,10 @@ __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __hal
 // ---------------------------------------------------------------------------
 constexpr int kIndexThreads = 1024;
 
-__global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint32_t *__restrict__ mask, int K,
-                                                                     int32_t *__restrict__ idx,
+// The mask is the OR of `nparts` partial masks (part p at part_masks + p*words);
+// it is written to `mask` (which may alias the first part when nparts == 1).
+__global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint32_t *part_masks, int nparts, int K,
+                                                                     uint32_t *mask, int32_t *__restrict__ idx,
                                                                      int32_t *__restrict__ count,
                                                                      float *__restrict__ frac_8bit) {
     __shared__ int32_t warp_sums[kIndexThreads / 32];
@@ -143,8 +164,14 @@ __global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint
     const int per = (nwords + kIndexThreads - 1) / kIndexThreads;
     const int w0 = threadIdx.x * per;
     const int w1 = min(w0 + per, nwords);
+    const bool copy = mask != part_masks;
     int local = 0;
-    for (int w = w0; w < w1; ++w) local += __popc(mask[w]);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t m = part_masks[w];
+        for (int p = 1; p < nparts; ++p) m |= part_masks[static_cast<size_t>(p) * nwords + w];
+        if (copy) mask[w] = m;          // each thread re-reads only the words it wrote
+        local += __popc(m);
+    }
     // block-wide exclusive scan of `local`
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int incl = local;
@@ -190,9 +217,13 @@ __global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint
 // and, when acc32 is given, zeroes row t of the int32 accumulator [T,N] that
 // the decode-shaped GEMM adds its split-K partial sums into.
 // ---------------------------------------------------------------------------
-constexpr int kRowThreads = 256;
-constexpr int kRowRegChunks = 8;     // 16-byte chunks kept in registers (K <= 16384)
+constexpr int kRowRegChunks = 8;     // 16-byte chunks kept in registers per thread
 
+// Threads per row: enough that a row fits the register chunks, few enough
+// that many rows are in flight per SM (the kernel is latency-bound per row).
+inline int row_threads(int K) { return K <= 4096 ? 64 : (K <= 8192 ? 128 : 256); }
+
+template <int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ mask, const int32_t *__restrict__ idx,
     const int32_t *__restrict__ count_ptr, float *__restrict__ sX, int8_t *__restrict__ Xq, __half *__restrict__ Xo,

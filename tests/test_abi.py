@@ -100,3 +100,17 @@ def test_workspace_size_grows_with_shape(so):
     # it covers Xq (T*K) and the fp16 outlier capacity (2*T*K) at least
     assert c >= 3 * 256 * 1024
     assert so.int8_mixed_linear_workspace_size(-1, 1024, 1024) == 0
+
+
+def test_selftest_rejects_bad_limit(so):
+    assert so.int8_selftest_wait_timeout(0, _null()) == 3
+    assert so.int8_selftest_wait_timeout(2000000, _null()) == 3
+
+
+def test_int8_weights_take_half_the_bytes():
+    """The stored weight (int8 codes + one fp32 scale per column) takes about
+    half the bytes of the fp16 weight (LLM.int8() abstract: inference memory
+    cut by half), approaching 1/2 as K grows."""
+    for K, N in ((5120, 20480), (12288, 49152), (49152, 12288)):
+        ratio = (K * N + 4 * N) / (2 * K * N)
+        assert 0.5 < ratio <= 0.5 + 2.0 / K + 1e-15

@@ -227,3 +227,20 @@ def test_outlier_stats_match_oracle(orc, T, K, cols, alpha):
     assert np.array_equal(to_host(idx)[:c], idx_o)
     assert np.array_equal(to_host(hits), orc.outlier_hits(X, alpha))
     assert to_host(frac)[0] == np.float32(orc.frac_8bit(c, K))
+
+
+# ------------------------------------------------------------------ failure detection
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait on a barrier nothing completes gives up after its limit and
+    records the timeout code; the GPU keeps working afterwards."""
+    assert i8.int8_read_and_clear_device_status() == 0
+    i8.int8_selftest_wait_timeout(2000)            # 2 ms
+    assert i8.int8_read_and_clear_device_status() == 1
+    assert i8.int8_read_and_clear_device_status() == 0   # read clears it
+    # the context is still usable
+    x = torch.ones(1024, device="cuda")
+    assert float(x.sum()) == 1024.0
+    acc = i8.int8_gemm_i8_s32(torch.ones((4, 64), dtype=torch.int8, device="cuda"),
+                              torch.ones((64, 16), dtype=torch.int8, device="cuda"))
+    assert int(acc.min()) == 64 and int(acc.max()) == 64

@@ -112,6 +112,33 @@ i8r_status int8_mixed_linear(const void *X, int T, int K,
                              cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * int8_mixed_linear_noalloc: the same layer, with no workspace argument and no
+ * device allocation of any kind.  The paper has no counterpart; this entry
+ * point exists for callers that cannot allocate device memory where they call
+ * the layer, such as a plugin inside an inference runtime that has reserved
+ * the GPU's memory for its own pool and passes in only input and output
+ * buffers, or a latency-critical path where cudaMalloc/cudaFree may not run
+ * because they can block or synchronise the device.
+ *
+ * Its scratch is one fixed array of int8_mixed_linear_noalloc_max_workspace()
+ * bytes (8 MiB) inside the library, which every GPU that runs the library
+ * holds until the process exits.  Shapes whose
+ * int8_mixed_linear_workspace_size(T, K, N) exceeds that are rejected with
+ * I8R_ERANGE before anything is enqueued (T <= 16 fits every 175B-sized
+ * projection).  The first call on a device looks up the array's address
+ * there, so make that first call before any stream capture.  Every call on a
+ * device shares the one array: two calls that overlap on the GPU (different
+ * streams, no ordering between them) race and corrupt each other's results.
+ * Arguments, layouts, result and errors are otherwise those of
+ * int8_mixed_linear.
+ * ------------------------------------------------------------------------- */
+size_t int8_mixed_linear_noalloc_max_workspace(void);
+
+i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K,
+                                     const int8_t *Wq, const float *sW, const void *W16, int N,
+                                     float alpha, void *Y, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Outlier statistics: the outlier feature dimensions of X and the share of
  * values that go through the 8-bit product (the pages report that share as
  * above 99.9% on large models; LLM.int8() abstract).

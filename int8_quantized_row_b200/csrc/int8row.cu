@@ -315,6 +315,38 @@ __global__ void zero_kernel(int4 *p, size_t n16) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch for int8_mixed_linear_noalloc.  Some callers cannot allocate device
+// memory where they call this layer: a plugin inside an inference runtime that
+// has reserved the GPU's memory for its own pool and hands the plugin only its
+// input and output buffers, or a latency-critical path where cudaMalloc and
+// cudaFree are not allowed because they can block or synchronise the device.
+// For them the workspace is this fixed array, reserved once per GPU when the
+// library's device code is loaded there and held until the process exits.
+// In host code `g_noalloc_scratch` names the symbol, not a device address:
+// the address each device uses is looked up with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+static constexpr size_t kNoAllocScratchBytes = 8u << 20;   // 8 MiB per GPU
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+static void *g_noalloc_scratch_ptr[kMaxDevices];           // guarded by g_dev_mutex
+
+// Device address of g_noalloc_scratch on the current device; looked up the first
+// time a device is seen, with that device current.
+static i8r_status noalloc_scratch_address(void **out) {
+    int dev = 0;
+    I8R_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return I8R_ERANGE;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!g_noalloc_scratch_ptr[dev]) {
+        void *p = nullptr;
+        I8R_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+        if (!p) return I8R_ECUDA;
+        g_noalloc_scratch_ptr[dev] = p;
+    }
+    *out = g_noalloc_scratch_ptr[dev];
+    return I8R_OK;
+}
+
 extern "C" {
 
 i8r_status int8_quantize_weight_colwise(const void *W16, int K, int N, int8_t *Wq, float *sW, cudaStream_t stream) {
@@ -380,6 +412,19 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
     decode::finalize_kernel<<<grid, decode::FIN_THREADS, 0, stream>>>(acc32, T, K, N, sX, sW, Xo, idx, count, w16, y);
     I8R_LAUNCHED();
     return I8R_OK;
+}
+
+size_t int8_mixed_linear_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
+
+i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K, const int8_t *Wq, const float *sW,
+                                     const void *W16, int N, float alpha, void *Y, cudaStream_t stream) {
+    I8R_TRY(check_shape(T, K, N, true));
+    if (ws_layout(T, K, N).total > kNoAllocScratchBytes) return I8R_ERANGE;
+    void *scratch = nullptr;
+    I8R_TRY(noalloc_scratch_address(&scratch));
+    // Nothing in the scratch has to start at zero: int8_mixed_linear writes
+    // every region before it reads it.
+    return int8_mixed_linear(X, T, K, Wq, sW, W16, N, alpha, Y, scratch, kNoAllocScratchBytes, stream);
 }
 
 size_t int8_outlier_stats_workspace_size(int K) {

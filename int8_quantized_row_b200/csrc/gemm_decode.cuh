@@ -4,13 +4,24 @@
 //
 // Swap-AB: the MMA's M = 128 columns of W (A = Wq tile, MN-major), its N = T
 // rounded up to 16 (B = Xq tile, K-major), so the weight fills the 128-lane
-// tensor-core dimension.  Split-K, stream-K style: the (column tile, k-block)
-// units are cut into gridDim.x equal contiguous ranges, one per CTA, so every
-// SM streams the same number of weight bytes.  A CTA accumulates each run of
-// k-blocks of one column tile in TMEM (double-buffered) and adds the exact
-// int32 partial sums into acc32 [T,N] (zeroed beforehand) with red.add.  A
-// second kernel applies the scales and the 16-bit outlier part.  No CTA
-// ever waits on another.
+// tensor-core dimension.  A tile is 256 columns: two 128-column MMAs per
+// k-step share one Xq tile, and every 256-byte weight line a stage touches is
+// used whole.  Split-K, stream-K style: the (tile, k-block) units are cut
+// into gridDim.x equal contiguous ranges, one per CTA, so every SM streams the
+// same number of weight bytes.  A CTA accumulates each run of k-blocks of one
+// tile in TMEM (double-buffered) and adds the exact int32 partial sums into
+// acc32 [T,N] (zeroed beforehand) with red.add.
+//
+// Finalisation without waiting: after adding its partial sums, each epilogue
+// warp bumps a counter for its (tile, 32-lane quadrant).  The warp that
+// brings the counter to the number of CTAs covering the tile knows every
+// partial sum has landed; it applies the scales and the 16-bit outlier part
+//   Y[t,n] = fp16( acc32[t,n] * sX[t] * sW[n] / 127^2 + sum_j Xo[t,j] W16[O_j,n] )
+// for its 64 columns.  No CTA ever waits on another.
+//
+// Launched as a programmatic dependent of the activation kernels: the weight
+// tiles of the first stages are requested before griddepcontrol.wait, since
+// they do not depend on the activation.
 #pragma once
 
 #include "device_common.cuh"
@@ -18,12 +29,14 @@
 namespace i8r {
 namespace decode {
 
-constexpr int BM = 128;            // columns of W per tile (MMA M)
+constexpr int BMH = 128;           // columns per MMA (MMA M)
+constexpr int BM = 2 * BMH;        // columns per tile
 constexpr int BK = 128;            // int8 K per stage (bytes)
-constexpr int A_BYTES = BM * BK;   // 16 KB
+constexpr int A_HALF = BMH * BK;   // 16 KB
+constexpr int A_BYTES = 2 * A_HALF;
 constexpr int THREADS = 192;
 constexpr int MAX_T = 128;
-constexpr int MAX_STAGES = 12;
+constexpr int MAX_STAGES = 8;
 constexpr size_t SMEM_BUDGET = 200 * 1024;
 
 struct Params {
@@ -31,8 +44,16 @@ struct Params {
     int KB, num_tiles;
     long long total_units;
     int stages, stage_bytes;
-    uint32_t tmem_cols;            // allocation (power of two >= 2*TP, >= 32); buffer b at b*tmem_cols/2
+    uint32_t tmem_cols;            // power of two >= 4*TP, >= 32; buffer b at b*tmem_cols/2
     int32_t *acc32;                // [T,N] int32, zero on entry
+    // finalisation (finalize != 0): Y from acc32 once a tile is complete
+    int finalize;
+    int32_t *counters;             // [num_tiles * 4], zero on entry
+    const float *sX, *sW;
+    const __half *Xo;              // [T,K] fp16, |O| valid columns
+    const int32_t *idx, *count;
+    const __half *W16;
+    __half *Y;
 };
 
 struct Barriers {
@@ -45,14 +66,88 @@ struct Barriers {
     int abort;
 };
 
+constexpr int FIN_SCRATCH_BYTES = 4 * 16 * 8 * 4;   // 16 x 8 floats per epilogue warp
+
 __host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes) {
-    return 1024 + static_cast<size_t>(stages) * stage_bytes + sizeof(Barriers);
+    return 1024 + static_cast<size_t>(stages) * stage_bytes + sizeof(Barriers) + FIN_SCRATCH_BYTES;
 }
 
-// The run of units [u0, u1) of CTA `cta` out of `ctas`.
-__device__ __forceinline__ void cta_range(long long total, int cta, int ctas, long long &u0, long long &u1) {
-    u0 = total * cta / ctas;
-    u1 = total * (cta + 1) / ctas;
+// CTA c of `ctas` owns units [floor(c*U/ctas), floor((c+1)*U/ctas)).
+__device__ __forceinline__ long long unit_begin(long long total, int c, int ctas) {
+    return total * c / ctas;
+}
+// The CTA whose range holds unit u.
+__device__ __forceinline__ int unit_owner(long long total, long long u, int ctas) {
+    return static_cast<int>(((u + 1) * ctas - 1) / total);
+}
+
+// Y for the columns of one finished (tile, quadrant): lane l owns columns
+// n0 + 32*quad + l and n0 + 128 + 32*quad + l.  Rows go in groups of 16 and
+// the outlier columns in chunks of 8, so each lane keeps 8 independent W16
+// loads and 16 accumulator loads in flight instead of a chain of dependent
+// loads.  `xo_s` is this warp's scratch of 16 x 8 floats.
+constexpr int FIN_ROWS = 16;
+constexpr int FIN_OUT = 8;
+
+__device__ __forceinline__ void finalize_columns(const Params &p, int tile, int quad, int lane, float *xo_s) {
+    const int count = *p.count;
+    const int nbase = tile * BM + quad * 32 + lane;
+    for (int t0 = 0; t0 < p.T; t0 += FIN_ROWS) {
+        float o[2][FIN_ROWS];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int r = 0; r < FIN_ROWS; ++r) o[h][r] = 0.0f;
+        for (int j0 = 0; j0 < count; j0 += FIN_OUT) {
+            const int kj = (lane < FIN_OUT && j0 + lane < count) ? p.idx[j0 + lane] : -1;
+            // Xo[t0 .. t0+15][j0 .. j0+7] -> scratch, one independent load per element
+            __syncwarp();
+            for (int e = lane; e < FIN_ROWS * FIN_OUT; e += 32) {
+                const int r = e / FIN_OUT, jj = e % FIN_OUT;
+                const int t = t0 + r;
+                xo_s[e] = (t < p.T && j0 + jj < count)
+                              ? __half2float(p.Xo[static_cast<size_t>(t) * p.K + j0 + jj]) : 0.0f;
+            }
+            float w[2][FIN_OUT];
+#pragma unroll
+            for (int jj = 0; jj < FIN_OUT; ++jj) {
+                const int k = __shfl_sync(0xFFFFFFFFu, kj, jj);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int n = nbase + h * BMH;
+                    w[h][jj] = (k >= 0 && n < p.N) ? __half2float(p.W16[static_cast<size_t>(k) * p.N + n]) : 0.0f;
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < FIN_ROWS; ++r)
+#pragma unroll
+                for (int jj = 0; jj < FIN_OUT; ++jj) {
+                    const float x = xo_s[r * FIN_OUT + jj];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) o[h][r] = fmaf(x, w[h][jj], o[h][r]);
+                }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int n = nbase + h * BMH;
+            if (n >= p.N) continue;
+            const float sw = p.sW[n];
+            int a[FIN_ROWS];
+#pragma unroll
+            for (int r = 0; r < FIN_ROWS; ++r)
+                a[r] = (t0 + r < p.T) ? __ldcg(p.acc32 + static_cast<size_t>(t0 + r) * p.N + n) : 0;
+#pragma unroll
+            for (int r = 0; r < FIN_ROWS; ++r) {
+                const int t = t0 + r;
+                if (t < p.T) {
+                    const float rs = p.sX[t] * (1.0f / 16129.0f);
+                    p.Y[static_cast<size_t>(t) * p.N + n] =
+                        __float2half_rn(fmaf(static_cast<float>(a[r]), rs * sw, o[h][r]));
+                }
+            }
+        }
+    }
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -88,18 +183,44 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
+    const uint32_t half_cols = p.tmem_cols / 2;
 
-    long long u0, u1;
-    cta_range(p.total_units, blockIdx.x, gridDim.x, u0, u1);
+    const long long u0 = unit_begin(p.total_units, blockIdx.x, gridDim.x);
+    const long long u1 = unit_begin(p.total_units, blockIdx.x + 1, gridDim.x);
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        int stage = 0;
-        uint32_t phase = 0;
+        const uint32_t tx = static_cast<uint32_t>(p.stage_bytes);
         int pending[MAX_STAGES];
         for (int s = 0; s < MAX_STAGES; ++s) pending[s] = -1;
-        const uint32_t tx = static_cast<uint32_t>(p.stage_bytes);
-        for (long long u = u0; u < u1; ++u) {
+        // Weight tiles of the first stages: they do not depend on the
+        // activation kernels, so they are requested before waiting on them.
+        const int pre = static_cast<int>(min(static_cast<long long>(p.stages), u1 - u0));
+        if (lane == 0) {
+            for (int i = 0; i < pre; ++i) {
+                const long long u = u0 + i;
+                const int tile = static_cast<int>(u / p.KB);
+                const int kb = static_cast<int>(u - static_cast<long long>(tile) * p.KB);
+                uint8_t *a = smem + static_cast<size_t>(i) * p.stage_bytes;
+                mbar_arrive_expect_tx(&bars->full[i], tx);   // fresh barrier: the slot is free
+                tma_load_2d(a, &map_wq, &bars->full[i], tile * BM, kb * BK);
+                tma_load_2d(a + A_HALF, &map_wq, &bars->full[i], tile * BM + BMH, kb * BK);
+                pending[i] = 0;
+            }
+        }
+        griddep_wait();
+        if (lane == 0) {
+            for (int i = 0; i < pre; ++i) {
+                const long long u = u0 + i;
+                const int kb = static_cast<int>(u % p.KB);
+                tma_load_2d(smem + static_cast<size_t>(i) * p.stage_bytes + A_BYTES, &map_xq, &bars->full[i],
+                            kb * BK, 0);
+            }
+        }
+        __syncwarp();
+        int stage = pre % p.stages;
+        uint32_t phase = (pre == p.stages) ? 1u : 0u;
+        for (long long u = u0 + pre; u < u1; ++u) {
             const int tile = static_cast<int>(u / p.KB);
             const int kb = static_cast<int>(u - static_cast<long long>(tile) * p.KB);
             if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) break;
@@ -107,6 +228,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint8_t *a = smem + static_cast<size_t>(stage) * p.stage_bytes;
                 mbar_arrive_expect_tx(&bars->full[stage], tx);
                 tma_load_2d(a, &map_wq, &bars->full[stage], tile * BM, kb * BK);
+                tma_load_2d(a + A_HALF, &map_wq, &bars->full[stage], tile * BM + BMH, kb * BK);
                 tma_load_2d(a + A_BYTES, &map_xq, &bars->full[stage], kb * BK, 0);
                 pending[stage] = static_cast<int>(phase);
             }
@@ -120,7 +242,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        const uint32_t id = idesc_i8(BM, p.TP, true, false);
+        const uint32_t id = idesc_i8(BMH, p.TP, true, false);
         int stage = 0;
         uint32_t phase = 0;
         uint32_t tph[2] = {0, 0};
@@ -132,7 +254,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int buf = seg & 1;
             if (!warp_wait(&bars->tmem_empty[buf], tph[buf] ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) break;
             tc_fence_after_sync();
-            const uint32_t d = tmem + static_cast<uint32_t>(buf) * (p.tmem_cols / 2);
+            const uint32_t d0 = tmem + static_cast<uint32_t>(buf) * half_cols;
+            const uint32_t d1 = d0 + static_cast<uint32_t>(p.TP);
             for (long long v = u; v < seg_end; ++v) {
                 if (!warp_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
                 tc_fence_after_sync();
@@ -141,9 +264,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t b = a + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk) {
-                        const uint64_t ad = smem_desc_sw128(a + kk * 32 * 128, A_BYTES, 1024);
+                        const uint32_t acc = (v != u || kk != 0) ? 1u : 0u;
                         const uint64_t bd = smem_desc_sw128(b + kk * 32, 16, 1024);
-                        mma_i8(d, ad, bd, id, (v != u || kk != 0) ? 1u : 0u);
+                        mma_i8(d0, smem_desc_sw128(a + kk * 32 * 128, A_HALF, 1024), bd, id, acc);
+                        mma_i8(d1, smem_desc_sw128(a + A_HALF + kk * 32 * 128, A_HALF, 1024), bd, id, acc);
                     }
                     mma_commit(&bars->empty[stage]);
                 }
@@ -166,32 +290,56 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;
+        griddep_wait();                                   // acc32 / counters zeroed, activation ready
         uint32_t tph[2] = {0, 0};
         int seg = 0;
         for (long long u = u0; u < u1;) {
             const int tile = static_cast<int>(u / p.KB);
-            const long long seg_end = min(u1, static_cast<long long>(tile + 1) * p.KB);
+            const long long tile_u0 = static_cast<long long>(tile) * p.KB;
+            const long long seg_end = min(u1, tile_u0 + p.KB);
             const int buf = seg & 1;
             if (!warp_wait(&bars->tmem_full[buf], tph[buf], abort, I8R_DEV_TMEM_TIMEOUT)) break;
             tc_fence_after_sync();
-            const int n = tile * BM + quad * 32 + lane;       // this thread's column of W / Y
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf) * (p.tmem_cols / 2);
-            for (int c = 0; c < p.TP; c += 16) {
-                uint32_t r[16];
-                tmem_ld16(taddr + c, r);
-                tmem_wait_ld();
-                if (n < p.N) {
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf) * half_cols;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int t = c + i;
-                        if (t < p.T && r[i] != 0u)
-                            atomicAdd(p.acc32 + static_cast<size_t>(t) * p.N + n, static_cast<int>(r[i]));
+            for (int h = 0; h < 2; ++h) {
+                const int n = tile * BM + h * BMH + quad * 32 + lane;   // this thread's column
+                for (int c = 0; c < p.TP; c += 16) {
+                    uint32_t r[16];
+                    tmem_ld16(taddr + h * p.TP + c, r);
+                    tmem_wait_ld();
+                    if (n < p.N) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int t = c + i;
+                            if (t < p.T && r[i] != 0u)
+                                atomicAdd(p.acc32 + static_cast<size_t>(t) * p.N + n, static_cast<int>(r[i]));
+                        }
                     }
                 }
             }
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
+            if (p.finalize) {
+                // publish this warp's partial sums, then count the contribution
+                __threadfence();
+                __syncwarp();
+                int last = 0;
+                if (lane == 0) {
+                    const int contributors = unit_owner(p.total_units, tile_u0 + p.KB - 1, gridDim.x) -
+                                             unit_owner(p.total_units, tile_u0, gridDim.x) + 1;
+                    const int before = atomicAdd(p.counters + tile * 4 + quad, 1);
+                    last = before == contributors - 1;
+                }
+                last = __shfl_sync(0xFFFFFFFFu, last, 0);
+                if (last) {
+                    __threadfence();
+                    float *xo_s = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + sizeof(Barriers)) +
+                                  (warp - 2) * FIN_ROWS * FIN_OUT;
+                    finalize_columns(p, tile, quad, lane, xo_s);
+                }
+            }
             tph[buf] ^= 1u;
             ++seg;
             u = seg_end;
@@ -203,69 +351,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 1) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, p.tmem_cols);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// Finaliser: Y[t,n] = fp16( acc32[t,n] * sX[t] * sW[n] / 127^2
-//                           + sum_j Xo[t,j] * W16[O_j, n] )
-// Thread = 8 consecutive columns x 8 rows; the 16-bit outlier part runs on
-// CUDA cores (|O| is small; W16's outlier rows stay in L2).
-// ---------------------------------------------------------------------------
-constexpr int FIN_THREADS = 128;
-constexpr int FIN_ROWS = 8;
-
-__global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(const int32_t *__restrict__ acc32, int T, int K, int N,
-                                                              const float *__restrict__ sX,
-                                                              const float *__restrict__ sW,
-                                                              const __half *__restrict__ Xo,
-                                                              const int32_t *__restrict__ idx,
-                                                              const int32_t *__restrict__ count_ptr,
-                                                              const __half *__restrict__ W16, __half *__restrict__ Y) {
-    const int n = (blockIdx.x * FIN_THREADS + threadIdx.x) * 8;
-    const int t0 = blockIdx.y * FIN_ROWS;
-    if (n >= N) return;
-    const int rows = min(FIN_ROWS, T - t0);
-    const int count = *count_ptr;
-    float o[FIN_ROWS][8];
-#pragma unroll
-    for (int r = 0; r < FIN_ROWS; ++r)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) o[r][e] = 0.0f;
-    for (int j = 0; j < count; ++j) {
-        Vec16 w;
-        w.u = __ldg(reinterpret_cast<const uint4 *>(W16 + static_cast<size_t>(idx[j]) * N + n));
-        float wf[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) wf[e] = __half2float(w.h[e]);
-#pragma unroll
-        for (int r = 0; r < FIN_ROWS; ++r) {
-            if (r < rows) {
-                const float x = __half2float(Xo[static_cast<size_t>(t0 + r) * K + j]);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[r][e] = fmaf(x, wf[e], o[r][e]);
-            }
-        }
-    }
-    const float4 s0 = __ldg(reinterpret_cast<const float4 *>(sW + n));
-    const float4 s1 = __ldg(reinterpret_cast<const float4 *>(sW + n + 4));
-    const float sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-    for (int r = 0; r < FIN_ROWS; ++r) {
-        if (r < rows) {
-            const int t = t0 + r;
-            const float rs = sX[t] * (1.0f / 16129.0f);
-            const int4 a0 = *reinterpret_cast<const int4 *>(acc32 + static_cast<size_t>(t) * N + n);
-            const int4 a1 = *reinterpret_cast<const int4 *>(acc32 + static_cast<size_t>(t) * N + n + 4);
-            const int a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            Vec16 out;
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                out.h2[e] = __floats2half2_rn(fmaf(static_cast<float>(a[2 * e]), rs * sw[2 * e], o[r][2 * e]),
-                                              fmaf(static_cast<float>(a[2 * e + 1]), rs * sw[2 * e + 1],
-                                                   o[r][2 * e + 1]));
-            *reinterpret_cast<uint4 *>(Y + static_cast<size_t>(t) * N + n) = out.u;
-        }
     }
 }
 

@@ -16,7 +16,10 @@
 //           W16 outlier rows are fetched by index with cp.async (all 32 lanes),
 //           then fenced into the async proxy before the stage is published
 //   warp 1  TMEM allocation + MMA issue (one lane)
-//   warps 2-5 epilogue: tcgen05.ld of their 32-lane quadrant, scale, store
+//   warps 2-5 epilogue: tcgen05.ld of their 32-lane quadrant, scale, then a
+//           32 x 32 fp16 block per chunk staged in shared memory and written
+//           by a TMA bulk store (rows/columns past T/N are clipped by TMA);
+//           sX and the tile's sW are fetched while the MMAs still run
 // Shared-memory stage: A 128 rows x 128 B (16 KB) + B 256 x 128 B (32 KB).  An
 // outlier stage reuses the same bytes: A = 128 rows x 64 fp16, B = 64 outlier
 // rows x 256 fp16 (4 MN-major chunks of 64 columns).
@@ -40,7 +43,13 @@ constexpr int B_CHUNK_F16 = 64 * OBK * 2;  // 64 columns x 64 rows of fp16 = 8 K
 constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC16_COL = 256;
-constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+// Per epilogue warp: a copy of the tile's 256 column scales and two 32 x 32
+// fp16 staging blocks for the bulk stores.
+constexpr int EPI_SW_BYTES = BN * 4;                     // 1 KB
+constexpr int EPI_STAGE_BYTES = 32 * 32 * 2;             // 2 KB
+constexpr int EPI_WARP_BYTES = EPI_SW_BYTES + 2 * EPI_STAGE_BYTES;
+constexpr int EPI_BYTES = 4 * EPI_WARP_BYTES;            // 20 KB
+constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + EPI_BYTES + 256 /*barriers*/;
 
 struct Params {
     int T, K, N;
@@ -67,16 +76,16 @@ struct Barriers {
 template <bool kS32>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_prefill_kernel(const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
-                        const __grid_constant__ CUtensorMap map_xo, const Params p) {
+                        const __grid_constant__ CUtensorMap map_xo, const __grid_constant__ CUtensorMap map_y,
+                        const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Barriers *bars = reinterpret_cast<Barriers *>(smem + STAGES * STAGE_BYTES);
+    uint8_t *epi = smem + STAGES * STAGE_BYTES;
+    Barriers *bars = reinterpret_cast<Barriers *>(epi + EPI_BYTES);
     volatile int *abort = &bars->abort;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int count = (!kS32 && p.count) ? *p.count : 0;
-    const int nob = (count + OBK - 1) / OBK;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -90,7 +99,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         fence_mbar_init();
         tma_prefetch_map(&map_xq);
         tma_prefetch_map(&map_wq);
-        if (nob) tma_prefetch_map(&map_xo);
+        if (!kS32) {
+            tma_prefetch_map(&map_xo);
+            tma_prefetch_map(&map_y);
+        }
     }
     if (warp == 1) {
         tmem_alloc(&bars->tmem_base, TMEM_COLS);
@@ -101,6 +113,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
 
+    // Launched as a programmatic dependent of the activation kernels: the
+    // weight tiles of this CTA's first stages do not depend on them and are
+    // requested first; everything else waits for them.
+    const int pre = p.KB < STAGES ? p.KB : STAGES;
+    if (warp == 0 && lane == 0) {
+        const int n0 = (blockIdx.x / p.num_m) * BN;
+        for (int i = 0; i < pre; ++i) {
+            uint8_t *b = smem + i * STAGE_BYTES + A_BYTES;
+            mbar_arrive_expect_tx(&bars->full[i], STAGE_BYTES);   // fresh barrier: the slot is free
+            tma_load_2d(b, &map_wq, &bars->full[i], n0, i * BK);
+            tma_load_2d(b + B_CHUNK_I8, &map_wq, &bars->full[i], n0 + 128, i * BK);
+        }
+    }
+    griddep_wait();
+    const int count = (!kS32 && p.count) ? *p.count : 0;
+    const int nob = (count + OBK - 1) / OBK;
+
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         int stage = 0;
@@ -109,24 +138,31 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int s = 0; s < STAGES; ++s) pending[s] = -1;
         bool ok = true;
+        bool first = true;
         for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
             const int m0 = (tile % p.num_m) * BM;
             const int n0 = (tile / p.num_m) * BN;
             for (int kb = 0; kb < p.KB; ++kb) {
-                if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
-                if (lane == 0) {
-                    uint8_t *a = smem + stage * STAGE_BYTES;
-                    uint8_t *b = a + A_BYTES;
-                    mbar_arrive_expect_tx(&bars->full[stage], STAGE_BYTES);
-                    tma_load_2d(a, &map_xq, &bars->full[stage], kb * BK, m0);
-                    tma_load_2d(b, &map_wq, &bars->full[stage], n0, kb * BK);
-                    tma_load_2d(b + B_CHUNK_I8, &map_wq, &bars->full[stage], n0 + 128, kb * BK);
+                if (first && kb < pre) {
+                    // weight half already requested above; add the activation tile
+                    if (lane == 0) tma_load_2d(smem + stage * STAGE_BYTES, &map_xq, &bars->full[stage], kb * BK, m0);
+                } else {
+                    if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
+                    if (lane == 0) {
+                        uint8_t *a = smem + stage * STAGE_BYTES;
+                        uint8_t *b = a + A_BYTES;
+                        mbar_arrive_expect_tx(&bars->full[stage], STAGE_BYTES);
+                        tma_load_2d(a, &map_xq, &bars->full[stage], kb * BK, m0);
+                        tma_load_2d(b, &map_wq, &bars->full[stage], n0, kb * BK);
+                        tma_load_2d(b + B_CHUNK_I8, &map_wq, &bars->full[stage], n0 + 128, kb * BK);
+                    }
                 }
                 __syncwarp();
 #pragma unroll
                 for (int s = 0; s < STAGES; ++s) if (s == stage) pending[s] = static_cast<int>(phase);
                 if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
+            first = false;
             for (int ob = 0; ok && ob < nob; ++ob) {
                 if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
                 uint8_t *a = smem + stage * STAGE_BYTES;
@@ -230,15 +266,33 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
         const int row = quad * 32 + lane;
+        uint8_t *mine = epi + (warp - 2) * EPI_WARP_BYTES;
+        float *sw_s = reinterpret_cast<float *>(mine);
+        uint8_t *stage_s = mine + EPI_SW_BYTES;
         uint32_t tphase = 0;
+        int chunk_seq = 0;                         // staging buffer = chunk_seq & 1
         for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-            if (!warp_wait(&bars->tmem_full, tphase, abort, I8R_DEV_TMEM_TIMEOUT)) break;
-            tc_fence_after_sync();
             const int m0 = (tile % p.num_m) * BM;
             const int n0 = (tile / p.num_m) * BN;
             const int t = m0 + row;
             const bool row_ok = t < p.T;
-            const float rs = (!kS32 && row_ok) ? p.sX[t] * (1.0f / 16129.0f) : 0.0f;
+            // fetched while this tile's MMAs still run
+            float rs = 0.0f;
+            if (!kS32) {
+                rs = row_ok ? p.sX[t] * (1.0f / 16129.0f) : 0.0f;
+                const int nl = n0 + lane * 8;
+                float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+                if (nl < p.N) {
+                    s0 = __ldg(reinterpret_cast<const float4 *>(p.sW + nl));
+                    s1 = __ldg(reinterpret_cast<const float4 *>(p.sW + nl + 4));
+                }
+                __syncwarp();                      // previous tile's readers are done
+                reinterpret_cast<float4 *>(sw_s)[lane * 2] = s0;
+                reinterpret_cast<float4 *>(sw_s)[lane * 2 + 1] = s1;
+                __syncwarp();
+            }
+            if (!warp_wait(&bars->tmem_full, tphase, abort, I8R_DEV_TMEM_TIMEOUT)) break;
+            tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
@@ -261,34 +315,41 @@ __global__ void __launch_bounds__(THREADS, 1)
                     uint4 out[4];
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
-                        float sw[8];
-                        if (nc + g * 8 < p.N) {
-                            const float4 s0 = __ldg(reinterpret_cast<const float4 *>(p.sW + nc + g * 8));
-                            const float4 s1 = __ldg(reinterpret_cast<const float4 *>(p.sW + nc + g * 8 + 4));
-                            sw[0] = s0.x; sw[1] = s0.y; sw[2] = s0.z; sw[3] = s0.w;
-                            sw[4] = s1.x; sw[5] = s1.y; sw[6] = s1.z; sw[7] = s1.w;
-                        } else {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) sw[e] = 0.0f;
-                        }
                         __half2 h[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
                             const int i0 = g * 8 + 2 * e, i1 = i0 + 1;
-                            const float y0 = fmaf(static_cast<float>(static_cast<int>(r[i0])), rs * sw[2 * e],
+                            const float y0 = fmaf(static_cast<float>(static_cast<int>(r[i0])), rs * sw_s[c * 32 + i0],
                                                   nob ? __uint_as_float(f[i0]) : 0.0f);
-                            const float y1 = fmaf(static_cast<float>(static_cast<int>(r[i1])), rs * sw[2 * e + 1],
+                            const float y1 = fmaf(static_cast<float>(static_cast<int>(r[i1])), rs * sw_s[c * 32 + i1],
                                                   nob ? __uint_as_float(f[i1]) : 0.0f);
                             h[e] = __floats2half2_rn(y0, y1);
                         }
                         out[g] = *reinterpret_cast<uint4 *>(h);
                     }
-                    if (row_ok) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(p.Y + static_cast<size_t>(t) * p.N + nc);
+                    // the staging block this chunk reuses must have been read out by its bulk store
+                    uint8_t *blk = stage_s + (chunk_seq & 1) * EPI_STAGE_BYTES;
+                    if (lane == 0) bulk_wait_group_read<1>();
+                    __syncwarp();
+                    // row `lane` of the 32 x 32 block; the 16-byte pieces are written in an
+                    // order rotated by lane/2 so that no two lanes of a quarter-warp hit the
+                    // same banks
 #pragma unroll
-                        for (int g = 0; g < 4; ++g)
-                            if (nc + g * 8 < p.N) dst[g] = out[g];
+                    for (int j = 0; j < 4; ++j) {
+                        const int g = (j + (lane >> 1)) & 3;
+                        uint4 v = out[0];
+                        if (g == 1) v = out[1];
+                        if (g == 2) v = out[2];
+                        if (g == 3) v = out[3];
+                        *reinterpret_cast<uint4 *>(blk + lane * 64 + g * 16) = v;
                     }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&map_y, blk, nc, m0 + quad * 32);
+                        bulk_commit_group();
+                    }
+                    ++chunk_seq;
                 }
             }
             tc_fence_before_sync();
@@ -296,6 +357,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (lane == 0) mbar_arrive(&bars->tmem_empty);
             tphase ^= 1u;
         }
+        if (!kS32 && lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before_sync();

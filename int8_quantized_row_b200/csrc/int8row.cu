@@ -2,12 +2,15 @@
 // The declarations and their contracts are in include/int8row.h.
 //
 // Pipeline of int8_mixed_linear (all on the caller's stream, no host sync):
-//   outlier_mask_kernel     X -> outlier column bitmask              (a1)
-//   outlier_index_kernel    bitmask -> ascending index list, |O|      (a1)
-//   quantize_rows_kernel    X -> sX, Xq (outliers zeroed), Xo gather  (a2, a3)
+//   outlier_mask_kernel     X -> outlier column bitmask (per 128-row chunk)  (a1)
+//   outlier_index_kernel    T > 128 only: OR of the chunk masks, index list  (a1)
+//   quantize_rows_kernel    X -> sX, Xq (outliers zeroed), Xo gather; for
+//                           T <= 128 it also publishes the index list         (a2, a3)
 //   T > 128:  gemm_prefill_kernel  int8 + fp16 tensor-core MMA, epilogue -> Y
-//   T <= 128: gemm_decode_kernel   split-K int8 MMA -> int32 partial sums,
-//             finalize_kernel      scales + fp16 outlier part -> Y
+//   T <= 128: gemm_decode_kernel   split-K int8 MMA -> int32 partial sums; the
+//             last contributor of each tile applies scales + fp16 outlier part
+// The GEMMs are launched as programmatic dependents of the quantiser, so their
+// prologue and first weight tiles overlap the activation kernels.
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -97,18 +100,19 @@ i8r_status device_setup(const DeviceInfo **out) {
 }
 
 // 2-D row-major tensor [rows, cols] of `elem` bytes, box [box_rows, box_cols],
-// 128-byte swizzle, zero fill out of bounds.
+// 128-byte swizzle unless asked otherwise, zero fill out of bounds on loads.
 // `promote` widens the L2 fetch of each box row (256 B helps when the next
 // 128 B are read soon by the same CTA; it doubles DRAM reads when they are not).
 i8r_status make_map(CUtensorMap *map, const void *base, CUtensorMapDataType type, int elem, uint64_t rows,
                     uint64_t cols, uint32_t box_rows, uint32_t box_cols,
-                    CUtensorMapL2promotion promote = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
+                    CUtensorMapL2promotion promote = CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem)};
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     CUresult r = g_encode(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, promote,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, promote,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         tl_last_cuda_error = static_cast<int>(r);
@@ -158,7 +162,7 @@ i8r_status check_ptr(const void *p) {
 
 // Workspace of int8_mixed_linear.
 struct Workspace {
-    size_t count, mask, parts, idx, sX, Xq, Xo, acc32, total;
+    size_t count, mask, parts, idx, sX, Xq, Xo, acc32, counters, total;
 };
 
 // Row chunks of the outlier scan; each writes one partial mask.
@@ -181,34 +185,69 @@ Workspace ws_layout(int T, int K, int N) {
     w.Xq = off;    off = align_up(off + static_cast<size_t>(T) * K);
     w.Xo = off;    off = align_up(off + static_cast<size_t>(T) * K * 2);
     w.acc32 = off;
-    if (T <= decode::MAX_T) off = align_up(off + static_cast<size_t>(T) * N * 4);
+    w.counters = off;
+    if (T <= decode::MAX_T) {
+        // split-K accumulator and per-(tile, quadrant) completion counters,
+        // contiguous so one pass of 16-byte stores clears both
+        off += static_cast<size_t>(T) * N * 4;
+        w.counters = off;
+        off = align_up(off + static_cast<size_t>((N + decode::BM - 1) / decode::BM) * 4 * 4);
+    }
     w.total = off;
     return w;
 }
 
 // a1-a3 on the stream: mask, index list, row quantisation and gather.
 // `parts` holds mask_parts(T) partial masks when there is more than one.
+// `zero` / `zero_bytes`: a region the mask kernel clears on the way (may be null).
 i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_t *mask, uint32_t *parts,
-                             int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, int32_t *acc32,
-                             int N, cudaStream_t s) {
+                             int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
+                             size_t zero_bytes, cudaStream_t s) {
     const int np = mask_parts(T);
     uint32_t *pm = np > 1 ? parts : mask;
     dim3 grid((K + kStripCols - 1) / kStripCols, np);
-    outlier_mask_kernel<false><<<grid, kStripThreads, 0, s>>>(X, T, K, alpha, kMaskRowsPerPart, pm, nullptr);
+    outlier_mask_kernel<false><<<grid, kStripThreads, 0, s>>>(X, T, K, alpha, kMaskRowsPerPart, pm, nullptr,
+                                                            static_cast<int4 *>(zero), zero_bytes / 16);
     I8R_LAUNCHED();
-    outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(pm, np, K, mask, idx, count, nullptr);
-    I8R_LAUNCHED();
+    if (np > 1) {
+        outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(pm, np, K, mask, idx, count, nullptr);
+        I8R_LAUNCHED();
+    }
+    int32_t *publish = np > 1 ? nullptr : idx;     // one part: the quantiser publishes the index list
     if (T > 0) {
         const int rt = row_threads(K);
         if (rt == 64)
-            quantize_rows_kernel<64><<<T, 64, 0, s>>>(X, T, K, mask, idx, count, sX, Xq, Xo, acc32, N);
+            quantize_rows_kernel<64><<<T, 64, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count);
         else if (rt == 128)
-            quantize_rows_kernel<128><<<T, 128, 0, s>>>(X, T, K, mask, idx, count, sX, Xq, Xo, acc32, N);
+            quantize_rows_kernel<128><<<T, 128, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count);
         else
-            quantize_rows_kernel<256><<<T, 256, 0, s>>>(X, T, K, mask, idx, count, sX, Xq, Xo, acc32, N);
+            quantize_rows_kernel<256><<<T, 256, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count);
+        I8R_LAUNCHED();
+    } else {
+        // no rows: an empty outlier set still has to be published
+        outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(mask, 1, K, mask, idx, count, nullptr);
         I8R_LAUNCHED();
     }
     return I8R_OK;
+}
+
+// Launch a GEMM kernel as a programmatic dependent of the previous kernel on
+// the stream (its prologue may overlap that kernel; it waits with
+// griddepcontrol.wait before touching the previous kernel's outputs).
+template <typename... Params, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                             Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 void record_before(cudaStream_t s) {
@@ -224,13 +263,20 @@ void record_after(cudaStream_t s) {
 i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
                           const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
                           const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
-    CUtensorMap map_xq, map_wq, map_xo;
+    CUtensorMap map_xq, map_wq, map_xo, map_y;
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, prefill::BM, prefill::BK));
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, prefill::BK, 128));
     if (Xo) {
         I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, prefill::BM, prefill::OBK));
     } else {
         map_xo = map_xq;   // unused: no 16-bit part
+    }
+    if (Y) {
+        // 32 x 32 output blocks, unswizzled 64-byte rows
+        I8R_TRY(make_map(&map_y, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, N, 32, 32,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
+    } else {
+        map_y = map_xq;    // unused: int32 output mode
     }
     prefill::Params p{};
     p.T = T;
@@ -249,22 +295,29 @@ i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half 
     p.acc_out = acc_out;
     const int grid = p.num_tiles < dev->sms ? p.num_tiles : dev->sms;
     record_before(s);
+    cudaError_t e;
     if (Y)
-        prefill::gemm_prefill_kernel<false><<<grid, prefill::THREADS, prefill::SMEM_BYTES, s>>>(map_xq, map_wq,
-                                                                                              map_xo, p);
+        e = launch_dependent(prefill::gemm_prefill_kernel<false>, dim3(grid), dim3(prefill::THREADS),
+                             prefill::SMEM_BYTES, s, map_xq, map_wq, map_xo, map_y, p);
     else
-        prefill::gemm_prefill_kernel<true><<<grid, prefill::THREADS, prefill::SMEM_BYTES, s>>>(map_xq, map_wq,
-                                                                                             map_xo, p);
+        e = launch_dependent(prefill::gemm_prefill_kernel<true>, dim3(grid), dim3(prefill::THREADS),
+                             prefill::SMEM_BYTES, s, map_xq, map_wq, map_xo, map_y, p);
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = static_cast<int>(e);
+        return I8R_ECUDA;
+    }
     I8R_LAUNCHED();
     record_after(s);
     return I8R_OK;
 }
 
 // Decode GEMM (T <= 128): int32 partial sums added into acc32, which must be
-// zero on entry.
+// zero on entry.  With `fin` (non-null) the last contributor of every tile also
+// writes Y; fin->counters must be zero on entry.
 i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, const int8_t *Wq, int N,
-                         int32_t *acc32, cudaStream_t s) {
-    decode::Params p{};
+                         int32_t *acc32, const decode::Params *fin, cudaStream_t s) {
+    decode::Params p = fin ? *fin : decode::Params{};
+    p.finalize = fin ? 1 : 0;
     p.T = T;
     p.TP = (T + 15) / 16 * 16;
     p.K = K;
@@ -276,27 +329,28 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.stages = static_cast<int>(decode::SMEM_BUDGET / p.stage_bytes);
     if (p.stages > decode::MAX_STAGES) p.stages = decode::MAX_STAGES;
     uint32_t cols = 32;
-    while (cols < static_cast<uint32_t>(2 * p.TP)) cols <<= 1;
+    while (cols < static_cast<uint32_t>(4 * p.TP)) cols <<= 1;
     p.tmem_cols = cols;
     p.acc32 = acc32;
     CUtensorMap map_wq, map_xq;
-    // each 128-B weight row is streamed exactly once: no L2 promotion, or the
-    // neighbouring tile's half of every 256-B line is fetched and thrown away
-    I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BM,
-                     CU_TENSOR_MAP_L2_PROMOTION_NONE));
+    // Two 128-column boxes per stage cover 256 contiguous bytes of every weight
+    // row, so the 256-byte L2 line is used whole.
+    I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BMH));
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, p.TP, decode::BK));
     const long long g = p.total_units < dev->sms ? p.total_units : dev->sms;
     const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes);
     record_before(s);
-    decode::gemm_decode_kernel<<<static_cast<int>(g), decode::THREADS, smem, s>>>(map_wq, map_xq, p);
+    cudaError_t e = launch_dependent(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(g)),
+                                     dim3(decode::THREADS), smem, s, map_wq, map_xq, p);
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = static_cast<int>(e);
+        return I8R_ECUDA;
+    }
     I8R_LAUNCHED();
     record_after(s);
     return I8R_OK;
 }
 
-// Failure-detection self-test: one thread waits on an mbarrier that nothing
-// ever arrives on.  The bounded wait gives up after `limit_ns`, records
-// I8R_DEV_PIPELINE_TIMEOUT in the device status word and the kernel returns.
 __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
     __shared__ uint64_t bar;
     __shared__ int abort_flag;
@@ -399,19 +453,28 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
     __half *Xo = reinterpret_cast<__half *>(ws + w.Xo);
     const bool small_t = T <= decode::MAX_T;
     int32_t *acc32 = small_t ? reinterpret_cast<int32_t *>(ws + w.acc32) : nullptr;
+    int32_t *counters = small_t ? reinterpret_cast<int32_t *>(ws + w.counters) : nullptr;
     const __half *x = static_cast<const __half *>(X);
     const __half *w16 = static_cast<const __half *>(W16);
     __half *y = static_cast<__half *>(Y);
 
-    I8R_TRY(launch_activation(x, T, K, alpha, mask, parts, idx, count, sX, Xq, Xo, acc32, N, stream));
+    // decode: the mask kernel clears the split-K accumulator and the tile counters
+    const size_t zero_bytes = small_t ? w.total - w.acc32 : 0;
+    I8R_TRY(launch_activation(x, T, K, alpha, mask, parts, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
+                              zero_bytes, stream));
     if (!small_t)
         return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream);
 
-    I8R_TRY(launch_decode(dev, Xq, T, K, Wq, N, acc32, stream));
-    dim3 grid((N / 8 + decode::FIN_THREADS - 1) / decode::FIN_THREADS, (T + decode::FIN_ROWS - 1) / decode::FIN_ROWS);
-    decode::finalize_kernel<<<grid, decode::FIN_THREADS, 0, stream>>>(acc32, T, K, N, sX, sW, Xo, idx, count, w16, y);
-    I8R_LAUNCHED();
-    return I8R_OK;
+    decode::Params fin{};
+    fin.counters = counters;
+    fin.sX = sX;
+    fin.sW = sW;
+    fin.Xo = Xo;
+    fin.idx = idx;
+    fin.count = count;
+    fin.W16 = w16;
+    fin.Y = y;
+    return launch_decode(dev, Xq, T, K, Wq, N, acc32, &fin, stream);
 }
 
 size_t int8_mixed_linear_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
@@ -450,9 +513,11 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha, int32_t 
     // one row part: every block scans all rows of its columns, so the hit counts are complete
     const int rows = T > 0 ? T : 1;
     if (col_hit_count)
-        outlier_mask_kernel<true><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, rows, mask, col_hit_count);
+        outlier_mask_kernel<true><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, rows, mask, col_hit_count,
+                                                                        nullptr, 0);
     else
-        outlier_mask_kernel<false><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, rows, mask, nullptr);
+        outlier_mask_kernel<false><<<blocks, kStripThreads, 0, stream>>>(x, T, K, alpha, rows, mask, nullptr,
+                                                                         nullptr, 0);
     I8R_LAUNCHED();
     outlier_index_kernel<<<1, kIndexThreads, 0, stream>>>(mask, 1, K, mask, col_idx, num_outlier_cols, frac_8bit);
     I8R_LAUNCHED();
@@ -511,7 +576,7 @@ i8r_status int8_gemm_i8_s32(const int8_t *Xq, int T, int K, const int8_t *Wq, in
     const size_t n16 = static_cast<size_t>(T) * N / 4;
     zero_kernel<<<dev->sms * 4, 256, 0, stream>>>(reinterpret_cast<int4 *>(acc), n16);
     I8R_LAUNCHED();
-    return launch_decode(dev, Xq, T, K, Wq, N, acc, stream);
+    return launch_decode(dev, Xq, T, K, Wq, N, acc, nullptr, stream);
 }
 
 i8r_status int8_read_and_clear_device_status(int *code, cudaStream_t stream) {

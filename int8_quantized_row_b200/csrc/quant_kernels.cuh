@@ -81,36 +81,45 @@ __global__ void __launch_bounds__(256) weight_codes_kernel(const __half *__restr
 // (y+1)*rows_per_part) and writes the two partial mask words
 // part_masks[y*words + 2x + {0,1}]; outlier_index_kernel ORs the parts.  With
 // one part (gridDim.y == 1) the partial words are the mask, and the optional
-// per-column hit counts are exact.  A thread keeps 4 row loads in flight.
+// per-column hit counts are exact.  A thread keeps 8 row loads in flight.
 // ---------------------------------------------------------------------------
-constexpr int kMaskRowsPerPart = 128;
+constexpr int kMaskRowsPerPart = 256;
 
 template <bool kHits>
 __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __half *__restrict__ X, int T, int K,
                                                                     float alpha, int rows_per_part,
                                                                     uint32_t *__restrict__ part_masks,
-                                                                    int32_t *__restrict__ hits) {
-    __shared__ uint32_t flags[kStripThreads];
-    __shared__ int32_t cnt[kHits ? kStripThreads / 8 : 1][kHits ? kStripCols : 1];
+                                                                    int32_t *__restrict__ hits, int4 *__restrict__ zero,
+                                                                    size_t zero16) {
+    constexpr int kWarps = kStripThreads / 32;
     constexpr int kSlots = kStripThreads / 8;          // 32 row slots per step
-    const int tid = threadIdx.x;
-    const int grp = tid & 7, sub = tid >> 3;
+    constexpr int kUnroll = 8;                         // row loads in flight per thread
+    __shared__ uint32_t wflags[kWarps][8];
+    __shared__ int32_t wcnt[kHits ? kWarps : 1][kHits ? kStripCols : 1];
+    if (zero) {
+        const size_t nthreads = static_cast<size_t>(gridDim.x) * gridDim.y * kStripThreads;
+        for (size_t i = (static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x) * kStripThreads + threadIdx.x;
+             i < zero16; i += nthreads)
+            zero[i] = make_int4(0, 0, 0, 0);
+    }
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int grp = tid & 7, sub = tid >> 3;           // column group (8 columns), row slot
     const int col = blockIdx.x * kStripCols + grp * 8;
     const int r0 = blockIdx.y * rows_per_part;
     const int r1 = min(T, r0 + rows_per_part);
     uint32_t f = 0;
     int32_t h[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (col < K) {
-        for (int t = r0 + sub; t < r1; t += 4 * kSlots) {
-            Vec16 v[4];
+        for (int t = r0 + sub; t < r1; t += kUnroll * kSlots) {
+            Vec16 v[kUnroll];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kUnroll; ++u) {
                 const int tt = t + u * kSlots;
                 v[u].u = tt < r1 ? __ldg(reinterpret_cast<const uint4 *>(X + static_cast<size_t>(tt) * K + col))
                                  : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < kUnroll; ++u) {
                 const bool live = t + u * kSlots < r1;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -121,19 +130,31 @@ __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __hal
             }
         }
     }
-    flags[tid] = f;
+    // lanes l, l^8, l^16, l^24 share a column group: combine them, then the warps
+    f |= __shfl_xor_sync(0xFFFFFFFFu, f, 8);
+    f |= __shfl_xor_sync(0xFFFFFFFFu, f, 16);
+    if (lane < 8) wflags[warp][lane] = f;
     if (kHits) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cnt[sub][grp * 8 + i] = h[i];
+        for (int i = 0; i < 8; ++i) {
+            h[i] += __shfl_xor_sync(0xFFFFFFFFu, h[i], 8);
+            h[i] += __shfl_xor_sync(0xFFFFFFFFu, h[i], 16);
+        }
+        if (lane < 8) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) wcnt[warp][lane * 8 + i] = h[i];
+        }
     }
     __syncthreads();
     const int words = (K + 31) / 32;
     if (tid < 2) {
-        // word tid covers column groups 4*tid .. 4*tid+3 (8 columns each)
+        // word tid covers column groups 4*tid .. 4*tid+3
         uint32_t w = 0;
+#pragma unroll
         for (int g = 0; g < 4; ++g) {
             uint32_t byte = 0;
-            for (int s = 0; s < kSlots; ++s) byte |= flags[s * 8 + tid * 4 + g];
+#pragma unroll
+            for (int ww = 0; ww < kWarps; ++ww) byte |= wflags[ww][tid * 4 + g];
             w |= byte << (8 * g);
         }
         const int word = blockIdx.x * 2 + tid;
@@ -141,7 +162,8 @@ __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __hal
     }
     if (kHits && tid < kStripCols) {
         int32_t r = 0;
-        for (int s = 0; s < kSlots; ++s) r += cnt[s][tid];
+#pragma unroll
+        for (int ww = 0; ww < kWarps; ++ww) r += wcnt[ww][tid];
         const int c = blockIdx.x * kStripCols + tid;
         if (c < K) hits[c] = r;
     }
@@ -213,9 +235,10 @@ __global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint
 // block per row of X):
 //   sX[t]   = max over k not in O of |X[t,k]|
 //   Xq[t,k] = 0 for k in O, else clamp(rhaz(X[t,k] * fl32(127/sX[t])), +-127)
-//   Xo[t,j] = X[t, idx[j]] for j < |O|, 0 up to the next multiple of 64
-// and, when acc32 is given, zeroes row t of the int32 accumulator [T,N] that
-// the decode-shaped GEMM adds its split-K partial sums into.
+//   Xo[t,j] = X[t, O_j] for j < |O|, 0 up to the next multiple of 64
+// Every block ranks the outlier columns itself from the mask (a prefix count
+// of the mask words' population counts), so no index kernel runs in between;
+// block 0 also publishes the ascending index list and |O| for the GEMM.
 // ---------------------------------------------------------------------------
 constexpr int kRowRegChunks = 8;     // 16-byte chunks kept in registers per thread
 
@@ -225,15 +248,32 @@ inline int row_threads(int K) { return K <= 4096 ? 64 : (K <= 8192 ? 128 : 256);
 
 template <int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
-    const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ mask, const int32_t *__restrict__ idx,
-    const int32_t *__restrict__ count_ptr, float *__restrict__ sX, int8_t *__restrict__ Xq, __half *__restrict__ Xo,
-    int32_t *__restrict__ acc32, int N) {
-    __shared__ float red[kRowThreads / 32];
+    const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ mask, float *__restrict__ sX,
+    int8_t *__restrict__ Xq, __half *__restrict__ Xo, int32_t *__restrict__ idx_out,
+    int32_t *__restrict__ count_out) {
+    constexpr int kWarps = kRowThreads / 32;
+    __shared__ float red[kWarps];
+    __shared__ int wsum[kWarps];
     const int t = blockIdx.x;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const __half *xrow = X + static_cast<size_t>(t) * K;
     const int chunks = K / 8;
     const uint8_t *mbytes = reinterpret_cast<const uint8_t *>(mask);
+    griddep_launch_dependents();        // the GEMM may start its prologue and weight loads
+
+    // outlier ranks: this thread's mask words [w0, w1) start at rank `base`
+    const int nwords = (K + 31) / 32;
+    const int per = (nwords + kRowThreads - 1) / kRowThreads;
+    const int w0 = min(tid * per, nwords), w1 = min(w0 + per, nwords);
+    int local = 0;
+    for (int w = w0; w < w1; ++w) local += __popc(mask[w]);
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
 
     Vec16 keep[kRowRegChunks];
     float amax = 0.0f;
@@ -258,11 +298,17 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     }
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
-    if ((tid & 31) == 0) red[tid >> 5] = amax;
+    if (lane == 0) red[warp] = amax;
     __syncthreads();
     float s = 0.0f;
+    int before = 0, total = 0;
 #pragma unroll
-    for (int w = 0; w < kRowThreads / 32; ++w) s = fmaxf(s, red[w]);
+    for (int w = 0; w < kWarps; ++w) {
+        s = fmaxf(s, red[w]);
+        if (w < warp) before += wsum[w];
+        total += wsum[w];
+    }
+    const int base = before + incl - local;
     const float inv = recip127(s);
     if (tid == 0) sX[t] = s;
 
@@ -289,16 +335,26 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
         emit(i, v);
     }
 
-    if (Xo) {
-        const int count = *count_ptr;
-        const int padded = (count + 63) / 64 * 64;
-        __half *orow = Xo + static_cast<size_t>(t) * K;
-        for (int j = tid; j < padded; j += kRowThreads)
-            orow[j] = j < count ? xrow[idx[j]] : __float2half_rn(0.0f);
-    }
-    if (acc32) {
-        int4 *arow = reinterpret_cast<int4 *>(acc32 + static_cast<size_t>(t) * N);
-        for (int i = tid; i < N / 4; i += kRowThreads) arow[i] = make_int4(0, 0, 0, 0);
+    // outlier gather (and, in block 0, the index list and its length)
+    const bool publish = blockIdx.x == 0 && idx_out != nullptr;
+    if (Xo || publish) {
+        __half *orow = Xo ? Xo + static_cast<size_t>(t) * K : nullptr;
+        int j = base;
+        for (int w = w0; w < w1; ++w) {
+            uint32_t m = mask[w];
+            while (m) {
+                const int k = w * 32 + (__ffs(m) - 1);
+                if (orow) orow[j] = xrow[k];
+                if (publish) idx_out[j] = k;
+                ++j;
+                m &= m - 1;
+            }
+        }
+        if (orow) {
+            const int padded = (total + 63) / 64 * 64;
+            for (int jj = total + tid; jj < padded; jj += kRowThreads) orow[jj] = __float2half_rn(0.0f);
+        }
+        if (publish && tid == 0) *count_out = total;
     }
 }
 

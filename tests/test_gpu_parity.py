@@ -168,6 +168,32 @@ def test_mixed_linear_matches_oracle(orc, T, K, N, cols, alpha, row_prob):
     assert device_status_clean()
 
 
+SCHEDULE_CASES = [
+    # prefill shapes with more tiles than SMs, so CTAs walk several tiles and
+    # the outlier blocks of one tile are issued inside the next one
+    (2048, 256, 4096, list(range(0, 256, 4)) + [255], 6.0),     # K < 4 k-blocks, |O| = 65: two blocks
+    (2048, 1024, 4096, list(range(0, 1024, 15)), 6.0),         # |O| = 69
+    (2200, 640, 3856, [7], 6.0),                               # ragged T, N; one outlier
+    (2048, 1024, 4096, [], 6.0),                               # no outliers: single-pass epilogue
+]
+
+
+@pytest.mark.parametrize("T,K,N,cols,alpha", SCHEDULE_CASES)
+def test_prefill_schedule_matches_oracle(orc, T, K, N, cols, alpha):
+    rng = np.random.default_rng(T + 5 * K + N)
+    X = outlier_x(rng, T, K, cols)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    Wq_o, sW_o = orc.quantize_weight_colwise(W)
+    Wq, sW = i8.int8_quantize_weight_colwise(to_dev(W))
+    Y = to_host(i8.int8_mixed_linear(to_dev(X), Wq, sW, to_dev(W), alpha))
+    rows = np.arange(0, T, 7, dtype=np.int32)              # rows are independent given O
+    Y_o, _, _, cnt = orc.mixed_linear(X, Wq_o, sW_o, W, alpha, rows=rows)
+    assert cnt == len(cols)
+    assert_y_close(Y[rows], Y_o, f"T={T} K={K} N={N} |O|={cnt}")
+    assert np.all(np.isfinite(Y.astype(np.float32)))
+    assert device_status_clean()
+
+
 def test_exact_integer_case_is_exact(orc):
     """alpha = +inf with integer inputs whose row / column absmax is 127: the
     codes are the inputs, and Y is the exact integer product (kept within

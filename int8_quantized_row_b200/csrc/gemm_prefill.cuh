@@ -242,8 +242,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int s = 0; s < STAGES; ++s)
                 if (pending[s] >= 0) mbar_wait(&bars->full[s], static_cast<uint32_t>(pending[s]), &never, 0);
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------------------ MMA issuer
+        // One thread: anything between two MMA bursts (a warp-wide shuffle, a
+        // reconvergence) delays the next burst and idles the tensor pipe.
         const uint32_t id_i8 = idesc_i8(BM, BN, false, true);
         const uint32_t id_f16 = idesc_f16(BM, BN, false, true);
         int stage = 0;
@@ -253,17 +255,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t use = static_cast<uint32_t>(it >> 1) & 1u;   // parity of this buffer's use
             const uint32_t d = tmem + static_cast<uint32_t>(buf * BN);
             if (kind == 0 && blk == 0) {
-                if (!warp_wait(&bars->acc_empty[buf], use ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
+                if (!mbar_wait(&bars->acc_empty[buf], use ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
                 tc_fence_after_sync();
             }
             if (kind == 1 && blk == 0) {
-                if (!warp_wait(&bars->acc_conv[buf], use, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
+                if (!mbar_wait(&bars->acc_conv[buf], use, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
                 tc_fence_after_sync();
             }
-            if (!warp_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+            if (!mbar_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
             tc_fence_after_sync();
             if (kind == 1) fence_proxy_async_smem();   // cp.async rows -> tensor core reads
-            if (lane == 0) {
+            {
                 const uint32_t a = smem_u32(smem + stage * STAGE_BYTES);
                 const uint32_t b = a + A_BYTES;
                 if (kind == 0) {
@@ -285,18 +287,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (kind == 0 && blk == p.KB - 1) mma_commit(&bars->acc_int_full[buf]);
                 if (kind == 1 && blk == nob - 1) mma_commit(&bars->acc_final_full[buf]);
             }
-            __syncwarp();
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             return true;
         });
         // Drain: every MMA this thread issued has completed before TMEM is freed.
-        if (lane == 0) {
-            volatile int never = 0;
-            mma_commit(&bars->drain);
-            mbar_wait(&bars->drain, 0, &never, 0);
-        }
-        __syncwarp();
-    } else {
+        volatile int never = 0;
+        mma_commit(&bars->drain);
+        mbar_wait(&bars->drain, 0, &never, 0);
+    } else if (warp >= 2) {
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
         const int row = quad * 32 + lane;
@@ -430,6 +428,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_before_sync();
     __syncthreads();
     if (warp == 1) {
+        __syncwarp();                                  // lane 0 issued the MMAs alone
         tc_fence_after_sync();
         tmem_dealloc(tmem, TMEM_COLS);
     }

@@ -6,7 +6,9 @@
 //   outlier_index_kernel    T > 128 only: OR of the chunk masks, index list  (a1)
 //   quantize_rows_kernel    X -> sX, Xq (outliers zeroed), Xo gather; for
 //                           T <= 128 it also publishes the index list         (a2, a3)
-//   T > 128:  gemm_prefill_kernel  int8 + fp16 tensor-core MMA, epilogue -> Y
+//   T > 128:  gemm_prefill_kernel (one CTA per 128 x 256 tile) or
+//             gemm_prefill_pair_kernel (CTA pairs, 256 x 256 tiles): int8 +
+//             fp16 tensor-core MMA, epilogue -> Y
 //   T <= 128: gemm_decode_kernel   split-K int8 MMA -> int32 partial sums; the
 //             last contributor of each tile applies scales + fp16 outlier part
 // The GEMMs are launched as programmatic dependents of the quantiser, so their
@@ -25,7 +27,14 @@
 #include "device_common.cuh"
 #include "quant_kernels.cuh"
 #include "gemm_prefill.cuh"
+#include "gemm_prefill_pair.cuh"
 #include "gemm_decode.cuh"
+
+// Which prefill GEMM int8_mixed_linear / int8_gemm_i32 use for T > 128:
+// 1 = CTA pairs (cta_group::2), 0 = one CTA per tile.
+#ifndef I8R_PREFILL_PAIR
+#define I8R_PREFILL_PAIR 1
+#endif
 
 namespace {
 
@@ -44,6 +53,7 @@ struct DeviceInfo {
     bool ready = false;
     bool sm100 = false;
     int sms = 0;
+    int pair_clusters = 0;     // CTA pairs of the prefill GEMM that fit the GPU at once
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -82,6 +92,25 @@ i8r_status device_setup(const DeviceInfo **out) {
             I8R_CUDA(cudaFuncSetAttribute(prefill::gemm_prefill_kernel<true>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(prefill::SMEM_BYTES)));
+            I8R_CUDA(cudaFuncSetAttribute(prefill2::gemm_prefill_pair_kernel<false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(prefill2::SMEM_BYTES)));
+            I8R_CUDA(cudaFuncSetAttribute(prefill2::gemm_prefill_pair_kernel<true>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(prefill2::SMEM_BYTES)));
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(2 * (d.sms / 2));
+            cfg.blockDim = dim3(prefill2::THREADS);
+            cfg.dynamicSmemBytes = prefill2::SMEM_BYTES;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            I8R_CUDA(cudaOccupancyMaxActiveClusters(&d.pair_clusters, prefill2::gemm_prefill_pair_kernel<false>, &cfg));
+            if (d.pair_clusters < 1) return I8R_EARCH;
             I8R_CUDA(cudaFuncSetAttribute(decode::gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(decode::SMEM_BUDGET + 4096)));
         }
@@ -234,19 +263,27 @@ i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_
 // Launch a GEMM kernel as a programmatic dependent of the previous kernel on
 // the stream (its prologue may overlap that kernel; it waits with
 // griddepcontrol.wait before touching the previous kernel's outputs).
+// `cluster_x` > 1 launches clusters of that many CTAs along x.
 template <typename... Params, typename... Args>
 cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                             Args &&...args) {
+                             int cluster_x, Args &&...args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
     cfg.numAttrs = 1;
+    if (cluster_x > 1) {
+        attr[1].id = cudaLaunchAttributeClusterDimension;
+        attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+        attr[1].val.clusterDim.y = 1;
+        attr[1].val.clusterDim.z = 1;
+        cfg.numAttrs = 2;
+    }
+    cfg.attrs = attr;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
@@ -260,9 +297,10 @@ void record_after(cudaStream_t s) {
 }
 
 // Prefill GEMM (T > 128): Y mode when Y != nullptr, else int32 accumulators.
-i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
-                          const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
-                          const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
+// One CTA per 128 x 256 tile, persistent over the tiles.
+[[maybe_unused]] i8r_status launch_prefill_single(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
+                                 const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
+                                 const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
     CUtensorMap map_xq, map_wq, map_xo, map_y;
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, prefill::BM, prefill::BK));
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, prefill::BK, 128));
@@ -298,10 +336,10 @@ i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half 
     cudaError_t e;
     if (Y)
         e = launch_dependent(prefill::gemm_prefill_kernel<false>, dim3(grid), dim3(prefill::THREADS),
-                             prefill::SMEM_BYTES, s, map_xq, map_wq, map_xo, map_y, p);
+                             prefill::SMEM_BYTES, s, 1, map_xq, map_wq, map_xo, map_y, p);
     else
         e = launch_dependent(prefill::gemm_prefill_kernel<true>, dim3(grid), dim3(prefill::THREADS),
-                             prefill::SMEM_BYTES, s, map_xq, map_wq, map_xo, map_y, p);
+                             prefill::SMEM_BYTES, s, 1, map_xq, map_wq, map_xo, map_y, p);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;
@@ -309,6 +347,69 @@ i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half 
     I8R_LAUNCHED();
     record_after(s);
     return I8R_OK;
+}
+
+// Same contract; CTA pairs (clusters of 2) compute 256 x 256 tiles with
+// cta_group::2 MMAs.
+[[maybe_unused]] i8r_status launch_prefill_pair(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
+                               const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
+                               const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
+    CUtensorMap map_xq, map_wq, map_xo, map_y;
+    I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, 128, prefill2::A_BOX_K));
+    I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, prefill2::BK, 128));
+    if (Xo) {
+        I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, 128, prefill2::OBK));
+    } else {
+        map_xo = map_xq;   // unused: no 16-bit part
+    }
+    if (Y) {
+        // 32 x 32 output blocks, unswizzled 64-byte rows
+        I8R_TRY(make_map(&map_y, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, N, 32, 32,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
+    } else {
+        map_y = map_xq;    // unused: int32 output mode
+    }
+    prefill2::Params p{};
+    p.T = T;
+    p.K = K;
+    p.N = N;
+    p.num_m = (T + prefill2::BM - 1) / prefill2::BM;
+    const int num_n = (N + prefill2::BN - 1) / prefill2::BN;
+    p.num_tiles = p.num_m * num_n;
+    p.KB = (K + prefill2::BK - 1) / prefill2::BK;
+    p.count = Y ? count : nullptr;
+    p.idx = idx;
+    p.W16 = W16;
+    p.sX = sX;
+    p.sW = sW;
+    p.Y = Y;
+    p.acc_out = acc_out;
+    const int clusters = p.num_tiles < dev->pair_clusters ? p.num_tiles : dev->pair_clusters;
+    record_before(s);
+    cudaError_t e;
+    if (Y)
+        e = launch_dependent(prefill2::gemm_prefill_pair_kernel<false>, dim3(2 * clusters), dim3(prefill2::THREADS),
+                             prefill2::SMEM_BYTES, s, 2, map_xq, map_wq, map_xo, map_y, p);
+    else
+        e = launch_dependent(prefill2::gemm_prefill_pair_kernel<true>, dim3(2 * clusters), dim3(prefill2::THREADS),
+                             prefill2::SMEM_BYTES, s, 2, map_xq, map_wq, map_xo, map_y, p);
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = static_cast<int>(e);
+        return I8R_ECUDA;
+    }
+    I8R_LAUNCHED();
+    record_after(s);
+    return I8R_OK;
+}
+
+i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
+                          const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
+                          const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
+#if I8R_PREFILL_PAIR
+    return launch_prefill_pair(dev, Xq, Xo, T, K, Wq, sW, W16, N, count, idx, sX, Y, acc_out, s);
+#else
+    return launch_prefill_single(dev, Xq, Xo, T, K, Wq, sW, W16, N, count, idx, sX, Y, acc_out, s);
+#endif
 }
 
 // Decode GEMM (T <= 128): int32 partial sums added into acc32, which must be
@@ -341,7 +442,7 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes);
     record_before(s);
     cudaError_t e = launch_dependent(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(g)),
-                                     dim3(decode::THREADS), smem, s, map_wq, map_xq, p);
+                                     dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, p);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;

@@ -175,6 +175,9 @@ SCHEDULE_CASES = [
     (2048, 1024, 4096, list(range(0, 1024, 15)), 6.0),         # |O| = 69
     (2200, 640, 3856, [7], 6.0),                               # ragged T, N; one outlier
     (2048, 1024, 4096, [], 6.0),                               # no outliers: single-pass epilogue
+    # long schedules: every stage is reused after outlier stages many times over
+    (2048, 2048, 8192, [5, 900, 2047], 6.0),                   # 3-4 tiles per CTA pair, 16 k-blocks
+    (3000, 1024, 16384, list(range(3, 1024, 15)), 6.0),        # ~10 tiles per pair, |O| = 69
 ]
 
 

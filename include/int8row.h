@@ -98,7 +98,8 @@ i8r_status int8_quantize_weight_colwise(const void *W16, int K, int N,
  *   workspace        device scratch of at least
  *                    int8_mixed_linear_workspace_size(T, K, N) bytes, 256-byte
  *                    aligned; its contents on entry are ignored and on return
- *                    are unspecified (it holds the quantised activation)
+ *                    are unspecified (it holds the quantised activation and,
+ *                    for T > 128, the W16 rows of up to 256 outlier columns)
  * Two calls that share a workspace must not overlap on the GPU.
  * T <= 128 runs the decode-shaped kernel (weight streaming, split over K);
  * larger T runs the prefill kernel (tensor-core bound).

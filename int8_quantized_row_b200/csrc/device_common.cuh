@@ -217,6 +217,19 @@ __device__ __forceinline__ void tma_load_2d_pair(void *dst, const CUtensorMap *m
         : "memory");
 }
 
+// Gather form of the CTA-pair load: four arbitrary rows r0..r3 (columns x ..
+// x + box width - 1) of a 2-D tensor whose map has a one-row box, written as
+// four consecutive box rows at dst (swizzled like a four-row tile).  Callers
+// pass in-range rows only.
+__device__ __forceinline__ void tma_gather4_pair(void *dst, const CUtensorMap *map, uint32_t bar_cluster, int x, int r0,
+                                                 int r1, int r2, int r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes.cta_group::2 "
+        "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(bar_cluster), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async
 
 // 16-byte asynchronous copy global -> shared; bytes beyond src_bytes are zero.

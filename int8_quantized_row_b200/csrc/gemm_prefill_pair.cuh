@@ -27,9 +27,8 @@
 //                  on it.  Every stage use goes through full[s], so its phase
 //                  flips exactly once per trip round the ring.  (The peer's
 //                  bytes need no arrival of their own, so the hot path has no
-//                  cluster-scope fence.)
-//   oready[s]      leader's, outlier stages only: the peer arrives (release,
-//                  cluster scope) once its cp.async-gathered W16 rows are fenced
+//                  cluster-scope fence.)  Outlier stages are all TMA as well:
+//                  the W16 rows of the outlier columns arrive as one-row loads.
 //   empty[s]       each CTA's own; the leader's MMA commit arrives on both
 //   acc_int_full, acc_final_full  each CTA's own; committed to both
 //   acc_conv, acc_empty           leader's, 8 arrivals (4 epilogue warps x 2)
@@ -69,16 +68,15 @@ struct Params {
     int num_m, num_tiles, KB;      // tiles of 256 x 256
     const int32_t *count;
     const int32_t *idx;
-    const __half *W16;
     const float *sX;
     const float *sW;
     __half *Y;
     int32_t *acc_out;
+    int o_rows;                    // outlier rows compacted into the W16o map (multiple of 64)
 };
 
 struct Barriers {
     uint64_t full[STAGES];
-    uint64_t oready[STAGES];
     uint64_t empty[STAGES];
     uint64_t acc_int_full[2];
     uint64_t acc_conv[2];
@@ -87,7 +85,9 @@ struct Barriers {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    int orow[OBK];                 // W16 row of each outlier of the stage being loaded
 };
+static_assert(sizeof(Barriers) <= 512, "barrier block outgrew its shared-memory reserve");
 
 // Same stage order for the producer (both CTAs) and the MMA warp (leader).
 template <typename Visit>
@@ -116,8 +116,9 @@ __device__ __forceinline__ bool walk_schedule(const Params &p, int nob, int clus
 template <bool kS32>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap map_xq, const __grid_constant__ CUtensorMap map_wq,
-                             const __grid_constant__ CUtensorMap map_xo, const __grid_constant__ CUtensorMap map_y,
-                             const Params p) {
+                             const __grid_constant__ CUtensorMap map_xo, const __grid_constant__ CUtensorMap map_w16,
+                             const __grid_constant__ CUtensorMap map_w16x4, const __grid_constant__ CUtensorMap map_w16o,
+                             const __grid_constant__ CUtensorMap map_y, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *epi = smem + STAGES * STAGE_BYTES;
@@ -134,7 +135,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&bars->full[s], 1);
-            mbar_init(&bars->oready[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -150,6 +150,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma_prefetch_map(&map_wq);
         if (!kS32) {
             tma_prefetch_map(&map_xo);
+            tma_prefetch_map(&map_w16);
+            tma_prefetch_map(&map_w16x4);
+            tma_prefetch_map(&map_w16o);
             tma_prefetch_map(&map_y);
         }
     }
@@ -164,7 +167,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     // shared::cluster addresses of the leader's barriers
     const uint32_t lead_full = mapa_shared(smem_u32(&bars->full[0]), 0);
-    const uint32_t lead_oready = mapa_shared(smem_u32(&bars->oready[0]), 0);
     const uint32_t lead_acc_conv = mapa_shared(smem_u32(&bars->acc_conv[0]), 0);
     const uint32_t lead_acc_empty = mapa_shared(smem_u32(&bars->acc_empty[0]), 0);
 
@@ -209,32 +211,53 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tma_load_2d_pair(a + A_BYTES, &map_wq, lead_full + 8u * stage, n0, blk * BK);
                     }
                 } else {
-                    // this CTA's 128 columns of the W16 rows of outliers blk*64 .. +63
-                    const uint32_t b = smem_u32(a + A_BYTES);
-                    const int rows = min(OBK, (count - blk * OBK + 15) / 16 * 16);
-                    const int g0 = blk * OBK + lane, g1 = blk * OBK + 32 + lane;
-                    const int k0 = g0 < count ? p.idx[g0] : -1;
-                    const int k1 = g1 < count ? p.idx[g1] : -1;
-                    // 16 lanes cover one row of 128 columns; two rows per step
-                    const int half = lane >> 4, l16 = lane & 15;
-                    const int n = n0 + l16 * 8;
-                    const uint32_t chunk = b + (l16 >> 3) * B_CHUNK_F16;
-                    const uint32_t unit = l16 & 7;
-                    for (int j2 = 0; j2 < rows; j2 += 2) {
-                        const int j = j2 + half;
-                        const int ksrc = __shfl_sync(0xFFFFFFFFu, j < 32 ? k0 : k1, j & 31);
-                        const bool have = (ksrc >= 0) && (n < p.N) && (j < rows);
-                        const __half *src = have ? p.W16 + static_cast<size_t>(ksrc) * p.N + n : p.W16;
-                        const uint32_t dst = chunk + j * 128 + ((unit ^ (j & 7)) << 4);   // 128-B swizzle
-                        if (j < rows) cp_async_16(dst, src, have ? 16u : 0u);
-                    }
-                    cp_async_wait_all();
-                    fence_proxy_async_smem();
+                    // The Xo tile, then this CTA's 128 columns (two 64-column
+                    // pieces) of the W16 rows of outliers blk*64 .. .  Blocks
+                    // inside the compacted rows (W16o, zero past |O|) are two
+                    // 64 x 64 boxes.  Past them, the MMAs read round16(rows left)
+                    // rows, in groups of four:
+                    //   four outliers     one gather of the four rows
+                    //   no outlier        a four-row box at row K: out of range,
+                    //                     so the TMA writes zeros
+                    //   some outliers     one-row loads, row K for the padding
+                    // The lanes fetch the row indices together; one lane issues
+                    // the loads (a TMA load takes its operands from uniform
+                    // registers, so per-lane operands are issued a lane at a time,
+                    // and each load has a fixed cost: the fewer, the better).
+                    const int left = count - blk * OBK;
+                    const bool compact = blk * OBK + OBK <= p.o_rows;
+                    const int rows = compact ? OBK : min(OBK, (left + 15) / 16 * 16);
+                    if (!compact)
+                        for (int j = lane; j < rows; j += 32) bars->orow[j] = j < left ? p.idx[blk * OBK + j] : p.K;
                     __syncwarp();
-                    if (lane == 0) {
-                        if (leader) mbar_arrive_expect_tx(&bars->full[stage], 2 * XO_BYTES);
-                        else mbar_arrive_cluster(lead_oready + 8u * stage);
-                        tma_load_2d_pair(a, &map_xo, lead_full + 8u * stage, blk * OBK, m0);
+                    if (lane == 0 && compact) {
+                        if (leader)
+                            mbar_arrive_expect_tx(&bars->full[stage], 2u * static_cast<uint32_t>(XO_BYTES + OBK * 256));
+                        const uint32_t fb = lead_full + 8u * stage;
+                        tma_load_2d_pair(a, &map_xo, fb, blk * OBK, m0);
+                        tma_load_2d_pair(a + A_BYTES, &map_w16o, fb, n0, blk * OBK);
+                        tma_load_2d_pair(a + A_BYTES + B_CHUNK_F16, &map_w16o, fb, n0 + 64, blk * OBK);
+                    } else if (lane == 0) {
+                        if (leader)
+                            mbar_arrive_expect_tx(&bars->full[stage], 2u * static_cast<uint32_t>(XO_BYTES + rows * 256));
+                        const uint32_t fb = lead_full + 8u * stage;
+                        tma_load_2d_pair(a, &map_xo, fb, blk * OBK, m0);
+                        uint8_t *b = a + A_BYTES;
+                        for (int j = 0; j < rows; j += 4) {
+                            for (int c = 0; c < 2; ++c) {
+                                uint8_t *dst = b + c * B_CHUNK_F16 + j * 128;
+                                const int x = n0 + 64 * c;
+                                if (j + 4 <= left) {
+                                    tma_gather4_pair(dst, &map_w16, fb, x, bars->orow[j], bars->orow[j + 1],
+                                                     bars->orow[j + 2], bars->orow[j + 3]);
+                                } else if (j >= left) {
+                                    tma_load_2d_pair(dst, &map_w16x4, fb, x, p.K);
+                                } else {
+                                    for (int e = 0; e < 4; ++e)
+                                        tma_load_2d_pair(dst + e * 128, &map_w16, fb, x, bars->orow[j + e]);
+                                }
+                            }
+                        }
                     }
                 }
             }
@@ -270,7 +293,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t own_final_c = mapa_shared(own_final, 0);
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t ophase = 0;                      // per-stage parity bits of oready
             walk_schedule(p, nob, cluster_id, clusters, [&](int kind, int, int it, int blk) -> bool {
                 const int buf = it & 1;
                 const uint32_t use = static_cast<uint32_t>(it >> 1) & 1u;
@@ -284,13 +306,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tc_fence_after_sync();
                 }
                 if (!mbar_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
-                if (kind == 1) {
-                    // the peer's cp.async-gathered W16 rows: cluster-scope acquire
-                    if (!mbar_wait_cluster(&bars->oready[stage], (ophase >> stage) & 1u, abort,
-                                           I8R_DEV_PIPELINE_TIMEOUT))
-                        return false;
-                    ophase ^= 1u << stage;
-                }
                 tc_fence_after_sync();
                 {
                     const uint32_t a = smem_u32(smem + stage * STAGE_BYTES);

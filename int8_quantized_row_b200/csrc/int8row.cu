@@ -13,6 +13,7 @@
 //             last contributor of each tile applies scales + fp16 outlier part
 // The GEMMs are launched as programmatic dependents of the quantiser, so their
 // prologue and first weight tiles overlap the activation kernels.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdio>
@@ -191,8 +192,11 @@ i8r_status check_ptr(const void *p) {
 
 // Workspace of int8_mixed_linear.
 struct Workspace {
-    size_t count, mask, parts, idx, sX, Xq, Xo, acc32, counters, total;
+    size_t count, mask, parts, idx, sX, Xq, Xo, W16o, acc32, counters, total;
 };
+
+// Rows of the compacted outlier weight rows kept for the prefill GEMM.
+inline int compact_rows(int K) { return std::min((K + 63) / 64 * 64, kCompactOutlierRows); }
 
 // Row chunks of the outlier scan; each writes one partial mask.
 inline int mask_parts(int T) { return T <= kMaskRowsPerPart ? 1 : (T + kMaskRowsPerPart - 1) / kMaskRowsPerPart; }
@@ -213,6 +217,8 @@ Workspace ws_layout(int T, int K, int N) {
     w.sX = off;    off = align_up(off + static_cast<size_t>(T) * 4);
     w.Xq = off;    off = align_up(off + static_cast<size_t>(T) * K);
     w.Xo = off;    off = align_up(off + static_cast<size_t>(T) * K * 2);
+    w.W16o = off;
+    if (T > decode::MAX_T) off = align_up(off + static_cast<size_t>(compact_rows(K)) * N * 2);
     w.acc32 = off;
     w.counters = off;
     if (T <= decode::MAX_T) {
@@ -229,9 +235,12 @@ Workspace ws_layout(int T, int K, int N) {
 // a1-a3 on the stream: mask, index list, row quantisation and gather.
 // `parts` holds mask_parts(T) partial masks when there is more than one.
 // `zero` / `zero_bytes`: a region the mask kernel clears on the way (may be null).
+// With W16o, the quantiser's launch also compacts the W16 rows of the first
+// compact_rows(K) outlier columns into W16o ([compact_rows(K), N]).
 i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_t *mask, uint32_t *parts,
                              int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
-                             size_t zero_bytes, cudaStream_t s) {
+                             size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
+                             __half *W16o = nullptr) {
     const int np = mask_parts(T);
     uint32_t *pm = np > 1 ? parts : mask;
     dim3 grid((K + kStripCols - 1) / kStripCols, np);
@@ -245,12 +254,17 @@ i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_
     int32_t *publish = np > 1 ? nullptr : idx;     // one part: the quantiser publishes the index list
     if (T > 0) {
         const int rt = row_threads(K);
+        const int o_rows = W16o ? compact_rows(K) : 0;
+        const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
         if (rt == 64)
-            quantize_rows_kernel<64><<<T, 64, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count);
+            quantize_rows_kernel<64><<<T + G, 64, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count, W16, N, W16o,
+                                                          o_rows, G);
         else if (rt == 128)
-            quantize_rows_kernel<128><<<T, 128, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count);
+            quantize_rows_kernel<128><<<T + G, 128, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count, W16, N,
+                                                            W16o, o_rows, G);
         else
-            quantize_rows_kernel<256><<<T, 256, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count);
+            quantize_rows_kernel<256><<<T + G, 256, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count, W16, N,
+                                                            W16o, o_rows, G);
         I8R_LAUNCHED();
     } else {
         // no rows: an empty outlier set still has to be published
@@ -353,14 +367,28 @@ void record_after(cudaStream_t s) {
 // cta_group::2 MMAs.
 [[maybe_unused]] i8r_status launch_prefill_pair(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
                                const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
-                               const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
-    CUtensorMap map_xq, map_wq, map_xo, map_y;
+                               const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s,
+                               const __half *W16o) {
+    CUtensorMap map_xq, map_wq, map_xo, map_w16, map_w16x4, map_w16o, map_y;
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, 128, prefill2::A_BOX_K));
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, prefill2::BK, 128));
     if (Xo) {
         I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, 128, prefill2::OBK));
+        // 64-column pieces of W16 rows: one-row box (also the gather map), and
+        // a four-row box for the zero padding
+        I8R_TRY(make_map(&map_w16, W16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, N, 1, 64));
+        I8R_TRY(make_map(&map_w16x4, W16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, N, 4, 64));
     } else {
         map_xo = map_xq;   // unused: no 16-bit part
+        map_w16 = map_xq;
+        map_w16x4 = map_xq;
+    }
+    // compacted outlier rows: 64 x 64 boxes
+    const int o_rows = (Xo && W16o) ? compact_rows(K) : 0;
+    if (o_rows > 0) {
+        I8R_TRY(make_map(&map_w16o, W16o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, o_rows, N, 64, 64));
+    } else {
+        map_w16o = map_xq;
     }
     if (Y) {
         // 32 x 32 output blocks, unswizzled 64-byte rows
@@ -379,20 +407,20 @@ void record_after(cudaStream_t s) {
     p.KB = (K + prefill2::BK - 1) / prefill2::BK;
     p.count = Y ? count : nullptr;
     p.idx = idx;
-    p.W16 = W16;
     p.sX = sX;
     p.sW = sW;
     p.Y = Y;
     p.acc_out = acc_out;
+    p.o_rows = o_rows;
     const int clusters = p.num_tiles < dev->pair_clusters ? p.num_tiles : dev->pair_clusters;
     record_before(s);
     cudaError_t e;
     if (Y)
         e = launch_dependent(prefill2::gemm_prefill_pair_kernel<false>, dim3(2 * clusters), dim3(prefill2::THREADS),
-                             prefill2::SMEM_BYTES, s, 2, map_xq, map_wq, map_xo, map_y, p);
+                             prefill2::SMEM_BYTES, s, 2, map_xq, map_wq, map_xo, map_w16, map_w16x4, map_w16o, map_y, p);
     else
         e = launch_dependent(prefill2::gemm_prefill_pair_kernel<true>, dim3(2 * clusters), dim3(prefill2::THREADS),
-                             prefill2::SMEM_BYTES, s, 2, map_xq, map_wq, map_xo, map_y, p);
+                             prefill2::SMEM_BYTES, s, 2, map_xq, map_wq, map_xo, map_w16, map_w16x4, map_w16o, map_y, p);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;
@@ -404,9 +432,10 @@ void record_after(cudaStream_t s) {
 
 i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
                           const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
-                          const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
+                          const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s,
+                          const __half *W16o = nullptr) {
 #if I8R_PREFILL_PAIR
-    return launch_prefill_pair(dev, Xq, Xo, T, K, Wq, sW, W16, N, count, idx, sX, Y, acc_out, s);
+    return launch_prefill_pair(dev, Xq, Xo, T, K, Wq, sW, W16, N, count, idx, sX, Y, acc_out, s, W16o);
 #else
     return launch_prefill_single(dev, Xq, Xo, T, K, Wq, sW, W16, N, count, idx, sX, Y, acc_out, s);
 #endif
@@ -561,10 +590,15 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
 
     // decode: the mask kernel clears the split-K accumulator and the tile counters
     const size_t zero_bytes = small_t ? w.total - w.acc32 : 0;
+#if I8R_PREFILL_PAIR
+    __half *W16o = small_t ? nullptr : reinterpret_cast<__half *>(ws + w.W16o);
+#else
+    __half *W16o = nullptr;        // the single-CTA GEMM gathers the rows itself
+#endif
     I8R_TRY(launch_activation(x, T, K, alpha, mask, parts, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
-                              zero_bytes, stream));
+                              zero_bytes, stream, w16, N, W16o));
     if (!small_t)
-        return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream);
+        return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream, W16o);
 
     decode::Params fin{};
     fin.counters = counters;

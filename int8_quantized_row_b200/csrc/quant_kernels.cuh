@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint
 
 // ---------------------------------------------------------------------------
 // Row quantisation of the non-outlier part plus the outlier gather (one
-// block per row of X):
+// block per row of X, after the G blocks that compact outlier weight rows):
 //   sX[t]   = max over k not in O of |X[t,k]|
 //   Xq[t,k] = 0 for k in O, else clamp(rhaz(X[t,k] * fl32(127/sX[t])), +-127)
 //   Xo[t,j] = X[t, O_j] for j < |O|, 0 up to the next multiple of 64
@@ -246,20 +246,82 @@ constexpr int kRowRegChunks = 8;     // 16-byte chunks kept in registers per thr
 // that many rows are in flight per SM (the kernel is latency-bound per row).
 inline int row_threads(int K) { return K <= 4096 ? 64 : (K <= 8192 ? 128 : 256); }
 
+// The W16 rows of the first o_rows outlier columns, compacted for the
+// prefill GEMM (its outlier stages then load two 64 x 64 boxes each instead
+// of gathering rows):  W16o[j,:] = W16[O_j,:] for j < |O|, zero rows up to the
+// next multiple of 64 (at most o_rows).  Runs in the first G blocks of the
+// row quantiser's launch (so that it overlaps the row blocks); block e copies
+// rows e, e+G, ...  Each block ranks the mask's set bits itself.
+constexpr int kCompactOutlierRows = 256;
+
+template <int kThreads>
+__device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *__restrict__ mask, int K,
+                                                           const __half *__restrict__ W16, int N,
+                                                           __half *__restrict__ W16o, int o_rows, int e, int G) {
+    constexpr int kWarps = kThreads / 32;
+    __shared__ int oidx[kCompactOutlierRows];
+    __shared__ int wsum[kWarps];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwords = (K + 31) / 32;
+    const int per = (nwords + kThreads - 1) / kThreads;
+    const int w0 = min(tid * per, nwords), w1 = min(w0 + per, nwords);
+    int local = 0;
+    for (int w = w0; w < w1; ++w) local += __popc(mask[w]);
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        if (w < warp) before += wsum[w];
+        total += wsum[w];
+    }
+    int j = before + incl - local;
+    for (int w = w0; w < w1 && j < o_rows; ++w) {
+        uint32_t m = mask[w];
+        while (m && j < o_rows) {
+            oidx[j++] = w * 32 + (__ffs(m) - 1);
+            m &= m - 1;
+        }
+    }
+    __syncthreads();
+    const int rows = min((total + 63) / 64 * 64, o_rows);
+    const int vec = N / 8;
+    for (int r = e; r < rows; r += G) {
+        uint4 *dst = reinterpret_cast<uint4 *>(W16o + static_cast<size_t>(r) * N);
+        if (r < total) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(W16 + static_cast<size_t>(oidx[r]) * N);
+            for (int c = tid; c < vec; c += kThreads) dst[c] = __ldg(src + c);
+        } else {
+            for (int c = tid; c < vec; c += kThreads) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
 template <int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ mask, float *__restrict__ sX,
     int8_t *__restrict__ Xq, __half *__restrict__ Xo, int32_t *__restrict__ idx_out,
-    int32_t *__restrict__ count_out) {
+    int32_t *__restrict__ count_out, const __half *__restrict__ W16, int N, __half *__restrict__ W16o,
+    int o_rows, int G) {
     constexpr int kWarps = kRowThreads / 32;
     __shared__ float red[kWarps];
     __shared__ int wsum[kWarps];
-    const int t = blockIdx.x;
+    const int t = static_cast<int>(blockIdx.x) - G;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    griddep_launch_dependents();        // the GEMM may start its prologue and weight loads
+    if (t < 0) {
+        gather_outlier_weight_rows<kRowThreads>(mask, K, W16, N, W16o, o_rows, static_cast<int>(blockIdx.x), G);
+        return;
+    }
     const __half *xrow = X + static_cast<size_t>(t) * K;
     const int chunks = K / 8;
     const uint8_t *mbytes = reinterpret_cast<const uint8_t *>(mask);
-    griddep_launch_dependents();        // the GEMM may start its prologue and weight loads
 
     // outlier ranks: this thread's mask words [w0, w1) start at rank `base`
     const int nwords = (K + 31) / 32;
@@ -336,7 +398,7 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     }
 
     // outlier gather (and, in block 0, the index list and its length)
-    const bool publish = blockIdx.x == 0 && idx_out != nullptr;
+    const bool publish = t == 0 && idx_out != nullptr;
     if (Xo || publish) {
         __half *orow = Xo ? Xo + static_cast<size_t>(t) * K : nullptr;
         int j = base;

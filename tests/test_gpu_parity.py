@@ -150,6 +150,10 @@ LINEAR_CASES = [
     (64, 256, 256, [], 0.0, 1.0),                     # alpha = 0: every column in 16-bit
     (200, 256, 256, [], 0.0, 1.0),
     (7, 12288, 1024, [1, 100, 12000], 6.0, 1.0),
+    # prefill past the 256 compacted outlier weight rows: the later outlier
+    # blocks gather their rows (four at a time, the tail one by one)
+    (300, 2048, 512, list(range(0, 2048, 7)), 6.0, 0.5),  # |O| = 293
+    (260, 1024, 256, [], 0.0, 1.0),                       # alpha = 0: |O| = K = 1024
 ]
 
 
@@ -178,6 +182,7 @@ SCHEDULE_CASES = [
     # long schedules: every stage is reused after outlier stages many times over
     (2048, 2048, 8192, [5, 900, 2047], 6.0),                   # 3-4 tiles per CTA pair, 16 k-blocks
     (3000, 1024, 16384, list(range(3, 1024, 15)), 6.0),        # ~10 tiles per pair, |O| = 69
+    (2048, 1024, 4096, list(range(0, 1024, 3)), 6.0),          # |O| = 342: compacted + gathered blocks
 ]
 
 

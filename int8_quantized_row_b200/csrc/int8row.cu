@@ -2,10 +2,10 @@
 // The declarations and their contracts are in include/int8row.h.
 //
 // Pipeline of int8_mixed_linear (all on the caller's stream, no host sync):
-//   outlier_mask_kernel     X -> outlier column bitmask (per 128-row chunk)  (a1)
-//   outlier_index_kernel    T > 128 only: OR of the chunk masks, index list  (a1)
-//   quantize_rows_kernel    X -> sX, Xq (outliers zeroed), Xo gather; for
-//                           T <= 128 it also publishes the index list         (a2, a3)
+//   outlier_mask_kernel     X -> outlier column bitmask (per 256-row chunk)  (a1)
+//   quantize_rows_kernel    OR of the chunk masks, X -> sX, Xq (outliers
+//                           zeroed), Xo gather, the index list; for T > 128
+//                           it also compacts the outliers' W16 rows        (a1-a3)
 //   T > 128:  gemm_prefill_kernel (one CTA per 128 x 256 tile) or
 //             gemm_prefill_pair_kernel (CTA pairs, 256 x 256 tiles): int8 +
 //             fp16 tensor-core MMA, epilogue -> Y
@@ -199,7 +199,14 @@ struct Workspace {
 inline int compact_rows(int K) { return std::min((K + 63) / 64 * 64, kCompactOutlierRows); }
 
 // Row chunks of the outlier scan; each writes one partial mask.
-inline int mask_parts(int T) { return T <= kMaskRowsPerPart ? 1 : (T + kMaskRowsPerPart - 1) / kMaskRowsPerPart; }
+inline int mask_parts(int T) {
+    return T <= kMaskRowsPerPart ? 1 : std::min((T + kMaskRowsPerPart - 1) / kMaskRowsPerPart, kMaxMaskParts);
+}
+// Rows of one part (the last may be shorter).
+inline int mask_rows_per_part(int T) {
+    const int np = mask_parts(T);
+    return np == 1 ? kMaskRowsPerPart : (T + np - 1) / np;
+}
 
 // Scratch for the partial masks when there is more than one (else none).
 inline size_t parts_bytes(int T, int K) {
@@ -232,49 +239,7 @@ Workspace ws_layout(int T, int K, int N) {
     return w;
 }
 
-// a1-a3 on the stream: mask, index list, row quantisation and gather.
-// `parts` holds mask_parts(T) partial masks when there is more than one.
-// `zero` / `zero_bytes`: a region the mask kernel clears on the way (may be null).
-// With W16o, the quantiser's launch also compacts the W16 rows of the first
-// compact_rows(K) outlier columns into W16o ([compact_rows(K), N]).
-i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_t *mask, uint32_t *parts,
-                             int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
-                             size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
-                             __half *W16o = nullptr) {
-    const int np = mask_parts(T);
-    uint32_t *pm = np > 1 ? parts : mask;
-    dim3 grid((K + kStripCols - 1) / kStripCols, np);
-    outlier_mask_kernel<false><<<grid, kStripThreads, 0, s>>>(X, T, K, alpha, kMaskRowsPerPart, pm, nullptr,
-                                                            static_cast<int4 *>(zero), zero_bytes / 16);
-    I8R_LAUNCHED();
-    if (np > 1) {
-        outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(pm, np, K, mask, idx, count, nullptr);
-        I8R_LAUNCHED();
-    }
-    int32_t *publish = np > 1 ? nullptr : idx;     // one part: the quantiser publishes the index list
-    if (T > 0) {
-        const int rt = row_threads(K);
-        const int o_rows = W16o ? compact_rows(K) : 0;
-        const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
-        if (rt == 64)
-            quantize_rows_kernel<64><<<T + G, 64, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count, W16, N, W16o,
-                                                          o_rows, G);
-        else if (rt == 128)
-            quantize_rows_kernel<128><<<T + G, 128, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count, W16, N,
-                                                            W16o, o_rows, G);
-        else
-            quantize_rows_kernel<256><<<T + G, 256, 0, s>>>(X, T, K, mask, sX, Xq, Xo, publish, count, W16, N,
-                                                            W16o, o_rows, G);
-        I8R_LAUNCHED();
-    } else {
-        // no rows: an empty outlier set still has to be published
-        outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(mask, 1, K, mask, idx, count, nullptr);
-        I8R_LAUNCHED();
-    }
-    return I8R_OK;
-}
-
-// Launch a GEMM kernel as a programmatic dependent of the previous kernel on
+// Launch a kernel as a programmatic dependent of the previous kernel on
 // the stream (its prologue may overlap that kernel; it waits with
 // griddepcontrol.wait before touching the previous kernel's outputs).
 // `cluster_x` > 1 launches clusters of that many CTAs along x.
@@ -300,6 +265,62 @@ cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, s
     cfg.attrs = attr;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
+
+// The row quantiser: G compaction blocks, then one block per row, launched as
+// a programmatic dependent of the outlier scan.
+template <int kThreads, typename... Args>
+cudaError_t launch_rows(cudaStream_t s, int T, int G, size_t smem, Args &&...args) {
+    return launch_dependent(quantize_rows_kernel<kThreads>, dim3(G + T), dim3(kThreads), smem, s, 1,
+                            std::forward<Args>(args)...);
+}
+
+// a1-a3 on the stream: mask, index list, row quantisation and gather.
+// `parts` holds mask_parts(T) partial masks when there is more than one.
+// `zero` / `zero_bytes`: a region the mask kernel clears on the way (may be null).
+// With W16o, the quantiser's launch also compacts the W16 rows of the first
+// compact_rows(K) outlier columns into W16o ([compact_rows(K), N]).
+i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_t *mask, uint32_t *parts,
+                             int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
+                             size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
+                             __half *W16o = nullptr) {
+    const int np = mask_parts(T);
+    uint32_t *pm = np > 1 ? parts : mask;
+    dim3 grid((K + kStripCols - 1) / kStripCols, np);
+    outlier_mask_kernel<false><<<grid, kStripThreads, 0, s>>>(X, T, K, alpha, mask_rows_per_part(T), pm, nullptr,
+                                                            static_cast<int4 *>(zero), zero_bytes / 16);
+    I8R_LAUNCHED();
+    if (T > 0) {
+        // the quantiser ORs the parts itself; row 0's block publishes the
+        // mask (when there are parts), the index list and |O|
+        const int rt = row_threads(K);
+        const int o_rows = W16o ? compact_rows(K) : 0;
+        const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
+        const size_t smem = quantize_smem_bytes(K);
+        uint32_t *mask_out = np > 1 ? mask : nullptr;
+        const uint32_t *parts_in = pm;
+        cudaError_t e;
+        if (rt == 64)
+            e = launch_rows<64>(s, T, G, smem, X, T, K, parts_in, np, sX, Xq, Xo, mask_out, idx, count, W16, N, W16o,
+                                o_rows, G);
+        else if (rt == 128)
+            e = launch_rows<128>(s, T, G, smem, X, T, K, parts_in, np, sX, Xq, Xo, mask_out, idx, count, W16, N,
+                                 W16o, o_rows, G);
+        else
+            e = launch_rows<256>(s, T, G, smem, X, T, K, parts_in, np, sX, Xq, Xo, mask_out, idx, count, W16, N,
+                                 W16o, o_rows, G);
+        if (e != cudaSuccess) {
+            tl_last_cuda_error = static_cast<int>(e);
+            return I8R_ECUDA;
+        }
+        I8R_LAUNCHED();
+    } else {
+        // no rows: an empty outlier set still has to be published
+        outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(mask, 1, K, mask, idx, count, nullptr);
+        I8R_LAUNCHED();
+    }
+    return I8R_OK;
+}
+
 
 void record_before(cudaStream_t s) {
     if (tl_ev_before) cudaEventRecord(tl_ev_before, s);

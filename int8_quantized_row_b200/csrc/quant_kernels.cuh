@@ -79,11 +79,13 @@ __global__ void __launch_bounds__(256) weight_codes_kernel(const __half *__restr
 // (outliers defined by magnitude; "The LLM.int8() Methodology").
 // Block (x, y) owns columns [64x, 64x+64) of rows [y*rows_per_part,
 // (y+1)*rows_per_part) and writes the two partial mask words
-// part_masks[y*words + 2x + {0,1}]; outlier_index_kernel ORs the parts.  With
-// one part (gridDim.y == 1) the partial words are the mask, and the optional
-// per-column hit counts are exact.  A thread keeps 8 row loads in flight.
+// part_masks[y*words + 2x + {0,1}]; the row quantiser (or, for the statistics,
+// outlier_index_kernel) ORs the parts.  With one part (gridDim.y == 1) the
+// partial words are the mask, and the optional per-column hit counts are
+// exact.  A thread keeps 8 row loads in flight.
 // ---------------------------------------------------------------------------
-constexpr int kMaskRowsPerPart = 256;
+constexpr int kMaskRowsPerPart = 256;   // rows of one part, up to kMaxMaskParts parts
+constexpr int kMaxMaskParts = 4;
 
 template <bool kHits>
 __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __half *__restrict__ X, int T, int K,
@@ -96,6 +98,7 @@ __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __hal
     constexpr int kUnroll = 8;                         // row loads in flight per thread
     __shared__ uint32_t wflags[kWarps][8];
     __shared__ int32_t wcnt[kHits ? kWarps : 1][kHits ? kStripCols : 1];
+    griddep_launch_dependents();       // the row quantiser may start loading its rows
     if (zero) {
         const size_t nthreads = static_cast<size_t>(gridDim.x) * gridDim.y * kStripThreads;
         for (size_t i = (static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x) * kStripThreads + threadIdx.x;
@@ -236,9 +239,13 @@ __global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint
 //   sX[t]   = max over k not in O of |X[t,k]|
 //   Xq[t,k] = 0 for k in O, else clamp(rhaz(X[t,k] * fl32(127/sX[t])), +-127)
 //   Xo[t,j] = X[t, O_j] for j < |O|, 0 up to the next multiple of 64
-// Every block ranks the outlier columns itself from the mask (a prefix count
-// of the mask words' population counts), so no index kernel runs in between;
-// block 0 also publishes the ascending index list and |O| for the GEMM.
+// ("Vector-wise quantization" and "Mixed-precision decomposition").
+// Every block ORs the partial masks of the outlier scan into shared memory
+// and ranks the outlier columns itself (prefix counts of the mask words'
+// population counts), so no index kernel runs in between; row 0's block also
+// publishes the mask, the ascending index list and |O|.
+// The kernel is launched as a programmatic dependent of the outlier scan: the
+// row is loaded before the block waits for the scan to finish.
 // ---------------------------------------------------------------------------
 constexpr int kRowRegChunks = 8;     // 16-byte chunks kept in registers per thread
 
@@ -246,44 +253,25 @@ constexpr int kRowRegChunks = 8;     // 16-byte chunks kept in registers per thr
 // that many rows are in flight per SM (the kernel is latency-bound per row).
 inline int row_threads(int K) { return K <= 4096 ? 64 : (K <= 8192 ? 128 : 256); }
 
+// Dynamic shared memory of quantize_rows_kernel: the mask words and the
+// exclusive prefix of their population counts.
+inline size_t quantize_smem_bytes(int K) { return static_cast<size_t>((K + 31) / 32) * 8; }
+
 // The W16 rows of the first o_rows outlier columns, compacted for the
 // prefill GEMM (its outlier stages then load two 64 x 64 boxes each instead
 // of gathering rows):  W16o[j,:] = W16[O_j,:] for j < |O|, zero rows up to the
-// next multiple of 64 (at most o_rows).  Runs in the first G blocks of the
-// row quantiser's launch (so that it overlaps the row blocks); block e copies
-// rows e, e+G, ...  Each block ranks the mask's set bits itself.
+// next multiple of 64 (at most o_rows).  Block e of the G compaction blocks
+// copies rows e, e+G, ... with eight 16-byte loads in flight per thread.
 constexpr int kCompactOutlierRows = 256;
 
 template <int kThreads>
-__device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *__restrict__ mask, int K,
-                                                           const __half *__restrict__ W16, int N,
+__device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *smask, const int *spre, int w0, int w1,
+                                                           int total, const __half *__restrict__ W16, int N,
                                                            __half *__restrict__ W16o, int o_rows, int e, int G) {
-    constexpr int kWarps = kThreads / 32;
     __shared__ int oidx[kCompactOutlierRows];
-    __shared__ int wsum[kWarps];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nwords = (K + 31) / 32;
-    const int per = (nwords + kThreads - 1) / kThreads;
-    const int w0 = min(tid * per, nwords), w1 = min(w0 + per, nwords);
-    int local = 0;
-    for (int w = w0; w < w1; ++w) local += __popc(mask[w]);
-    int incl = local;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const int y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += y;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int before = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-        if (w < warp) before += wsum[w];
-        total += wsum[w];
-    }
-    int j = before + incl - local;
-    for (int w = w0; w < w1 && j < o_rows; ++w) {
-        uint32_t m = mask[w];
+    for (int w = w0; w < w1; ++w) {
+        int j = spre[w];
+        uint32_t m = smask[w];
         while (m && j < o_rows) {
             oidx[j++] = w * 32 + (__ffs(m) - 1);
             m &= m - 1;
@@ -292,43 +280,95 @@ __device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *__res
     __syncthreads();
     const int rows = min((total + 63) / 64 * 64, o_rows);
     const int vec = N / 8;
+    constexpr int kBatch = 8;
     for (int r = e; r < rows; r += G) {
         uint4 *dst = reinterpret_cast<uint4 *>(W16o + static_cast<size_t>(r) * N);
-        if (r < total) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(W16 + static_cast<size_t>(oidx[r]) * N);
-            for (int c = tid; c < vec; c += kThreads) dst[c] = __ldg(src + c);
-        } else {
-            for (int c = tid; c < vec; c += kThreads) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 *src = r < total ? reinterpret_cast<const uint4 *>(W16 + static_cast<size_t>(oidx[r]) * N) : nullptr;
+        for (int c0 = static_cast<int>(threadIdx.x); c0 < vec; c0 += kThreads * kBatch) {
+            uint4 v[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int c = c0 + b * kThreads;
+                v[b] = (src && c < vec) ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+                const int c = c0 + b * kThreads;
+                if (c < vec) dst[c] = v[b];
+            }
         }
     }
 }
 
+// Absolute value of eight fp16 lanes (sign bits cleared) folded into a
+// running fp16x2 maximum; exact, since max and |.| are exact in fp16.
+__device__ __forceinline__ __half2 habs_max8(__half2 m, const uint4 &u) {
+    const uint32_t a[4] = {u.x & 0x7FFF7FFFu, u.y & 0x7FFF7FFFu, u.z & 0x7FFF7FFFu, u.w & 0x7FFF7FFFu};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m = __hmax2(m, *reinterpret_cast<const __half2 *>(&a[k]));
+    return m;
+}
+
+// The int8 code of y = fl32(x * inv) with the rule of quant_code, in fewer
+// steps: |y| + 1/2 rounded toward -inf has the same floor as the exact sum
+// (the floor is an integer, hence a float, below the exact sum), so
+// floor(fl_rd(|y| + 1/2)) = rhaz(|y|) for every finite y; the sign is put
+// back afterwards.  |y| <= 127 * (1 + 2^-23) for x in the row's range, so the
+// clamp only matters for infinities.
+__device__ __forceinline__ int quant_code_fast(float x, float inv) {
+    const float y = __fmul_rn(x, inv);
+    const int q = min(__float2int_rd(__fadd_rd(fabsf(y), 0.5f)), 127);
+    return y < 0.0f ? -q : q;
+}
+
+// Four codes in [-127, 127] as the bytes of a word, q0 lowest.
+__device__ __forceinline__ uint32_t pack4_s8(int q0, int q1, int q2, int q3) {
+    const uint32_t p01 = __byte_perm(static_cast<uint32_t>(q0), static_cast<uint32_t>(q1), 0x0040u);
+    const uint32_t p23 = __byte_perm(static_cast<uint32_t>(q2), static_cast<uint32_t>(q3), 0x0040u);
+    return __byte_perm(p01, p23, 0x5410u);
+}
+
 template <int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
-    const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ mask, float *__restrict__ sX,
-    int8_t *__restrict__ Xq, __half *__restrict__ Xo, int32_t *__restrict__ idx_out,
-    int32_t *__restrict__ count_out, const __half *__restrict__ W16, int N, __half *__restrict__ W16o,
-    int o_rows, int G) {
+    const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ parts, int nparts,
+    float *__restrict__ sX, int8_t *__restrict__ Xq, __half *__restrict__ Xo, uint32_t *__restrict__ mask_out,
+    int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out, const __half *__restrict__ W16, int N,
+    __half *__restrict__ W16o, int o_rows, int G) {
     constexpr int kWarps = kRowThreads / 32;
+    extern __shared__ uint32_t qs[];
     __shared__ float red[kWarps];
     __shared__ int wsum[kWarps];
-    const int t = static_cast<int>(blockIdx.x) - G;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    griddep_launch_dependents();        // the GEMM may start its prologue and weight loads
-    if (t < 0) {
-        gather_outlier_weight_rows<kRowThreads>(mask, K, W16, N, W16o, o_rows, static_cast<int>(blockIdx.x), G);
-        return;
-    }
-    const __half *xrow = X + static_cast<size_t>(t) * K;
-    const int chunks = K / 8;
-    const uint8_t *mbytes = reinterpret_cast<const uint8_t *>(mask);
-
-    // outlier ranks: this thread's mask words [w0, w1) start at rank `base`
     const int nwords = (K + 31) / 32;
+    uint32_t *smask = qs;
+    int *spre = reinterpret_cast<int *>(qs + nwords);
+    const int t = static_cast<int>(blockIdx.x) - G;             // row; < 0: compaction block
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int chunks = K / 8;
+    griddep_launch_dependents();        // the GEMM may start its prologue and weight loads
+
+    // The row goes into registers first: X does not depend on the outlier scan.
+    const __half *xrow = X + static_cast<size_t>(t < 0 ? 0 : t) * K;
+    Vec16 keep[kRowRegChunks];
+    if (t >= 0) {
+#pragma unroll
+        for (int c = 0; c < kRowRegChunks; ++c) {
+            const int i = tid + c * kRowThreads;
+            if (i < chunks) keep[c].u = __ldg(reinterpret_cast<const uint4 *>(xrow) + i);
+        }
+    }
+    griddep_wait();                     // the outlier scan's partial masks are complete
+
+    // the mask (OR of the parts), then each word's count of earlier outliers
+    for (int w = tid; w < nwords; w += kRowThreads) {
+        uint32_t m = parts[w];
+        for (int q = 1; q < nparts; ++q) m |= parts[static_cast<size_t>(q) * nwords + w];
+        smask[w] = m;
+    }
+    __syncthreads();
     const int per = (nwords + kRowThreads - 1) / kRowThreads;
     const int w0 = min(tid * per, nwords), w1 = min(w0 + per, nwords);
     int local = 0;
-    for (int w = w0; w < w1; ++w) local += __popc(mask[w]);
+    for (int w = w0; w < w1; ++w) local += __popc(smask[w]);
     int incl = local;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -336,55 +376,84 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
         if (lane >= d) incl += y;
     }
     if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+        if (w < warp) before += wsum[w];
+        total += wsum[w];
+    }
+    {
+        int run = before + incl - local;
+        for (int w = w0; w < w1; ++w) {
+            spre[w] = run;
+            run += __popc(smask[w]);
+        }
+    }
+    __syncthreads();
+    if (t < 0) {
+        gather_outlier_weight_rows<kRowThreads>(smask, spre, w0, w1, total, W16, N, W16o, o_rows,
+                                                static_cast<int>(blockIdx.x), G);
+        return;
+    }
+    const uint8_t *mbytes = reinterpret_cast<const uint8_t *>(smask);
 
-    Vec16 keep[kRowRegChunks];
+    // row absmax over the non-outlier columns
+    __half2 hmax = __float2half2_rn(0.0f);
     float amax = 0.0f;
+    auto scan = [&](int i, const Vec16 &v) {
+        const uint32_t mb = mbytes[i];
+        if (mb == 0) {
+            hmax = habs_max8(hmax, v.u);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if (!((mb >> e) & 1u)) amax = fmaxf(amax, fabsf(__half2float(v.h[e])));
+        }
+    };
 #pragma unroll
     for (int c = 0; c < kRowRegChunks; ++c) {
         const int i = tid + c * kRowThreads;
-        if (i < chunks) {
-            keep[c].u = __ldg(reinterpret_cast<const uint4 *>(xrow) + i);
-            const uint32_t mb = mbytes[i];
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                if (!((mb >> e) & 1u)) amax = fmaxf(amax, fabsf(__half2float(keep[c].h[e])));
-        }
+        if (i < chunks) scan(i, keep[c]);
     }
     for (int i = tid + kRowRegChunks * kRowThreads; i < chunks; i += kRowThreads) {
         Vec16 v;
         v.u = __ldg(reinterpret_cast<const uint4 *>(xrow) + i);
-        const uint32_t mb = mbytes[i];
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-            if (!((mb >> e) & 1u)) amax = fmaxf(amax, fabsf(__half2float(v.h[e])));
+        scan(i, v);
     }
+    amax = fmaxf(amax, fmaxf(__low2float(hmax), __high2float(hmax)));
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, d));
     if (lane == 0) red[warp] = amax;
     __syncthreads();
     float s = 0.0f;
-    int before = 0, total = 0;
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-        s = fmaxf(s, red[w]);
-        if (w < warp) before += wsum[w];
-        total += wsum[w];
-    }
-    const int base = before + incl - local;
+    for (int w = 0; w < kWarps; ++w) s = fmaxf(s, red[w]);
     const float inv = recip127(s);
     if (tid == 0) sX[t] = s;
 
     int8_t *qrow = Xq + static_cast<size_t>(t) * K;
+    __half *orow = Xo ? Xo + static_cast<size_t>(t) * K : nullptr;
     auto emit = [&](int i, const Vec16 &v) {
         const uint32_t mb = mbytes[i];
-        uint32_t lo = 0, hi = 0;
+        int q[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int q = ((mb >> e) & 1u) ? 0 : quant_code(__half2float(v.h[e]), inv);
-            const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
-            if (e < 4) lo |= b << (8 * e); else hi |= b << (8 * (e - 4));
+        for (int e = 0; e < 8; ++e) q[e] = quant_code_fast(__half2float(v.h[e]), inv);
+        if (mb) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if ((mb >> e) & 1u) q[e] = 0;
         }
-        reinterpret_cast<uint2 *>(qrow)[i] = make_uint2(lo, hi);
+        reinterpret_cast<uint2 *>(qrow)[i] =
+            make_uint2(pack4_s8(q[0], q[1], q[2], q[3]), pack4_s8(q[4], q[5], q[6], q[7]));
+        if (orow && mb) {
+            // this chunk's outliers go to their ranks in Xo
+            const int w = i >> 2, sh = (i & 3) * 8;
+            int j = spre[w] + __popc(smask[w] & ((1u << sh) - 1u));
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                if ((mb >> e) & 1u) orow[j++] = v.h[e];
+        }
     };
 #pragma unroll
     for (int c = 0; c < kRowRegChunks; ++c) {
@@ -396,27 +465,24 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
         v.u = __ldg(reinterpret_cast<const uint4 *>(xrow) + i);
         emit(i, v);
     }
+    if (orow) {
+        const int padded = (total + 63) / 64 * 64;
+        for (int jj = total + tid; jj < padded; jj += kRowThreads) orow[jj] = __float2half_rn(0.0f);
+    }
 
-    // outlier gather (and, in block 0, the index list and its length)
-    const bool publish = t == 0 && idx_out != nullptr;
-    if (Xo || publish) {
-        __half *orow = Xo ? Xo + static_cast<size_t>(t) * K : nullptr;
-        int j = base;
+    // row 0's block: the mask, the index list and its length
+    if (t == 0 && idx_out) {
+        if (mask_out)
+            for (int w = tid; w < nwords; w += kRowThreads) mask_out[w] = smask[w];
         for (int w = w0; w < w1; ++w) {
-            uint32_t m = mask[w];
+            int j = spre[w];
+            uint32_t m = smask[w];
             while (m) {
-                const int k = w * 32 + (__ffs(m) - 1);
-                if (orow) orow[j] = xrow[k];
-                if (publish) idx_out[j] = k;
-                ++j;
+                idx_out[j++] = w * 32 + (__ffs(m) - 1);
                 m &= m - 1;
             }
         }
-        if (orow) {
-            const int padded = (total + 63) / 64 * 64;
-            for (int jj = total + tid; jj < padded; jj += kRowThreads) orow[jj] = __float2half_rn(0.0f);
-        }
-        if (publish && tid == 0) *count_out = total;
+        if (tid == 0) *count_out = total;
     }
 }
 

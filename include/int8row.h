@@ -170,8 +170,7 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha,
  *   Xo    [T,K] fp16 (nullable) Xo[t,j] = X[t, idx[j]] for j < |O|, 0 for
  *                               |O| <= j < 64*ceil(|O|/64); later columns untouched
  *   workspace  at least int8_quantize_activation_workspace_size(T, K) bytes
- *              (partial outlier masks of up to 4 row chunks; 0 bytes when
- *              T <= 256)
+ *              (currently 0: it may be NULL)
  *
  * int8_gemm_i8_s32: acc [T,N] int32 = Xq [T,K] int8 x Wq [K,N] int8, exact,
  *   by the same tensor-core kernels int8_mixed_linear uses (decode-shaped for

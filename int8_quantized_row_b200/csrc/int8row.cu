@@ -2,10 +2,13 @@
 // The declarations and their contracts are in include/int8row.h.
 //
 // Pipeline of int8_mixed_linear (all on the caller's stream, no host sync):
-//   outlier_mask_kernel     X -> outlier column bitmask (per 256-row chunk)  (a1)
-//   quantize_rows_kernel    OR of the chunk masks, X -> sX, Xq (outliers
-//                           zeroed), Xo gather, the index list; for T > 128
-//                           it also compacts the outliers' W16 rows        (a1-a3)
+//   clear_mask_kernel       zeroes the outlier column bitmask
+//   outlier_scan_kernel     X -> outlier column bitmask, atomic OR per word   (a1)
+//   quantize_rows_kernel    X -> sX, Xq (outliers zeroed), Xo gather, the
+//                           index list; for T > 128 it also compacts the
+//                           outliers' W16 rows                              (a1-a3)
+// The scan and the quantiser are programmatic dependents of the kernel
+// before them, so each loads its rows of X before waiting for it.
 //   T > 128:  gemm_prefill_kernel (one CTA per 128 x 256 tile) or
 //             gemm_prefill_pair_kernel (CTA pairs, 256 x 256 tiles): int8 +
 //             fp16 tensor-core MMA, epilogue -> Y
@@ -192,34 +195,17 @@ i8r_status check_ptr(const void *p) {
 
 // Workspace of int8_mixed_linear.
 struct Workspace {
-    size_t count, mask, parts, idx, sX, Xq, Xo, W16o, acc32, counters, total;
+    size_t count, mask, idx, sX, Xq, Xo, W16o, acc32, counters, total;
 };
 
 // Rows of the compacted outlier weight rows kept for the prefill GEMM.
 inline int compact_rows(int K) { return std::min((K + 63) / 64 * 64, kCompactOutlierRows); }
-
-// Row chunks of the outlier scan; each writes one partial mask.
-inline int mask_parts(int T) {
-    return T <= kMaskRowsPerPart ? 1 : std::min((T + kMaskRowsPerPart - 1) / kMaskRowsPerPart, kMaxMaskParts);
-}
-// Rows of one part (the last may be shorter).
-inline int mask_rows_per_part(int T) {
-    const int np = mask_parts(T);
-    return np == 1 ? kMaskRowsPerPart : (T + np - 1) / np;
-}
-
-// Scratch for the partial masks when there is more than one (else none).
-inline size_t parts_bytes(int T, int K) {
-    const int np = mask_parts(T);
-    return np > 1 ? align_up(static_cast<size_t>(np) * ((K + 31) / 32) * 4) : 0;
-}
 
 Workspace ws_layout(int T, int K, int N) {
     Workspace w{};
     size_t off = 0;
     w.count = off; off = align_up(off + sizeof(int32_t));
     w.mask = off;  off = align_up(off + static_cast<size_t>((K + 31) / 32) * 4);
-    w.parts = off; off += parts_bytes(T, K);
     w.idx = off;   off = align_up(off + static_cast<size_t>(K) * 4);
     w.sX = off;    off = align_up(off + static_cast<size_t>(T) * 4);
     w.Xq = off;    off = align_up(off + static_cast<size_t>(T) * K);
@@ -274,50 +260,62 @@ cudaError_t launch_rows(cudaStream_t s, int T, int G, size_t smem, Args &&...arg
                             std::forward<Args>(args)...);
 }
 
-// a1-a3 on the stream: mask, index list, row quantisation and gather.
-// `parts` holds mask_parts(T) partial masks when there is more than one.
-// `zero` / `zero_bytes`: a region the mask kernel clears on the way (may be null).
+// Grid of the row-band outlier scan: bands of 2048 columns, row blocks of at
+// least 8 rows, about four blocks per SM.
+dim3 scan_grid(int T, int K, int sms, int *rows_per_block) {
+    const int bands = (K + kBandCols - 1) / kBandCols;
+    const int want = std::max(1, (4 * sms + bands - 1) / bands);
+    const int chunks = std::max(1, std::min((T + 7) / 8, want));
+    *rows_per_block = std::max(1, (T + chunks - 1) / chunks);
+    return dim3(bands, (T + *rows_per_block - 1) / *rows_per_block);
+}
+
+// a1-a3 on the stream: mask, row quantisation, index list and gather.
+// `zero` / `zero_bytes`: a region the scan clears on the way (may be null).
 // With W16o, the quantiser's launch also compacts the W16 rows of the first
 // compact_rows(K) outlier columns into W16o ([compact_rows(K), N]).
-i8r_status launch_activation(const __half *X, int T, int K, float alpha, uint32_t *mask, uint32_t *parts,
+i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int K, float alpha, uint32_t *mask,
                              int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
                              size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
                              __half *W16o = nullptr) {
-    const int np = mask_parts(T);
-    uint32_t *pm = np > 1 ? parts : mask;
-    dim3 grid((K + kStripCols - 1) / kStripCols, np);
-    outlier_mask_kernel<false><<<grid, kStripThreads, 0, s>>>(X, T, K, alpha, mask_rows_per_part(T), pm, nullptr,
-                                                            static_cast<int4 *>(zero), zero_bytes / 16);
+    const int nwords = (K + 31) / 32;
+    clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords);
     I8R_LAUNCHED();
-    if (T > 0) {
-        // the quantiser ORs the parts itself; row 0's block publishes the
-        // mask (when there are parts), the index list and |O|
-        const int rt = row_threads(K);
-        const int o_rows = W16o ? compact_rows(K) : 0;
-        const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
-        const size_t smem = quantize_smem_bytes(K);
-        uint32_t *mask_out = np > 1 ? mask : nullptr;
-        const uint32_t *parts_in = pm;
-        cudaError_t e;
-        if (rt == 64)
-            e = launch_rows<64>(s, T, G, smem, X, T, K, parts_in, np, sX, Xq, Xo, mask_out, idx, count, W16, N, W16o,
-                                o_rows, G);
-        else if (rt == 128)
-            e = launch_rows<128>(s, T, G, smem, X, T, K, parts_in, np, sX, Xq, Xo, mask_out, idx, count, W16, N,
-                                 W16o, o_rows, G);
-        else
-            e = launch_rows<256>(s, T, G, smem, X, T, K, parts_in, np, sX, Xq, Xo, mask_out, idx, count, W16, N,
-                                 W16o, o_rows, G);
-        if (e != cudaSuccess) {
-            tl_last_cuda_error = static_cast<int>(e);
-            return I8R_ECUDA;
-        }
-        I8R_LAUNCHED();
-    } else {
+    if (T == 0) {
         // no rows: an empty outlier set still has to be published
         outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(mask, 1, K, mask, idx, count, nullptr);
         I8R_LAUNCHED();
+        return I8R_OK;
     }
+    int rows_per_block = 0;
+    const dim3 grid = scan_grid(T, K, dev->sms, &rows_per_block);
+    cudaError_t e = launch_dependent(outlier_scan_kernel, grid, dim3(kScanThreads), 0, s, 1, X, T, K, alpha,
+                                     rows_per_block, mask, static_cast<int4 *>(zero), zero_bytes / 16);
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = static_cast<int>(e);
+        return I8R_ECUDA;
+    }
+    I8R_LAUNCHED();
+    // row 0's block of the quantiser publishes the index list and |O|
+    const int rt = row_threads(K);
+    const int o_rows = W16o ? compact_rows(K) : 0;
+    const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
+    const size_t smem = quantize_smem_bytes(K);
+    const uint32_t *m = mask;
+    uint32_t *no_mask_out = nullptr;
+    if (rt == 64)
+        e = launch_rows<64>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, N, W16o, o_rows, G);
+    else if (rt == 128)
+        e = launch_rows<128>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, N, W16o, o_rows,
+                             G);
+    else
+        e = launch_rows<256>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, N, W16o, o_rows,
+                             G);
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = static_cast<int>(e);
+        return I8R_ECUDA;
+    }
+    I8R_LAUNCHED();
     return I8R_OK;
 }
 
@@ -597,7 +595,6 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int32_t *count = reinterpret_cast<int32_t *>(ws + w.count);
     uint32_t *mask = reinterpret_cast<uint32_t *>(ws + w.mask);
-    uint32_t *parts = reinterpret_cast<uint32_t *>(ws + w.parts);
     int32_t *idx = reinterpret_cast<int32_t *>(ws + w.idx);
     float *sX = reinterpret_cast<float *>(ws + w.sX);
     int8_t *Xq = reinterpret_cast<int8_t *>(ws + w.Xq);
@@ -609,14 +606,14 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
     const __half *w16 = static_cast<const __half *>(W16);
     __half *y = static_cast<__half *>(Y);
 
-    // decode: the mask kernel clears the split-K accumulator and the tile counters
+    // decode: the outlier scan clears the split-K accumulator and the tile counters
     const size_t zero_bytes = small_t ? w.total - w.acc32 : 0;
 #if I8R_PREFILL_PAIR
     __half *W16o = small_t ? nullptr : reinterpret_cast<__half *>(ws + w.W16o);
 #else
     __half *W16o = nullptr;        // the single-CTA GEMM gathers the rows itself
 #endif
-    I8R_TRY(launch_activation(x, T, K, alpha, mask, parts, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
+    I8R_TRY(launch_activation(dev, x, T, K, alpha, mask, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
                               zero_bytes, stream, w16, N, W16o));
     if (!small_t)
         return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream, W16o);
@@ -681,8 +678,9 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha, int32_t 
 }
 
 size_t int8_quantize_activation_workspace_size(int T, int K) {
-    if (T < 0 || K < 0) return 0;
-    return parts_bytes(T, K);
+    (void)T;
+    (void)K;
+    return 0;                      // the activation side needs no scratch of its own
 }
 
 i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha, uint32_t *mask, int32_t *idx,
@@ -699,13 +697,12 @@ i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha, ui
     I8R_TRY(check_ptr(mask));
     I8R_TRY(check_ptr(idx));
     if (!count) return I8R_EINVAL;
-    const size_t need = parts_bytes(T, K);
-    if (need && (!workspace || workspace_bytes < need)) return I8R_EWORKSPACE;
-    if (need && !aligned16(workspace)) return I8R_EALIGN;
+    (void)workspace;
+    (void)workspace_bytes;
     const DeviceInfo *dev = nullptr;
     I8R_TRY(device_setup(&dev));
-    return launch_activation(static_cast<const __half *>(X), T, K, alpha, mask, static_cast<uint32_t *>(workspace),
-                             idx, count, sX, Xq, static_cast<__half *>(Xo), nullptr, 0, stream);
+    return launch_activation(dev, static_cast<const __half *>(X), T, K, alpha, mask, idx, count, sX, Xq,
+                             static_cast<__half *>(Xo), nullptr, 0, stream);
 }
 
 size_t int8_gemm_i8_s32_workspace_size(int T, int K, int N) {

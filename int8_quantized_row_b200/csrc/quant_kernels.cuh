@@ -77,15 +77,12 @@ __global__ void __launch_bounds__(256) weight_codes_kernel(const __half *__restr
 // ---------------------------------------------------------------------------
 // Outlier feature dimensions: mask bit k set when any |X[t,k]| >= alpha
 // (outliers defined by magnitude; "The LLM.int8() Methodology").
-// Block (x, y) owns columns [64x, 64x+64) of rows [y*rows_per_part,
-// (y+1)*rows_per_part) and writes the two partial mask words
-// part_masks[y*words + 2x + {0,1}]; the row quantiser (or, for the statistics,
-// outlier_index_kernel) ORs the parts.  With one part (gridDim.y == 1) the
-// partial words are the mask, and the optional per-column hit counts are
-// exact.  A thread keeps 8 row loads in flight.
+// Column-strip form, used by the outlier statistics: block (x, y) owns
+// columns [64x, 64x+64) of rows [y*rows_per_part, (y+1)*rows_per_part) and
+// writes the two partial mask words part_masks[y*words + 2x + {0,1}].  With
+// one part (gridDim.y == 1) the partial words are the mask, and the optional
+// per-column hit counts are exact.  A thread keeps 8 row loads in flight.
 // ---------------------------------------------------------------------------
-constexpr int kMaskRowsPerPart = 256;   // rows of one part, up to kMaxMaskParts parts
-constexpr int kMaxMaskParts = 4;
 
 template <bool kHits>
 __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __half *__restrict__ X, int T, int K,
@@ -170,6 +167,64 @@ __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __hal
         const int c = blockIdx.x * kStripCols + tid;
         if (c < K) hits[c] = r;
     }
+}
+
+// ---------------------------------------------------------------------------
+// Outlier feature dimensions for int8_mixed_linear: the same mask bits as
+// outlier_mask_kernel, scanned in row bands so that every warp load is 512
+// contiguous bytes of one row.  Block (b, c) covers columns
+// [2048b, 2048b + 2048) (8 per thread) of rows [c*rows_per_block, ...) and
+// ORs its non-zero 32-column words into `mask` with atomics; clear_mask_kernel
+// zeroes the mask first, and this kernel, its programmatic dependent, waits
+// for that only after its row loads.  Optionally clears `zero` on the way.
+// ---------------------------------------------------------------------------
+constexpr int kScanThreads = 256;
+constexpr int kBandCols = kScanThreads * 8;
+
+__global__ void __launch_bounds__(256) clear_mask_kernel(uint32_t *__restrict__ mask, int nwords) {
+    griddep_launch_dependents();        // the scan may start loading rows
+    for (int w = threadIdx.x; w < nwords; w += blockDim.x) mask[w] = 0u;
+}
+
+__global__ void __launch_bounds__(kScanThreads) outlier_scan_kernel(const __half *__restrict__ X, int T, int K,
+                                                                   float alpha, int rows_per_block,
+                                                                   uint32_t *__restrict__ mask,
+                                                                   int4 *__restrict__ zero, size_t zero16) {
+    constexpr int kUnroll = 8;          // row loads in flight per thread
+    griddep_launch_dependents();        // the row quantiser may start loading its rows
+    if (zero) {
+        const size_t nthreads = static_cast<size_t>(gridDim.x) * gridDim.y * kScanThreads;
+        for (size_t i = (static_cast<size_t>(blockIdx.y) * gridDim.x + blockIdx.x) * kScanThreads + threadIdx.x;
+             i < zero16; i += nthreads)
+            zero[i] = make_int4(0, 0, 0, 0);
+    }
+    const int col = blockIdx.x * kBandCols + threadIdx.x * 8;
+    const int r0 = blockIdx.y * rows_per_block;
+    const int r1 = min(T, r0 + rows_per_block);
+    uint32_t f = 0;
+    if (col < K) {
+        const __half *xc = X + col;
+        for (int t = r0; t < r1; t += kUnroll) {
+            Vec16 v[kUnroll];
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u)
+                v[u].u = t + u < r1 ? __ldg(reinterpret_cast<const uint4 *>(xc + static_cast<size_t>(t + u) * K))
+                                    : make_uint4(0, 0, 0, 0);
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const bool live = t + u < r1;
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    f |= static_cast<uint32_t>(live && fabsf(__half2float(v[u].h[i])) >= alpha) << i;
+            }
+        }
+    }
+    // four neighbouring threads hold the four bytes of one 32-column word
+    uint32_t w = f << (8 * (threadIdx.x & 3));
+    w |= __shfl_xor_sync(0xFFFFFFFFu, w, 1);
+    w |= __shfl_xor_sync(0xFFFFFFFFu, w, 2);
+    griddep_wait();                     // the mask has been cleared
+    if ((threadIdx.x & 3) == 0 && w != 0u) atomicOr(mask + col / 32, w);
 }
 
 // ---------------------------------------------------------------------------
@@ -309,16 +364,15 @@ __device__ __forceinline__ __half2 habs_max8(__half2 m, const uint4 &u) {
     return m;
 }
 
-// The int8 code of y = fl32(x * inv) with the rule of quant_code, in fewer
-// steps: |y| + 1/2 rounded toward -inf has the same floor as the exact sum
-// (the floor is an integer, hence a float, below the exact sum), so
-// floor(fl_rd(|y| + 1/2)) = rhaz(|y|) for every finite y; the sign is put
-// back afterwards.  |y| <= 127 * (1 + 2^-23) for x in the row's range, so the
-// clamp only matters for infinities.
+// The int8 code of y = fl32(x * inv) with the rule of quant_code, in four
+// steps: rhaz(y) = trunc(y + copysign(1/2, y)) for the exact sum, and the sum
+// rounded toward zero truncates to the same integer (that integer lies
+// between zero and the exact sum and is a float, so rounding toward zero
+// cannot pass it).  |y| <= 127 * (1 + 2^-23) for x in the row's range, so
+// no clamp is needed.
 __device__ __forceinline__ int quant_code_fast(float x, float inv) {
     const float y = __fmul_rn(x, inv);
-    const int q = min(__float2int_rd(__fadd_rd(fabsf(y), 0.5f)), 127);
-    return y < 0.0f ? -q : q;
+    return __float2int_rz(__fadd_rz(y, copysignf(0.5f, y)));
 }
 
 // Four codes in [-127, 127] as the bytes of a word, q0 lowest.

@@ -62,6 +62,7 @@ ACT_CASES = [
     (17, 256, [], 0.0),                      # every column is an outlier
     (17, 256, [10, 20], float("inf")),       # none is
     (5, 12288, [7, 12287], 6.0),
+    (2100, 1024, [5, 1000], 6.0),            # eight partial masks of 263 rows
 ]
 
 
@@ -87,6 +88,31 @@ def test_activation_quantisation_bit_exact(orc, T, K, cols, alpha):
     pad = (cnt + 63) // 64 * 64
     assert np.array_equal(Xo[:, :cnt].view(np.uint16), X[:, idx_o].view(np.uint16))
     assert np.all(Xo[:, cnt:pad] == 0)
+    assert device_status_clean()
+
+
+def test_quantiser_ties_round_half_away(orc):
+    # Rows whose scale puts x * fl32(127/absmax) exactly on k + 1/2 (and just
+    # below 1/2), where round-half-away and other rules part ways.
+    K = 576
+    X = np.zeros((3, K), np.float16)
+    halves = np.arange(-126.5, 127.0, 1.0)                # absmax 127: inv = 1
+    X[0, :2] = [127, -127]
+    X[0, 2:2 + len(halves)] = halves
+    below = np.nextafter(np.float16(0.5), np.float16(0))  # largest fp16 < 1/2
+    X[0, 300:306] = [below, -below, 0.5, -0.5, np.nextafter(np.float16(1.5), np.float16(0)), -1.5]
+    odd = np.arange(-253, 254, 2)                         # absmax 254: inv = 1/2
+    X[1, :2] = [254, -254]
+    X[1, 2:2 + len(odd)] = odd
+    X[2] = np.linspace(-3.0, 3.0, K).astype(np.float16)   # an ordinary scale
+    out = i8.int8_quantize_activation(to_dev(X), float("inf"))
+    torch.cuda.synchronize()
+    mask_o, _ = orc.outlier_columns(X, float("inf"))
+    Xq_o, sX_o = orc.quantize_rows(X, mask_o)
+    Xq = to_host(out["Xq"])[:3]
+    assert np.array_equal(Xq, Xq_o)
+    assert list(Xq[0, 300:306]) == [0, 0, 1, -1, 1, -2]
+    assert Xq[0, 2] == -127 and Xq[0, 3] == -126 and Xq[0, 2 + 127] == 1    # -126.5, -125.5, 0.5
     assert device_status_clean()
 
 

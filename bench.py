@@ -370,13 +370,19 @@ def run_ours(args, cfg, world, rank, local, pg):
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "peak_src": f"{pk['src']} HBM copy bandwidth"}
     else:
-        peak = 2.0 * pk["bf16_tflops"]
+        # the GEMM is timed inside thousands of back-to-back steps, under the
+        # power cap: the sustained GEMM figure is the matching denominator
+        # (the burst one is reported beside it)
+        burst = 2.0 * pk["bf16_tflops"]
+        sustained = 2.0 * (pk["bf16_tflops_sustained"] or pk["bf16_tflops"])
         achieved = ops / (gemm_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak,
-                "peak_src": f"{pk['src']} bf16 burst x 2 (dense int8 : bf16 nominal ratio 4.5 : 2.25)"}
+        roof = {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
+                "frac": achieved / sustained,
+                "peak_src": f"{pk['src']} bf16 sustained x 2 (dense int8 : bf16 nominal ratio 4.5 : 2.25)",
+                "peak_burst": burst, "frac_of_burst": achieved / burst}
     roof["traffic"] = ncu_traffic(args.workload)
-    roof["kernel"] = "gemm_decode_kernel (split-K GEMM + fused finalisation)" if decode else "gemm_prefill_kernel"
+    roof["kernel"] = ("gemm_decode_kernel (split-K GEMM + fused finalisation)" if decode
+                      else "gemm_prefill_pair_kernel (CTA-pair int8 + fp16 MMA, fused epilogue)")
     roof["kernel_ms"] = gemm_ms
 
     line = {

@@ -53,6 +53,8 @@ def _bind(so):
     so.orc_quantize_rows.restype = None
     so.orc_int8_gemm.argtypes = [_P, _P, _I, _I, _I, _P, _I, _P]
     so.orc_int8_gemm.restype = _I
+    so.orc_dequantize_weight.argtypes = [_P, _P, _I, _I, _P]
+    so.orc_dequantize_weight.restype = None
     so.orc_mixed_linear.argtypes = [_P, _I, _I, _P, _P, _P, _I, _F, _P, _I, _P, _P, _P]
     so.orc_mixed_linear.restype = _I
     return so
@@ -135,12 +137,22 @@ class Oracle:
         return acc
 
     # --- a1..a6 ---
+    def dequantize_weight(self, Wq, sW):
+        """fp16 [K,N]: binary16 RNE of q * fl32(sW/127), the Wq-only variant's outlier rows."""
+        Wq = _c(Wq, np.int8)
+        sW = _c(sW, np.float32)
+        K, N = Wq.shape
+        out = np.empty((K, N), np.uint16)
+        self.so.orc_dequantize_weight(_ptr(Wq), _ptr(sW), K, N, _ptr(out))
+        return out.view(np.float16)
+
     def mixed_linear(self, X, Wq, sW, W16, alpha, rows=None):
-        """Returns (Y fp16 [r,N], Ypre float64 [r,N], acc int32 [r,N], n_outliers)."""
+        """Returns (Y fp16 [r,N], Ypre float64 [r,N], acc int32 [r,N], n_outliers).
+        W16 None: the Wq-only variant (the outlier rows of W are dequantised from Wq)."""
         X = _c(X, np.float16)
         Wq = _c(Wq, np.int8)
         sW = _c(sW, np.float32)
-        W16 = _c(W16, np.float16)
+        W16 = None if W16 is None else _c(W16, np.float16)
         T, K = X.shape
         N = Wq.shape[1]
         rows = _c(np.arange(T) if rows is None else rows, np.int32)
@@ -148,7 +160,7 @@ class Oracle:
         Y = np.empty((R, N), np.uint16)
         Ypre = np.empty((R, N), np.float64)
         acc = np.empty((R, N), np.int32)
-        cnt = self.so.orc_mixed_linear(_ptr(X), T, K, _ptr(Wq), _ptr(sW), _ptr(W16), N,
+        cnt = self.so.orc_mixed_linear(_ptr(X), T, K, _ptr(Wq), _ptr(sW), None if W16 is None else _ptr(W16), N,
                                        float(alpha), _ptr(rows), R, _ptr(Y), _ptr(Ypre), _ptr(acc))
         if cnt < 0:
             raise ArithmeticError("oracle: an int32 accumulator disagreed with its int64 sum")

@@ -32,6 +32,10 @@
  *     before any activation is seen);
  *   - the 16-bit part uses the fp16 W rows; accumulation is int32 for the
  *     8-bit part and (here) double for the 16-bit part and the merge;
+ *   - the variant that keeps only Wq and sW resident (no fp16 weights; the
+ *     memory-halving use of the method [P1 abstract]) takes the outlier rows
+ *     of W dequantised: binary16 RNE of q * fl32(sW / 127), one fp32
+ *     division per column and one fp32 multiply per element;
  *   - Y is rounded to binary16 with round-to-nearest-even.
  *
  * Quantisation decisions are taken in fp32, the precision the CUDA kernels
@@ -250,11 +254,28 @@ int orc_int8_gemm(const int8_t *Xq, const int8_t *Wq, int T, int K, int N,
 }
 
 /* ------------------------------------------------------------------ */
+/* Dequantised weight rows (the Wq-only variant's 16-bit operand).      */
+/* ------------------------------------------------------------------ */
+
+/* W16d[k, n] = binary16 RNE of the fp32 product q * d[n], d[n] = fl32(sW[n] / 127),
+ * for K rows of N columns: the inverse of the weight conversion, rounded to
+ * the 16-bit type the outlier product runs in.  sW[n] = 0 gives zeros. */
+void orc_dequantize_weight(const int8_t *Wq, const float *sW, int K, int N, uint16_t *W16d)
+{
+    for (int k = 0; k < K; ++k)
+        for (int n = 0; n < N; ++n) {
+            float d = sW[n] / 127.0f;                       /* IEEE fp32 division */
+            float v = (float)Wq[(size_t)k * N + n] * d;     /* one fp32 multiply */
+            W16d[(size_t)k * N + n] = orc_double_to_half((double)v);
+        }
+}
+
+/* ------------------------------------------------------------------ */
 /* a1-a6 together: the whole method for a list of rows of Y.            */
 /* ------------------------------------------------------------------ */
 
 /* X [T,K] fp16, Wq [K,N] int8, sW [N], W16 [K,N] fp16 (only its outlier rows
- * are read).  The outlier set is found over ALL T rows (it is a property of
+ * are read; NULL: the Wq-only variant, which dequantises those rows of Wq).  The outlier set is found over ALL T rows (it is a property of
  * the feature dimension, not of one row); rows of Y are then independent, so
  * only the listed rows are computed.  Outputs, per listed row r:
  *   Y[r, n]    binary16 bits of the result,
@@ -285,13 +306,21 @@ int orc_mixed_linear(const uint16_t *X, int T, int K,
         const uint16_t *xrow = X + (size_t)rows[r] * K;
         /* a5: the 16-bit part over the outlier columns, in double */
         double *y16 = (double *)calloc((size_t)N, sizeof(double));
+        uint16_t *wdq = W16 ? NULL : (uint16_t *)malloc((size_t)N * sizeof(uint16_t));
         for (int j = 0; j < count; ++j) {
             int k = idx[j];
             double xv = (double)orc_half_to_float(xrow[k]);
-            const uint16_t *wrow = W16 + (size_t)k * N;
+            const uint16_t *wrow;
+            if (W16) {
+                wrow = W16 + (size_t)k * N;
+            } else {
+                orc_dequantize_weight(Wq + (size_t)k * N, sW, 1, N, wdq);
+                wrow = wdq;
+            }
             for (int n = 0; n < N; ++n)
                 y16[n] += xv * (double)orc_half_to_float(wrow[n]);
         }
+        free(wdq);
         /* a6: dequantise by the outer product of the two scales, then merge */
         for (int n = 0; n < N; ++n) {
             double y = (double)acc[(size_t)r * N + n] * (double)sX[r] * (double)sW[n] / 16129.0

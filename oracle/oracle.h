@@ -26,6 +26,7 @@ void orc_quantize_rows(const uint16_t *X, int T, int K, const uint8_t *is_outlie
                        int8_t *Xq, float *sX);
 int  orc_int8_gemm(const int8_t *Xq, const int8_t *Wq, int T, int K, int N,
                    const int32_t *rows, int nrows, int32_t *acc);
+void orc_dequantize_weight(const int8_t *Wq, const float *sW, int K, int N, uint16_t *W16d);
 int  orc_mixed_linear(const uint16_t *X, int T, int K,
                       const int8_t *Wq, const float *sW, const uint16_t *W16, int N,
                       float alpha, const int32_t *rows, int nrows,

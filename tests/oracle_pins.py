@@ -372,4 +372,91 @@ def pin_golden_worked_example(o):
     assert Y.astype(np.float64).tolist() == g["Y_fp16"]
 
 
+
+# ------------------------------------------------- the Wq-only variant (NEXT-1)
+
+def _grid_weights(rng, K, N):
+    """fp16 weights on the quantisation grid: W[:, n] = q * 2^e[n] with
+    |q| <= 127 and a +-127 in every column, so conversion gives codes q and
+    scale 127 * 2^e[n] exactly (all values are exact in fp16)."""
+    e = rng.integers(-8, 4, size=N)
+    q = rng.integers(-127, 128, size=(K, N))
+    q[rng.integers(0, K, size=N), np.arange(N)] = 127 * rng.choice([-1, 1], size=N)
+    return q, e, (q * 2.0 ** e[None, :]).astype(np.float16)
+
+
+def pin_dequantize_weight_grid(o):
+    """On the grid, sW/127 = 2^e and q * 2^e are exact, so dequantising the
+    converted weight gives it back bit for bit; a zero column stays zero."""
+    rng = np.random.default_rng(11)
+    q, e, W = _grid_weights(rng, 37, 24)
+    W[:, 5] = 0
+    Wq, sW = o.quantize_weight_colwise(W)
+    q[:, 5] = 0
+    assert np.array_equal(Wq.astype(np.int64), q)
+    Wd = o.dequantize_weight(Wq, sW)
+    assert np.array_equal(Wd.view(np.uint16), W.view(np.uint16))
+
+
+def _half_ulp(v):
+    """Half the binary16 spacing at the magnitude of the binary16 value v."""
+    a = abs(float(v))
+    if a < 2.0 ** -14:
+        return 2.0 ** -25
+    return 2.0 ** (math.floor(math.log2(a)) - 11)
+
+
+def pin_dequantize_weight_rounding(o):
+    """Against exact rationals: every dequantised value is within half an fp16
+    ulp of q * sW / 127, plus the fp32 division and product (2^-23 relative
+    each); odd in q and non-decreasing in q for a positive scale."""
+    rng = np.random.default_rng(12)
+    scales = np.concatenate([rng.uniform(1e-3, 3.0, 20), [1e-6, 2.0 ** -14, 0.5, 127.0, 3000.0]]).astype(np.float32)
+    q = np.arange(-127, 128, dtype=np.int8)
+    Wq = np.repeat(q[:, None], len(scales), axis=1)
+    Wd = o.dequantize_weight(Wq, scales)
+    for n, s in enumerate(scales):
+        col = Wd[:, n]
+        for i, qi in enumerate(q):
+            exact = Fraction(int(qi)) * Fraction(float(s)) / 127
+            err = abs(Fraction(float(col[i])) - exact)
+            assert err <= Fraction(_half_ulp(col[i])) + abs(exact) * Fraction(2, 2 ** 22), (float(s), int(qi))
+        assert np.array_equal(col[::-1].astype(np.float64), -col.astype(np.float64))   # q -> -q
+        assert np.all(np.diff(col.astype(np.float64)) >= 0)
+
+
+def pin_wq_only_variant_on_grid(o):
+    """With W16 on the quantisation grid the Wq-only variant is the same
+    computation as the fp16-weight one: identical Y, at every outlier index."""
+    rng = np.random.default_rng(13)
+    T, K, N = 9, 48, 20
+    _, _, W = _grid_weights(rng, K, N)
+    X = rng.standard_normal((T, K)).astype(np.float16)
+    X[:, [4, 17, 40]] = rng.uniform(6.5, 30.0, size=(T, 3)).astype(np.float16)
+    Wq, sW = o.quantize_weight_colwise(W)
+    Y1, P1, _, c1 = o.mixed_linear(X, Wq, sW, W, 6.0)
+    Y2, P2, _, c2 = o.mixed_linear(X, Wq, sW, None, 6.0)
+    assert c1 == c2 >= 3
+    assert np.array_equal(P1, P2) and np.array_equal(Y1.view(np.uint16), Y2.view(np.uint16))
+
+
+def pin_wq_only_variant_error(o):
+    """Off the grid the variants differ only through the outlier rows:
+    |Ypre_wq - Ypre_w16| <= sum over outlier k of |x_k| (sW/254 + half ulp + 2^-22 sW)."""
+    rng = np.random.default_rng(14)
+    T, K, N = 6, 64, 16
+    W = (rng.standard_normal((K, N)) * 0.05).astype(np.float16)
+    X = rng.standard_normal((T, K)).astype(np.float16)
+    cols = [3, 30, 63]
+    X[:, cols] = rng.uniform(7.0, 40.0, size=(T, 3)).astype(np.float16)
+    Wq, sW = o.quantize_weight_colwise(W)
+    _, P1, _, c1 = o.mixed_linear(X, Wq, sW, W, 6.0)
+    _, P2, _, c2 = o.mixed_linear(X, Wq, sW, None, 6.0)
+    assert c1 == c2 == 3
+    xs = np.abs(X[:, cols].astype(np.float64))
+    per_w = sW.astype(np.float64) / 254.0 * (1 + 2.0 ** -20) + 2.0 ** -11 * (np.abs(W[cols].astype(np.float64)) + sW / 254.0)
+    bound = xs @ per_w
+    assert np.all(np.abs(P2 - P1) <= bound * (1 + 1e-9) + 1e-12)
+    assert np.any(P2 != P1)                     # the variant really uses other rows
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -29,7 +29,11 @@ MUTANTS = {
     "weight_scale_per_row": ("float a = fabsf(orc_half_to_float(W16[(size_t)k * N + n]));",
                              "float a = fabsf(orc_half_to_float(W16[(size_t)(n % K) * N + (k % N)]));"),
     "gemm_transposed_weight": ("const int8_t *wrow = Wq + (size_t)k * N;", "const int8_t *wrow = Wq + (size_t)(k % N) * N;"),
-    "outlier_w_row_index": ("const uint16_t *wrow = W16 + (size_t)k * N;", "const uint16_t *wrow = W16 + (size_t)j * N;"),
+    "outlier_w_row_index": ("wrow = W16 + (size_t)k * N;", "wrow = W16 + (size_t)j * N;"),
+    "dequant_scale_128": ("float d = sW[n] / 127.0f;", "float d = sW[n] / 128.0f;"),
+    "dequant_biased": ("float v = (float)Wq[(size_t)k * N + n] * d;", "float v = (float)Wq[(size_t)k * N + n] * d * 0.999f;"),
+    "wq_variant_row_index": ("orc_dequantize_weight(Wq + (size_t)k * N, sW, 1, N, wdq);",
+                             "orc_dequantize_weight(Wq + (size_t)j * N, sW, 1, N, wdq);"),
     "half_subnormal_exponent": ("mag = ldexp((double)frac, -24);", "mag = ldexp((double)frac, -25);"),
     "y_round_truncate": ("if (diff > 0.5) return fl + 1.0;", "if (diff > 2.0) return fl + 1.0;"),
     "scale_x_instead_of_w": ("* (double)sX[r] * (double)sW[n]", "* (double)sX[r] * (double)sX[r]"),

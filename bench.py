@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="input sets rotated between steps (default 3: operands not in L2)")
+    ap.add_argument("--variant", default="w16", choices=["w16", "wq"],
+                    help="w16: int8_mixed_linear (fp16 weight resident for the outlier rows); "
+                         "wq: int8_mixed_linear_wq (only Wq and sW resident)")
     return ap.parse_args()
 
 
@@ -59,10 +62,13 @@ def all_configs():
     return c
 
 
-def work(cfg, n_out):
+def work(cfg, n_out, variant="w16"):
+    """Effective ops and algorithmic weight bytes of one call: Wq, sW and the
+    outlier rows actually read (fp16 rows of W16, or int8 rows of Wq again
+    for the Wq-only variant)."""
     T, K, N = cfg["T"], cfg["K"], cfg["N"]
     ops = 2.0 * T * K * N
-    weight_bytes = K * N + 4 * N + 2 * n_out * N
+    weight_bytes = K * N + 4 * N + (1 if variant == "wq" else 2) * n_out * N
     return ops, weight_bytes
 
 
@@ -191,7 +197,7 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
-def oracle_sample(cfg, X, W, target_s=15.0, orc_state=None):
+def oracle_sample(cfg, X, W, target_s=15.0, orc_state=None, variant="w16"):
     """Time the oracle on a bounded, seeded sample of the workload: a sub-batch
     of R rows of X (the whole method, outlier scan included, on those R
     tokens) against the first C columns of the weight (a column slice is the
@@ -213,7 +219,7 @@ def oracle_sample(cfg, X, W, target_s=15.0, orc_state=None):
         Wqs, sWs, Ws = (np.ascontiguousarray(Wq[:, :C]), np.ascontiguousarray(sW[:C]),
                         np.ascontiguousarray(W[:, :C]))
         t0 = time.perf_counter()
-        orc.mixed_linear(Xs, Wqs, sWs, Ws, cfg["alpha"])
+        orc.mixed_linear(Xs, Wqs, sWs, None if variant == "wq" else Ws, cfg["alpha"])
         return time.perf_counter() - t0
 
     R, C = min(T, threads), N
@@ -235,7 +241,7 @@ def run_reference(args, cfg, world, rank, pg):
     X, W = wl.generate(cfg)
     T, K, N = cfg["T"], cfg["K"], cfg["N"]
     per_step = 100.0 / max(1, args.steps + args.warmup)          # whole run ~2 minutes
-    _, R, C, _, cores, state, run = oracle_sample(cfg, X, W, target_s=min(per_step, 15.0))
+    _, R, C, _, cores, state, run = oracle_sample(cfg, X, W, target_s=min(per_step, 15.0), variant=args.variant)
     times = []
     for i in range(args.warmup + args.steps):
         dt = run(R, C)
@@ -251,7 +257,7 @@ def run_reference(args, cfg, world, rank, pg):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
         "data": "synthetic, seeded", "config": {"workload": args.workload, "T": T, "K": K, "N": N,
-                                                "alpha": cfg["alpha"]},
+                                                "alpha": cfg["alpha"], "variant": args.variant},
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -282,21 +288,30 @@ def run_ours(args, cfg, world, rank, local, pg):
         Xd = torch.from_numpy(X).to(dev)
         Wd = torch.from_numpy(W).to(dev)
         Wq, sW = i8.int8_quantize_weight_colwise(Wd)
+        if args.variant == "wq":
+            torch.cuda.synchronize()
+            Wd = None                   # only Wq and sW stay resident
         sets.append((Xd, Wq, sW, Wd))
         host_x.append(torch.from_numpy(X).pin_memory())
     Y = torch.empty((T, N), dtype=torch.float16, device=dev)
     Y_host = torch.empty((T, N), dtype=torch.float16).pin_memory()
-    ws = i8.workspace(T, K, N, dev)
+    if args.variant == "wq":
+        ws = torch.empty(max(1, i8.int8_mixed_linear_wq_workspace_size(T, K, N)), dtype=torch.uint8, device=dev)
+    else:
+        ws = i8.workspace(T, K, N, dev)
     torch.cuda.synchronize()
 
     stats = i8.int8_outlier_stats(sets[0][0], alpha)
     n_out = int(stats[0].item())
     frac8 = float(stats[3].item())
-    ops, wbytes = work(cfg, n_out)
+    ops, wbytes = work(cfg, n_out, args.variant)
 
     def step(i):
         Xd, Wq, sW, Wd = sets[i % nrot]
-        i8.int8_mixed_linear(Xd, Wq, sW, Wd, alpha, Y=Y, workspace_buf=ws)
+        if Wd is None:
+            i8.int8_mixed_linear_wq(Xd, Wq, sW, alpha, Y=Y, workspace_buf=ws)
+        else:
+            i8.int8_mixed_linear(Xd, Wq, sW, Wd, alpha, Y=Y, workspace_buf=ws)
 
     for i in range(args.warmup):
         step(i)
@@ -380,7 +395,7 @@ def run_ours(args, cfg, world, rank, local, pg):
                 "frac": achieved / sustained,
                 "peak_src": f"{pk['src']} bf16 sustained x 2 (dense int8 : bf16 nominal ratio 4.5 : 2.25)",
                 "peak_burst": burst, "frac_of_burst": achieved / burst}
-    roof["traffic"] = ncu_traffic(args.workload)
+    roof["traffic"] = ncu_traffic(args.workload) if args.variant == "w16" else None
     roof["kernel"] = ("gemm_decode_kernel (split-K GEMM + fused finalisation)" if decode
                       else "gemm_prefill_pair_kernel (CTA-pair int8 + fp16 MMA, fused epilogue)")
     roof["kernel_ms"] = gemm_ms
@@ -393,7 +408,10 @@ def run_ours(args, cfg, world, rank, local, pg):
         "config": {"workload": args.workload, "T": T, "K": K, "N": N, "alpha": alpha, "outlier_cols": n_out,
                    "frac_8bit": frac8, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": f"{nrot} rotating input sets" + (" (each step's operands not in L2)" if nrot >= 3 else
-                                                          " (operands may be partly L2-resident)")},
+                                                          " (operands may be partly L2-resident)"),
+                   "variant": ("wq-only: outlier rows dequantised from Wq, no fp16 weight resident"
+                               if args.variant == "wq" else "w16: fp16 weight rows for the outliers"),
+                   "resident_weight_bytes": K * N + 4 * N + (0 if args.variant == "wq" else 2 * K * N)},
         "weight_gbs": world * wbytes / (ms_step * 1e-3) / 1e9,
         "roofline": roof,
         "e2e": {"value": e_value, "unit": "TOPS", "h2d_bytes_per_step": 2 * T * K,
@@ -403,7 +421,7 @@ def run_ours(args, cfg, world, rank, local, pg):
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tops, R, C, dt, cores, _, _ = oracle_sample(cfg, X0, W0)
+        tops, R, C, dt, cores, _, _ = oracle_sample(cfg, X0, W0, variant=args.variant)
         line["cpu_baseline"] = {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
                                 "sample": f"sub-batch of {R} of {T} rows x {C} of {N} columns ({dt:.1f} s, "
                                           f"whole method incl. outlier scan); weight conversion untimed"}

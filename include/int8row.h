@@ -70,6 +70,9 @@ typedef enum {
 #define I8R_DEV_OK 0
 #define I8R_DEV_PIPELINE_TIMEOUT 1   /* a shared-memory pipeline wait gave up */
 #define I8R_DEV_TMEM_TIMEOUT 2       /* a tensor-memory hand-off wait gave up */
+#define I8R_DEV_OUTLIER_CAP 3        /* int8_mixed_linear_wq found more outlier columns
+                                        than its workspace holds rows for; Y lacks the
+                                        16-bit part of the excess columns */
 
 /* ---------------------------------------------------------------------------
  * Weight conversion.  The pages describe a 16/32-bit checkpoint converted to
@@ -111,6 +114,33 @@ i8r_status int8_mixed_linear(const void *X, int T, int K,
                              float alpha, void *Y,
                              void *workspace, size_t workspace_bytes,
                              cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * int8_mixed_linear_wq: the same layer with only Wq and sW resident.  The
+ * fp16 weight need not be kept, which is the memory-halving use of the method
+ * (LLM.int8() abstract).  The 16-bit part multiplies X[:,O] by the outlier
+ * rows of W dequantised from the int8 codes:
+ *   W~[k,n] = fp16_rn( Wq[k,n] * fl32(sW[n] / 127) )
+ * (one fp32 division per column, one fp32 multiply, round to nearest even),
+ * so Y = fp16( acc*sX[t]*sW[n]/127^2 + X[:,O] W~[O,:] ).
+ * Arguments, layouts and workspace rules are those of int8_mixed_linear,
+ * with workspace of at least int8_mixed_linear_wq_workspace_size(T, K, N)
+ * bytes.  For T > 128 that workspace holds the dequantised rows of at most
+ * int8_mixed_linear_wq_max_outliers(K) outlier columns (at least 256 and
+ * 1/16 of K, rounded up to a multiple of 64, and not more than K rounded
+ * up to 64).  A call that finds more outlier columns than that sets
+ * I8R_DEV_OUTLIER_CAP in the device status word, and its Y lacks the 16-bit
+ * part of the excess columns.  T <= 128 has no such limit.
+ * ------------------------------------------------------------------------- */
+size_t int8_mixed_linear_wq_workspace_size(int T, int K, int N);
+
+int int8_mixed_linear_wq_max_outliers(int K);
+
+i8r_status int8_mixed_linear_wq(const void *X, int T, int K,
+                                const int8_t *Wq, const float *sW, int N,
+                                float alpha, void *Y,
+                                void *workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * int8_mixed_linear_noalloc: the same layer, with no workspace argument and no

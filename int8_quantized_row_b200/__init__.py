@@ -13,6 +13,7 @@ import os
 __all__ = [
     "lib", "I8RError",
     "int8_quantize_weight_colwise", "int8_mixed_linear_workspace_size", "int8_mixed_linear",
+    "int8_mixed_linear_wq_workspace_size", "int8_mixed_linear_wq_max_outliers", "int8_mixed_linear_wq",
     "int8_outlier_stats_workspace_size", "int8_outlier_stats", "int8_quantize_activation",
     "int8_gemm_i8_s32", "int8_read_and_clear_device_status", "int8_status_string",
     "int8_selftest_wait_timeout",
@@ -52,6 +53,11 @@ def lib():
     so.int8_mixed_linear_workspace_size.argtypes = [_I, _I, _I]
     so.int8_mixed_linear_workspace_size.restype = _Z
     so.int8_mixed_linear.argtypes = [_P, _I, _I, _P, _P, _P, _I, _F, _P, _P, _Z, _P]
+    so.int8_mixed_linear_wq_workspace_size.argtypes = [_I, _I, _I]
+    so.int8_mixed_linear_wq_workspace_size.restype = _Z
+    so.int8_mixed_linear_wq_max_outliers.argtypes = [_I]
+    so.int8_mixed_linear_wq_max_outliers.restype = _I
+    so.int8_mixed_linear_wq.argtypes = [_P, _I, _I, _P, _P, _I, _F, _P, _P, _Z, _P]
     so.int8_outlier_stats_workspace_size.argtypes = [_I]
     so.int8_outlier_stats_workspace_size.restype = _Z
     so.int8_outlier_stats.argtypes = [_P, _I, _I, _F, _P, _P, _P, _P, _P, _Z, _P]
@@ -133,6 +139,31 @@ def int8_mixed_linear(X, Wq, sW, W16, alpha=6.0, Y=None, workspace_buf=None, str
     _check("int8_mixed_linear", lib().int8_mixed_linear(
         _dev(X, torch.float16, "X", 2), T, K, _dev(Wq, torch.int8, "Wq", 2), _dev(sW, torch.float32, "sW"),
         _dev(W16, torch.float16, "W16", 2), N, float(alpha), _dev(Y, torch.float16, "Y"),
+        ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(), _stream(stream)))
+    return Y
+
+
+def int8_mixed_linear_wq_workspace_size(T, K, N):
+    return int(lib().int8_mixed_linear_wq_workspace_size(int(T), int(K), int(N)))
+
+
+def int8_mixed_linear_wq_max_outliers(K):
+    return int(lib().int8_mixed_linear_wq_max_outliers(int(K)))
+
+
+def int8_mixed_linear_wq(X, Wq, sW, alpha=6.0, Y=None, workspace_buf=None, stream=None):
+    """Y fp16 [T,N] = the Wq-only variant: the outlier rows of W are dequantised from (Wq, sW)."""
+    import torch
+    T, K = X.shape
+    N = Wq.shape[1]
+    Y = torch.empty((T, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    if workspace_buf is None:
+        workspace_buf = torch.empty(max(1, int8_mixed_linear_wq_workspace_size(T, K, N)), dtype=torch.uint8,
+                                    device=X.device)
+    ws = workspace_buf
+    _check("int8_mixed_linear_wq", lib().int8_mixed_linear_wq(
+        _dev(X, torch.float16, "X", 2), T, K, _dev(Wq, torch.int8, "Wq", 2), _dev(sW, torch.float32, "sW"),
+        N, float(alpha), _dev(Y, torch.float16, "Y"),
         ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(), _stream(stream)))
     return Y
 

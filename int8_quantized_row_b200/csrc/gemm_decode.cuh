@@ -52,7 +52,8 @@ struct Params {
     const float *sX, *sW;
     const __half *Xo;              // [T,K] fp16, |O| valid columns
     const int32_t *idx, *count;
-    const __half *W16;
+    const __half *W16;             // outlier rows of the fp16 weight, or null:
+    const int8_t *Wq;              // then those rows are dequantised from Wq and sW
     __half *Y;
 };
 
@@ -92,6 +93,15 @@ constexpr int FIN_OUT = 8;
 __device__ __forceinline__ void finalize_columns(const Params &p, int tile, int quad, int lane, float *xo_s) {
     const int count = *p.count;
     const int nbase = tile * BM + quad * 32 + lane;
+    // Wq-only: W~[k,n] = fp16_rn(q * fl32(sW[n]/127)) for this lane's two columns
+    float dq[2] = {0.0f, 0.0f};
+    if (!p.W16) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int n = nbase + h * BMH;
+            if (n < p.N) dq[h] = __fdiv_rn(p.sW[n], 127.0f);
+        }
+    }
     for (int t0 = 0; t0 < p.T; t0 += FIN_ROWS) {
         float o[2][FIN_ROWS];
 #pragma unroll
@@ -115,7 +125,13 @@ __device__ __forceinline__ void finalize_columns(const Params &p, int tile, int 
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int n = nbase + h * BMH;
-                    w[h][jj] = (k >= 0 && n < p.N) ? __half2float(p.W16[static_cast<size_t>(k) * p.N + n]) : 0.0f;
+                    float wv = 0.0f;
+                    if (k >= 0 && n < p.N) {
+                        const size_t at = static_cast<size_t>(k) * p.N + n;
+                        wv = p.W16 ? __half2float(p.W16[at])
+                                   : __half2float(__float2half_rn(__fmul_rn(static_cast<float>(p.Wq[at]), dq[h])));
+                    }
+                    w[h][jj] = wv;
                 }
             }
             __syncwarp();

@@ -73,6 +73,7 @@ struct Params {
     __half *Y;
     int32_t *acc_out;
     int o_rows;                    // outlier rows compacted into the W16o map (multiple of 64)
+    int wq_only;                   // no W16 map: blocks past o_rows read zeros (flagged upstream)
 };
 
 struct Barriers {
@@ -227,16 +228,18 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const int left = count - blk * OBK;
                     const bool compact = blk * OBK + OBK <= p.o_rows;
                     const int rows = compact ? OBK : min(OBK, (left + 15) / 16 * 16);
-                    if (!compact)
+                    if (!compact && !p.wq_only)
                         for (int j = lane; j < rows; j += 32) bars->orow[j] = j < left ? p.idx[blk * OBK + j] : p.K;
                     __syncwarp();
-                    if (lane == 0 && compact) {
+                    if (lane == 0 && (compact || p.wq_only)) {
+                        // Wq-only past the compacted rows: an out-of-range box of W16o, i.e. zeros
+                        const int y = compact ? blk * OBK : p.o_rows;
                         if (leader)
                             mbar_arrive_expect_tx(&bars->full[stage], 2u * static_cast<uint32_t>(XO_BYTES + OBK * 256));
                         const uint32_t fb = lead_full + 8u * stage;
                         tma_load_2d_pair(a, &map_xo, fb, blk * OBK, m0);
-                        tma_load_2d_pair(a + A_BYTES, &map_w16o, fb, n0, blk * OBK);
-                        tma_load_2d_pair(a + A_BYTES + B_CHUNK_F16, &map_w16o, fb, n0 + 64, blk * OBK);
+                        tma_load_2d_pair(a + A_BYTES, &map_w16o, fb, n0, y);
+                        tma_load_2d_pair(a + A_BYTES + B_CHUNK_F16, &map_w16o, fb, n0 + 64, y);
                     } else if (lane == 0) {
                         if (leader)
                             mbar_arrive_expect_tx(&bars->full[stage], 2u * static_cast<uint32_t>(XO_BYTES + rows * 256));

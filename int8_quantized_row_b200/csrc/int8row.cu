@@ -198,10 +198,17 @@ struct Workspace {
     size_t count, mask, idx, sX, Xq, Xo, W16o, acc32, counters, total;
 };
 
-// Rows of the compacted outlier weight rows kept for the prefill GEMM.
-inline int compact_rows(int K) { return std::min((K + 63) / 64 * 64, kCompactOutlierRows); }
+// Rows of the compacted outlier weight rows kept for the prefill GEMM: 256
+// with W16 (past them the GEMM gathers W16 rows itself); for the Wq-only
+// variant, which has no other source, at least 256 and K/16 (rounded up to
+// 64), at most K rounded up to 64.
+inline int compact_rows(int K, bool wq_only = false) {
+    const int all = (K + 63) / 64 * 64;
+    if (!wq_only) return std::min(all, kCompactOutlierRows);
+    return std::min(all, std::max(kCompactOutlierRows, ((K + 15) / 16 + 63) / 64 * 64));
+}
 
-Workspace ws_layout(int T, int K, int N) {
+Workspace ws_layout(int T, int K, int N, bool wq_only = false) {
     Workspace w{};
     size_t off = 0;
     w.count = off; off = align_up(off + sizeof(int32_t));
@@ -211,7 +218,7 @@ Workspace ws_layout(int T, int K, int N) {
     w.Xq = off;    off = align_up(off + static_cast<size_t>(T) * K);
     w.Xo = off;    off = align_up(off + static_cast<size_t>(T) * K * 2);
     w.W16o = off;
-    if (T > decode::MAX_T) off = align_up(off + static_cast<size_t>(compact_rows(K)) * N * 2);
+    if (T > decode::MAX_T) off = align_up(off + static_cast<size_t>(compact_rows(K, wq_only)) * N * 2);
     w.acc32 = off;
     w.counters = off;
     if (T <= decode::MAX_T) {
@@ -273,11 +280,12 @@ dim3 scan_grid(int T, int K, int sms, int *rows_per_block) {
 // a1-a3 on the stream: mask, row quantisation, index list and gather.
 // `zero` / `zero_bytes`: a region the scan clears on the way (may be null).
 // With W16o, the quantiser's launch also compacts the W16 rows of the first
-// compact_rows(K) outlier columns into W16o ([compact_rows(K), N]).
+// compact_rows(K) outlier columns into W16o ([compact_rows(K), N]); with W16
+// null (the Wq-only variant) it dequantises those rows of Wq instead.
 i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int K, float alpha, uint32_t *mask,
                              int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
                              size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
-                             __half *W16o = nullptr) {
+                             __half *W16o = nullptr, const int8_t *Wq = nullptr, const float *sW = nullptr) {
     const int nwords = (K + 31) / 32;
     clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords);
     I8R_LAUNCHED();
@@ -298,19 +306,20 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     I8R_LAUNCHED();
     // row 0's block of the quantiser publishes the index list and |O|
     const int rt = row_threads(K);
-    const int o_rows = W16o ? compact_rows(K) : 0;
+    const int o_rows = W16o ? compact_rows(K, W16 == nullptr) : 0;
     const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
     const size_t smem = quantize_smem_bytes(K);
     const uint32_t *m = mask;
     uint32_t *no_mask_out = nullptr;
     if (rt == 64)
-        e = launch_rows<64>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, N, W16o, o_rows, G);
+        e = launch_rows<64>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N, W16o,
+                            o_rows, G);
     else if (rt == 128)
-        e = launch_rows<128>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, N, W16o, o_rows,
-                             G);
+        e = launch_rows<128>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N, W16o,
+                             o_rows, G);
     else
-        e = launch_rows<256>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, N, W16o, o_rows,
-                             G);
+        e = launch_rows<256>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N, W16o,
+                             o_rows, G);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;
@@ -391,19 +400,23 @@ void record_after(cudaStream_t s) {
     CUtensorMap map_xq, map_wq, map_xo, map_w16, map_w16x4, map_w16o, map_y;
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, 128, prefill2::A_BOX_K));
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, prefill2::BK, 128));
+    const bool wq_only = Xo && !W16;
     if (Xo) {
         I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, 128, prefill2::OBK));
+    } else {
+        map_xo = map_xq;   // unused: no 16-bit part
+    }
+    if (Xo && W16) {
         // 64-column pieces of W16 rows: one-row box (also the gather map), and
         // a four-row box for the zero padding
         I8R_TRY(make_map(&map_w16, W16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, N, 1, 64));
         I8R_TRY(make_map(&map_w16x4, W16, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, N, 4, 64));
     } else {
-        map_xo = map_xq;   // unused: no 16-bit part
-        map_w16 = map_xq;
+        map_w16 = map_xq;  // unused: no W16 (int32 output mode, or the Wq-only variant)
         map_w16x4 = map_xq;
     }
     // compacted outlier rows: 64 x 64 boxes
-    const int o_rows = (Xo && W16o) ? compact_rows(K) : 0;
+    const int o_rows = (Xo && W16o) ? compact_rows(K, wq_only) : 0;
     if (o_rows > 0) {
         I8R_TRY(make_map(&map_w16o, W16o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, o_rows, N, 64, 64));
     } else {
@@ -431,6 +444,7 @@ void record_after(cudaStream_t s) {
     p.Y = Y;
     p.acc_out = acc_out;
     p.o_rows = o_rows;
+    p.wq_only = wq_only ? 1 : 0;
     const int clusters = p.num_tiles < dev->pair_clusters ? p.num_tiles : dev->pair_clusters;
     record_before(s);
     cudaError_t e;
@@ -576,17 +590,24 @@ size_t int8_mixed_linear_workspace_size(int T, int K, int N) {
     return ws_layout(T, K, N).total;
 }
 
-i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, const float *sW, const void *W16, int N,
+namespace {
+
+// int8_mixed_linear and its Wq-only variant (W16 null).
+i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, const float *sW, const void *W16, int N,
                              float alpha, void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    const bool wq_only = W16 == nullptr;
     I8R_TRY(check_shape(T, K, N, true));
     if (std::isnan(alpha) || alpha < 0.0f) return I8R_EINVAL;
     if (T == 0) return I8R_OK;
     I8R_TRY(check_ptr(X));
     I8R_TRY(check_ptr(Wq));
     I8R_TRY(check_ptr(sW));
-    I8R_TRY(check_ptr(W16));
+    if (!wq_only) I8R_TRY(check_ptr(W16));
     I8R_TRY(check_ptr(Y));
-    const Workspace w = ws_layout(T, K, N);
+#if !I8R_PREFILL_PAIR
+    if (wq_only && T > decode::MAX_T) return I8R_EARCH;      // the one-CTA GEMM needs W16
+#endif
+    const Workspace w = ws_layout(T, K, N, wq_only);
     if (!workspace || workspace_bytes < w.total) return I8R_EWORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return I8R_EALIGN;
     const DeviceInfo *dev = nullptr;
@@ -614,7 +635,7 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
     __half *W16o = nullptr;        // the single-CTA GEMM gathers the rows itself
 #endif
     I8R_TRY(launch_activation(dev, x, T, K, alpha, mask, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
-                              zero_bytes, stream, w16, N, W16o));
+                              zero_bytes, stream, w16, N, W16o, Wq, sW));
     if (!small_t)
         return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream, W16o);
 
@@ -626,8 +647,29 @@ i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, cons
     fin.idx = idx;
     fin.count = count;
     fin.W16 = w16;
+    fin.Wq = Wq;
     fin.Y = y;
     return launch_decode(dev, Xq, T, K, Wq, N, acc32, &fin, stream);
+}
+
+}  // namespace
+
+i8r_status int8_mixed_linear(const void *X, int T, int K, const int8_t *Wq, const float *sW, const void *W16, int N,
+                             float alpha, void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!W16) return I8R_EINVAL;
+    return mixed_linear_impl(X, T, K, Wq, sW, W16, N, alpha, Y, workspace, workspace_bytes, stream);
+}
+
+size_t int8_mixed_linear_wq_workspace_size(int T, int K, int N) {
+    if (T < 0 || K < 0 || N < 0) return 0;
+    return ws_layout(T, K, N, true).total;
+}
+
+int int8_mixed_linear_wq_max_outliers(int K) { return K < 0 ? 0 : compact_rows(K, true); }
+
+i8r_status int8_mixed_linear_wq(const void *X, int T, int K, const int8_t *Wq, const float *sW, int N, float alpha,
+                                void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return mixed_linear_impl(X, T, K, Wq, sW, nullptr, N, alpha, Y, workspace, workspace_bytes, stream);
 }
 
 size_t int8_mixed_linear_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }

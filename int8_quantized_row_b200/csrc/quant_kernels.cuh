@@ -315,14 +315,19 @@ inline size_t quantize_smem_bytes(int K) { return static_cast<size_t>((K + 31) /
 // The W16 rows of the first o_rows outlier columns, compacted for the
 // prefill GEMM (its outlier stages then load two 64 x 64 boxes each instead
 // of gathering rows):  W16o[j,:] = W16[O_j,:] for j < |O|, zero rows up to the
-// next multiple of 64 (at most o_rows).  Block e of the G compaction blocks
-// copies rows e, e+G, ... with eight 16-byte loads in flight per thread.
+// next multiple of 64 (at most o_rows).  Without W16 (the Wq-only variant) the
+// rows are dequantised instead, W16o[j,n] = fp16_rn(Wq[O_j,n] * fl32(sW[n]/127)),
+// and more than o_rows outlier columns is reported (I8R_DEV_OUTLIER_CAP).
+// Block e of the G compaction blocks copies rows e, e+G, ... with eight
+// 16-byte stores in flight per thread.
 constexpr int kCompactOutlierRows = 256;
 
 template <int kThreads>
 __device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *smask, const int *spre, int w0, int w1,
-                                                           int total, const __half *__restrict__ W16, int N,
-                                                           __half *__restrict__ W16o, int o_rows, int e, int G) {
+                                                           int total, const __half *__restrict__ W16,
+                                                           const int8_t *__restrict__ Wq, const float *__restrict__ sW,
+                                                           int N, __half *__restrict__ W16o, int o_rows, int e, int G) {
+    if (!W16 && total > o_rows && e == 0 && threadIdx.x == 0) report_status(I8R_DEV_OUTLIER_CAP);
     __shared__ int oidx[kCompactOutlierRows];
     for (int w = w0; w < w1; ++w) {
         int j = spre[w];
@@ -338,6 +343,27 @@ __device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *smask
     constexpr int kBatch = 8;
     for (int r = e; r < rows; r += G) {
         uint4 *dst = reinterpret_cast<uint4 *>(W16o + static_cast<size_t>(r) * N);
+        if (!W16) {
+            // dequantised rows: 8 codes and 8 column scales per 16-byte store
+            const uint2 *q8 = r < total ? reinterpret_cast<const uint2 *>(Wq + static_cast<size_t>(oidx[r]) * N) : nullptr;
+            for (int c = static_cast<int>(threadIdx.x); c < vec; c += kThreads) {
+                Vec16 v;
+                v.u = make_uint4(0u, 0u, 0u, 0u);
+                if (q8) {
+                    const uint2 qq = __ldg(q8 + c);
+                    const float4 s0 = __ldg(reinterpret_cast<const float4 *>(sW) + 2 * c);
+                    const float4 s1 = __ldg(reinterpret_cast<const float4 *>(sW) + 2 * c + 1);
+                    const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int q = static_cast<int8_t>(((i < 4 ? qq.x : qq.y) >> (8 * (i & 3))) & 0xFFu);
+                        v.h[i] = __float2half_rn(__fmul_rn(static_cast<float>(q), __fdiv_rn(sc[i], 127.0f)));
+                    }
+                }
+                dst[c] = v.u;
+            }
+            continue;
+        }
         const uint4 *src = r < total ? reinterpret_cast<const uint4 *>(W16 + static_cast<size_t>(oidx[r]) * N) : nullptr;
         for (int c0 = static_cast<int>(threadIdx.x); c0 < vec; c0 += kThreads * kBatch) {
             uint4 v[kBatch];
@@ -386,8 +412,9 @@ template <int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ parts, int nparts,
     float *__restrict__ sX, int8_t *__restrict__ Xq, __half *__restrict__ Xo, uint32_t *__restrict__ mask_out,
-    int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out, const __half *__restrict__ W16, int N,
-    __half *__restrict__ W16o, int o_rows, int G) {
+    int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out, const __half *__restrict__ W16,
+    const int8_t *__restrict__ Wq, const float *__restrict__ sW, int N, __half *__restrict__ W16o, int o_rows,
+    int G) {
     constexpr int kWarps = kRowThreads / 32;
     extern __shared__ uint32_t qs[];
     __shared__ float red[kWarps];
@@ -446,7 +473,7 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     }
     __syncthreads();
     if (t < 0) {
-        gather_outlier_weight_rows<kRowThreads>(smask, spre, w0, w1, total, W16, N, W16o, o_rows,
+        gather_outlier_weight_rows<kRowThreads>(smask, spre, w0, w1, total, W16, Wq, sW, N, W16o, o_rows,
                                                 static_cast<int>(blockIdx.x), G);
         return;
     }

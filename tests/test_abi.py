@@ -78,6 +78,31 @@ def test_host_rejects_bad_shapes_before_any_launch(so):
     assert f(*args(0, 1024, 1024)) == 0           # T == 0: a no-op
 
 
+def test_wq_variant_host_checks_and_capacity(so):
+    f = so.int8_mixed_linear_wq
+    ws = so.int8_mixed_linear_wq_workspace_size(16, 1024, 1024)
+    args = lambda T, K, N, alpha=6.0, x=_p(), wsb=ws: (x, T, K, _p(), _p(), N, alpha, _p(), _p(), wsb, _null())
+    assert f(*args(16, 1000, 1024)) == 2          # K % 16
+    assert f(*args(16, 133152, 1024)) == 3
+    assert f(*args(16, 1024, 1024, alpha=float("nan"))) == 1
+    assert f(*args(16, 1024, 1024, x=_null())) == 1
+    assert f(*args(16, 1024, 1024, wsb=ws - 1)) == 4
+    assert f(*args(0, 1024, 1024)) == 0
+    # the plain entry point still needs W16
+    g = so.int8_mixed_linear
+    assert g(_p(), 16, 1024, _p(), _p(), _null(), 1024, 6.0, _p(), _p(),
+             so.int8_mixed_linear_workspace_size(16, 1024, 1024), _null()) == 1
+    # rows of dequantised outlier weights the prefill workspace holds:
+    # at least 256 and K/16, rounded up to 64, at most K rounded up to 64
+    cap = so.int8_mixed_linear_wq_max_outliers
+    assert [cap(k) for k in (16, 64, 1024, 5120, 12288, 49152)] == [64, 64, 256, 320, 768, 3072]
+    # the workspace holds exactly those rows on top of the plain one (prefill), none at decode
+    for T, K, N in ((2048, 12288, 49152), (300, 1024, 512)):
+        extra = so.int8_mixed_linear_wq_workspace_size(T, K, N) - so.int8_mixed_linear_workspace_size(T, K, N)
+        assert extra == (cap(K) - min(256, (K + 63) // 64 * 64)) * N * 2
+    assert so.int8_mixed_linear_wq_workspace_size(16, 12288, 49152) == so.int8_mixed_linear_workspace_size(16, 12288, 49152)
+
+
 def test_host_rejects_bad_weight_conversion(so):
     f = so.int8_quantize_weight_colwise
     assert f(_p(), 1024, 1000, _p(), _p(), _null()) == 2

@@ -12,12 +12,19 @@
 // tile in TMEM (double-buffered) and adds the exact int32 partial sums into
 // acc32 [T,N] (zeroed beforehand) with red.add.
 //
-// Finalisation without waiting: after adding its partial sums, each epilogue
-// warp bumps a counter for its (tile, 32-lane quadrant).  The warp that
-// brings the counter to the number of CTAs covering the tile knows every
-// partial sum has landed; it applies the scales and the 16-bit outlier part
-//   Y[t,n] = fp16( acc32[t,n] * sX[t] * sW[n] / 127^2 + sum_j Xo[t,j] W16[O_j,n] )
-// for its 64 columns.  No CTA ever waits on another.
+// The 16-bit outlier part Yo[t,n] = sum_j X[t,O_j] W16[O_j,n] (fp32) comes
+// from the row quantiser's launch (its outlier-product blocks), which this
+// kernel waits for with griddepcontrol.wait like the rest of the activation.
+//
+// Finalisation: after adding its partial sums, each epilogue warp bumps a
+// counter for its (tile, 32-lane quadrant).  The warp that brings the counter
+// to the number of CTAs covering the tile knows every partial sum has landed;
+// it writes
+//   Y[t,n] = fp16( acc32[t,n] * sX[t] * sW[n] / 127^2 + Yo[t,n] )
+// for its 64 columns.  No CTA ever waits on another.  (Stream-K leaves most
+// tiles split between the end of one CTA's range and the start of the next,
+// so these finalisations run in the kernel's tail, which is why they do no
+// more than combine two loaded values per output.)
 //
 // Launched as a programmatic dependent of the activation kernels: the weight
 // tiles of the first stages are requested before griddepcontrol.wait, since
@@ -50,11 +57,9 @@ struct Params {
     int finalize;
     int32_t *counters;             // [num_tiles * 4], zero on entry
     const float *sX, *sW;
-    const __half *Xo;              // [T,K] fp16, |O| valid columns
-    const int32_t *idx, *count;
-    const __half *W16;             // outlier rows of the fp16 weight, or null:
-    const int8_t *Wq;              // then those rows are dequantised from Wq and sW
+    const int32_t *count;
     __half *Y;
+    const float *Yo;               // [T,N] fp32: the 16-bit outlier part (read when |O| > 0)
 };
 
 struct Barriers {
@@ -67,10 +72,8 @@ struct Barriers {
     int abort;
 };
 
-constexpr int FIN_SCRATCH_BYTES = 4 * 16 * 8 * 4;   // 16 x 8 floats per epilogue warp
-
 __host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes) {
-    return 1024 + static_cast<size_t>(stages) * stage_bytes + sizeof(Barriers) + FIN_SCRATCH_BYTES;
+    return 1024 + static_cast<size_t>(stages) * stage_bytes + sizeof(Barriers);
 }
 
 // CTA c of `ctas` owns units [floor(c*U/ctas), floor((c+1)*U/ctas)).
@@ -82,84 +85,34 @@ __device__ __forceinline__ int unit_owner(long long total, long long u, int ctas
     return static_cast<int>(((u + 1) * ctas - 1) / total);
 }
 
-// Y for the columns of one finished (tile, quadrant): lane l owns columns
-// n0 + 32*quad + l and n0 + 128 + 32*quad + l.  Rows go in groups of 16 and
-// the outlier columns in chunks of 8, so each lane keeps 8 independent W16
-// loads and 16 accumulator loads in flight instead of a chain of dependent
-// loads.  `xo_s` is this warp's scratch of 16 x 8 floats.
 constexpr int FIN_ROWS = 16;
-constexpr int FIN_OUT = 8;
 
-__device__ __forceinline__ void finalize_columns(const Params &p, int tile, int quad, int lane, float *xo_s) {
-    const int count = *p.count;
+// Y for the columns of one finished (tile, quadrant), from the int32 sums and
+// (with outliers) Yo; 16 rows at a time with all loads of a group in flight.
+__device__ __forceinline__ void finalize_columns(const Params &p, int tile, int quad, int lane, int count) {
     const int nbase = tile * BM + quad * 32 + lane;
-    // Wq-only: W~[k,n] = fp16_rn(q * fl32(sW[n]/127)) for this lane's two columns
-    float dq[2] = {0.0f, 0.0f};
-    if (!p.W16) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int n = nbase + h * BMH;
-            if (n < p.N) dq[h] = __fdiv_rn(p.sW[n], 127.0f);
-        }
-    }
     for (int t0 = 0; t0 < p.T; t0 += FIN_ROWS) {
-        float o[2][FIN_ROWS];
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int r = 0; r < FIN_ROWS; ++r) o[h][r] = 0.0f;
-        for (int j0 = 0; j0 < count; j0 += FIN_OUT) {
-            const int kj = (lane < FIN_OUT && j0 + lane < count) ? p.idx[j0 + lane] : -1;
-            // Xo[t0 .. t0+15][j0 .. j0+7] -> scratch, one independent load per element
-            __syncwarp();
-            for (int e = lane; e < FIN_ROWS * FIN_OUT; e += 32) {
-                const int r = e / FIN_OUT, jj = e % FIN_OUT;
-                const int t = t0 + r;
-                xo_s[e] = (t < p.T && j0 + jj < count)
-                              ? __half2float(p.Xo[static_cast<size_t>(t) * p.K + j0 + jj]) : 0.0f;
-            }
-            float w[2][FIN_OUT];
-#pragma unroll
-            for (int jj = 0; jj < FIN_OUT; ++jj) {
-                const int k = __shfl_sync(0xFFFFFFFFu, kj, jj);
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int n = nbase + h * BMH;
-                    float wv = 0.0f;
-                    if (k >= 0 && n < p.N) {
-                        const size_t at = static_cast<size_t>(k) * p.N + n;
-                        wv = p.W16 ? __half2float(p.W16[at])
-                                   : __half2float(__float2half_rn(__fmul_rn(static_cast<float>(p.Wq[at]), dq[h])));
-                    }
-                    w[h][jj] = wv;
-                }
-            }
-            __syncwarp();
-#pragma unroll
-            for (int r = 0; r < FIN_ROWS; ++r)
-#pragma unroll
-                for (int jj = 0; jj < FIN_OUT; ++jj) {
-                    const float x = xo_s[r * FIN_OUT + jj];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) o[h][r] = fmaf(x, w[h][jj], o[h][r]);
-                }
-        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
             const int n = nbase + h * BMH;
             if (n >= p.N) continue;
             const float sw = p.sW[n];
             int a[FIN_ROWS];
+            float yo[FIN_ROWS];
 #pragma unroll
-            for (int r = 0; r < FIN_ROWS; ++r)
-                a[r] = (t0 + r < p.T) ? __ldcg(p.acc32 + static_cast<size_t>(t0 + r) * p.N + n) : 0;
+            for (int r = 0; r < FIN_ROWS; ++r) {
+                const bool ok = t0 + r < p.T;
+                const size_t at = static_cast<size_t>(t0 + r) * p.N + n;
+                a[r] = ok ? __ldcg(p.acc32 + at) : 0;
+                yo[r] = (ok && count > 0) ? __ldcg(p.Yo + at) : 0.0f;
+            }
 #pragma unroll
             for (int r = 0; r < FIN_ROWS; ++r) {
                 const int t = t0 + r;
                 if (t < p.T) {
                     const float rs = p.sX[t] * (1.0f / 16129.0f);
                     p.Y[static_cast<size_t>(t) * p.N + n] =
-                        __float2half_rn(fmaf(static_cast<float>(a[r]), rs * sw, o[h][r]));
+                        __float2half_rn(fmaf(static_cast<float>(a[r]), rs * sw, yo[r]));
                 }
             }
         }
@@ -307,6 +260,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;
         griddep_wait();                                   // acc32 / counters zeroed, activation ready
+        const int count = p.finalize ? *p.count : 0;
         uint32_t tph[2] = {0, 0};
         int seg = 0;
         for (long long u = u0; u < u1;) {
@@ -351,9 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 last = __shfl_sync(0xFFFFFFFFu, last, 0);
                 if (last) {
                     __threadfence();
-                    float *xo_s = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(bars) + sizeof(Barriers)) +
-                                  (warp - 2) * FIN_ROWS * FIN_OUT;
-                    finalize_columns(p, tile, quad, lane, xo_s);
+                    finalize_columns(p, tile, quad, lane, count);
                 }
             }
             tph[buf] ^= 1u;

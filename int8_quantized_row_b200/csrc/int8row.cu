@@ -195,7 +195,7 @@ i8r_status check_ptr(const void *p) {
 
 // Workspace of int8_mixed_linear.
 struct Workspace {
-    size_t count, mask, idx, sX, Xq, Xo, W16o, acc32, counters, total;
+    size_t count, mask, idx, sX, Xq, Xo, W16o, Yo, acc32, counters, total;
 };
 
 // Rows of the compacted outlier weight rows kept for the prefill GEMM: 256
@@ -219,6 +219,8 @@ Workspace ws_layout(int T, int K, int N, bool wq_only = false) {
     w.Xo = off;    off = align_up(off + static_cast<size_t>(T) * K * 2);
     w.W16o = off;
     if (T > decode::MAX_T) off = align_up(off + static_cast<size_t>(compact_rows(K, wq_only)) * N * 2);
+    w.Yo = off;
+    if (T <= decode::MAX_T) off = align_up(off + static_cast<size_t>(T) * N * 4);   // fp32 outlier part
     w.acc32 = off;
     w.counters = off;
     if (T <= decode::MAX_T) {
@@ -262,8 +264,11 @@ cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, s
 // The row quantiser: G compaction blocks, then one block per row, launched as
 // a programmatic dependent of the outlier scan.
 template <int kThreads, typename... Args>
-cudaError_t launch_rows(cudaStream_t s, int T, int G, size_t smem, Args &&...args) {
-    return launch_dependent(quantize_rows_kernel<kThreads>, dim3(G + T), dim3(kThreads), smem, s, 1,
+cudaError_t launch_rows(cudaStream_t s, int T, int G, size_t smem, bool product, Args &&...args) {
+    if (product)
+        return launch_dependent(quantize_rows_kernel<kThreads, true>, dim3(G + T), dim3(kThreads), smem, s, 1,
+                                std::forward<Args>(args)...);
+    return launch_dependent(quantize_rows_kernel<kThreads, false>, dim3(G + T), dim3(kThreads), smem, s, 1,
                             std::forward<Args>(args)...);
 }
 
@@ -281,11 +286,14 @@ dim3 scan_grid(int T, int K, int sms, int *rows_per_block) {
 // `zero` / `zero_bytes`: a region the scan clears on the way (may be null).
 // With W16o, the quantiser's launch also compacts the W16 rows of the first
 // compact_rows(K) outlier columns into W16o ([compact_rows(K), N]); with W16
-// null (the Wq-only variant) it dequantises those rows of Wq instead.
+// null (the Wq-only variant) it dequantises those rows of Wq instead.  With
+// Yo ([T,N] fp32, decode sizes) its leading blocks also compute the 16-bit
+// outlier part of Y.
 i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int K, float alpha, uint32_t *mask,
                              int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
                              size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
-                             __half *W16o = nullptr, const int8_t *Wq = nullptr, const float *sW = nullptr) {
+                             __half *W16o = nullptr, const int8_t *Wq = nullptr, const float *sW = nullptr,
+                             float *Yo = nullptr) {
     const int nwords = (K + 31) / 32;
     clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords);
     I8R_LAUNCHED();
@@ -308,18 +316,20 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     const int rt = row_threads(K);
     const int o_rows = W16o ? compact_rows(K, W16 == nullptr) : 0;
     const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
+    const int Gy = Yo ? 2 * dev->sms : 0;                    // outlier-product blocks (decode): two per SM still
+                                                             // leave room for a decode GEMM CTA
     const size_t smem = quantize_smem_bytes(K);
     const uint32_t *m = mask;
     uint32_t *no_mask_out = nullptr;
     if (rt == 64)
-        e = launch_rows<64>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N, W16o,
-                            o_rows, G);
+        e = launch_rows<64>(s, T, G + Gy, smem, Gy > 0, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
+                            W16o, o_rows, G, Yo, Gy);
     else if (rt == 128)
-        e = launch_rows<128>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N, W16o,
-                             o_rows, G);
+        e = launch_rows<128>(s, T, G + Gy, smem, Gy > 0, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
+                             W16o, o_rows, G, Yo, Gy);
     else
-        e = launch_rows<256>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N, W16o,
-                             o_rows, G);
+        e = launch_rows<256>(s, T, G + Gy, smem, Gy > 0, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
+                             W16o, o_rows, G, Yo, Gy);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;
@@ -623,6 +633,7 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     const bool small_t = T <= decode::MAX_T;
     int32_t *acc32 = small_t ? reinterpret_cast<int32_t *>(ws + w.acc32) : nullptr;
     int32_t *counters = small_t ? reinterpret_cast<int32_t *>(ws + w.counters) : nullptr;
+    float *Yo = small_t ? reinterpret_cast<float *>(ws + w.Yo) : nullptr;
     const __half *x = static_cast<const __half *>(X);
     const __half *w16 = static_cast<const __half *>(W16);
     __half *y = static_cast<__half *>(Y);
@@ -635,7 +646,7 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     __half *W16o = nullptr;        // the single-CTA GEMM gathers the rows itself
 #endif
     I8R_TRY(launch_activation(dev, x, T, K, alpha, mask, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
-                              zero_bytes, stream, w16, N, W16o, Wq, sW));
+                              zero_bytes, stream, w16, N, W16o, Wq, sW, Yo));
     if (!small_t)
         return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream, W16o);
 
@@ -643,12 +654,9 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     fin.counters = counters;
     fin.sX = sX;
     fin.sW = sW;
-    fin.Xo = Xo;
-    fin.idx = idx;
     fin.count = count;
-    fin.W16 = w16;
-    fin.Wq = Wq;
     fin.Y = y;
+    fin.Yo = Yo;
     return launch_decode(dev, Xq, T, K, Wq, N, acc32, &fin, stream);
 }
 

@@ -50,6 +50,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=ROTATE,
                     help="input sets rotated between steps (default 3: operands not in L2)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every point of the 175B decoder-layer sweep in one process (one JSON line each; "
+                         "not the one-line contract run)")
     ap.add_argument("--variant", default="w16", choices=["w16", "wq"],
                     help="w16: int8_mixed_linear (fp16 weight resident for the outlier rows); "
                          "wq: int8_mixed_linear_wq (only Wq and sW resident)")
@@ -431,8 +434,82 @@ def run_ours(args, cfg, world, rank, local, pg):
         pg.destroy_process_group()
 
 
+def run_sweep(args):
+    """The 175B decoder-layer sweep: each layer's weight is drawn and converted
+    once, then every (T, outlier fraction, alpha) point is timed on it: whole
+    calls with CUDA events, then the GEMM alone through int8_time_next_gemm.
+    The weights (151-604 MB of int8) exceed L2, so steps stream them from HBM."""
+    import torch
+    import int8_quantized_row_b200 as i8
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+    cfgs = wl.sweep_configs()
+    for layer, (K, N) in wl.SWEEP_LAYERS.items():
+        W = torch.from_numpy(wl.make_w(K, N, 0.01)).to(dev)
+        Wq, sW = i8.int8_quantize_weight_colwise(W)
+        Tmax = max(wl.SWEEP_T)
+        if args.variant == "wq":
+            W = None
+            ws = torch.empty(max(1, i8.int8_mixed_linear_wq_workspace_size(Tmax, K, N)), dtype=torch.uint8, device=dev)
+        else:
+            ws = i8.workspace(Tmax, K, N, dev)
+        Y = torch.empty((Tmax, N), dtype=torch.float16, device=dev)
+        for name, cfg in cfgs.items():
+            if not name.startswith(f"b175_sweep_{layer}_"):
+                continue
+            T, alpha = cfg["T"], cfg["alpha"]
+            X = torch.from_numpy(wl.make_x(T, K, cfg["n_out"], cfg["lo"], cfg["hi"], cfg["row_prob"], cfg["seed"])).to(dev)
+            Yt = Y[:T]
+
+            def step():
+                if W is None:
+                    i8.int8_mixed_linear_wq(X, Wq, sW, alpha, Y=Yt, workspace_buf=ws)
+                else:
+                    i8.int8_mixed_linear(X, Wq, sW, W, alpha, Y=Yt, workspace_buf=ws)
+            steps = 40 if T >= 2048 else 200
+            for _ in range(5):
+                step()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                step()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / steps
+            gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for x, y in gev:            # torch only reports times of events it has seen recorded
+                x.record(stream)
+                y.record(stream)
+            torch.cuda.synchronize()
+            for i in range(steps):
+                i8.int8_time_next_gemm(gev[i][0], gev[i][1])
+                step()
+            torch.cuda.synchronize()
+            gemm_ms = sum(x.elapsed_time(y) for x, y in gev) / steps
+            n_out = int(i8.int8_outlier_stats(X, alpha)[0].item())
+            ops, wbytes = work(cfg, n_out, args.variant)
+            line = {"workload": name, "T": T, "K": K, "N": N, "alpha": alpha, "outlier_cols": n_out,
+                    "variant": args.variant, "ms_per_call": ms, "tops": ops / (ms * 1e-3) / 1e12,
+                    "weight_gbs": wbytes / (ms * 1e-3) / 1e9, "gemm_ms": gemm_ms,
+                    "status": i8.int8_read_and_clear_device_status()}
+            if T <= i8.DECODE_MAX_T:
+                line["gemm_frac_hbm"] = (wbytes + 2 * T * K + 2 * T * N) / (gemm_ms * 1e-3) / 1e9 / pk["hbm_gbs"]
+            if T >= 128:
+                line["gemm_frac_int8_sustained"] = ops / (gemm_ms * 1e-3) / 1e12 / (
+                    2.0 * (pk["bf16_tflops_sustained"] or pk["bf16_tflops"]))
+            print(json.dumps(line), flush=True)
+            del X
+        del W, Wq, sW, ws, Y
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     cfgs = all_configs()
     if args.workload not in cfgs:
         raise SystemExit(f"unknown workload {args.workload}; known: {sorted(cfgs)[:8]} ...")

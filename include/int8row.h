@@ -125,12 +125,12 @@ i8r_status int8_mixed_linear(const void *X, int T, int K,
  * so Y = fp16( acc*sX[t]*sW[n]/127^2 + X[:,O] W~[O,:] ).
  * Arguments, layouts and workspace rules are those of int8_mixed_linear,
  * with workspace of at least int8_mixed_linear_wq_workspace_size(T, K, N)
- * bytes.  For T > 128 that workspace holds the dequantised rows of at most
+ * bytes.  That workspace holds the dequantised rows of at most
  * int8_mixed_linear_wq_max_outliers(K) outlier columns (at least 256 and
  * 1/16 of K, rounded up to a multiple of 64, and not more than K rounded
- * up to 64).  A call that finds more outlier columns than that sets
- * I8R_DEV_OUTLIER_CAP in the device status word, and its Y lacks the 16-bit
- * part of the excess columns.  T <= 128 has no such limit.
+ * up to 64), at every T.  A call that finds more outlier columns than that
+ * sets I8R_DEV_OUTLIER_CAP in the device status word, and its Y lacks the
+ * 16-bit part of the excess columns.
  * ------------------------------------------------------------------------- */
 size_t int8_mixed_linear_wq_workspace_size(int T, int K, int N);
 

@@ -12,14 +12,25 @@
 // tile in TMEM (double-buffered) and adds the exact int32 partial sums into
 // acc32 [T,N] (zeroed beforehand) with red.add.
 //
-// The 16-bit outlier part Yo[t,n] = sum_j X[t,O_j] W16[O_j,n] (fp32) comes
-// from the row quantiser's launch (its outlier-product blocks), which this
-// kernel waits for with griddepcontrol.wait like the rest of the activation.
+// The 16-bit outlier part (LLM.int8() abstract: the outlier feature
+// dimensions go through a 16-bit matrix multiplication) runs on the same
+// tensor cores: the CTA that owns k-block 0 of a tile also runs an outlier
+// segment for it, ceil(|O|/64) stages of kind::f16 MMAs
+//   Yo[t,n] = sum_j Xo[t,j] * W16[O_j,n]      (fp32 in TMEM)
+// with A = the W16 rows of the outliers (MN-major, copied in place by the
+// lanes with cp.async, 16 bytes each, or the dequantised rows the quantiser
+// compacted for the Wq-only variant) and B = Xo (K-major), and stores it to
+// Yo [T,N].  Those stages have a shared-memory buffer of their own, filled
+// by a second producer warp, so the row copies never hold up the weight
+// stream's requests.  Each buffer (the weight ring, the outlier buffer) has
+// exactly one producer, which waits on every use of every slot: a parity
+// wait cannot tell a phase from the one two uses later, so a producer that
+// skipped slots could get two phases ahead of the consumer.
 //
-// Finalisation: after adding its partial sums, each epilogue warp bumps a
-// counter for its (tile, 32-lane quadrant).  The warp that brings the counter
-// to the number of CTAs covering the tile knows every partial sum has landed;
-// it writes
+// Finalisation: after adding its partial sums (or storing its Yo piece),
+// each epilogue warp bumps a counter for its (tile, 32-lane quadrant).  The
+// warp that brings the counter to the number of contributions the tile gets
+// knows every piece has landed; it writes
 //   Y[t,n] = fp16( acc32[t,n] * sX[t] * sW[n] / 127^2 + Yo[t,n] )
 // for its 64 columns.  No CTA ever waits on another.  (Stream-K leaves most
 // tiles split between the end of one CTA's range and the start of the next,
@@ -41,10 +52,15 @@ constexpr int BM = 2 * BMH;        // columns per tile
 constexpr int BK = 128;            // int8 K per stage (bytes)
 constexpr int A_HALF = BMH * BK;   // 16 KB
 constexpr int A_BYTES = 2 * A_HALF;
-constexpr int THREADS = 192;
+constexpr int OBK = 64;            // outliers per outlier stage: 64 W16 rows x 256 columns = A_BYTES,
+                                   // and T x 64 fp16 of Xo = the bytes of a T x 128 Xq tile
+constexpr int O_CHUNK = 64 * OBK * 2;   // 64 columns x 64 W16 rows (one 128-byte swizzle span)
+constexpr int THREADS = 224;       // warp 0 weight producer, 1 MMA, 2-5 epilogue, 6 outlier producer
 constexpr int MAX_T = 128;
 constexpr int MAX_STAGES = 8;
-constexpr size_t SMEM_BUDGET = 200 * 1024;
+constexpr size_t SMEM_BUDGET = 200 * 1024;     // the weight ring
+constexpr size_t SMEM_MAX = 220 * 1024;        // ring + outlier buffer (a row-quantiser block still fits beside)
+static_assert(4 * O_CHUNK == A_BYTES, "an outlier stage's W16 rows fill the weight slot");
 
 struct Params {
     int T, TP, K, N;
@@ -53,13 +69,18 @@ struct Params {
     int stages, stage_bytes;
     uint32_t tmem_cols;            // power of two >= 4*TP, >= 32; buffer b at b*tmem_cols/2
     int32_t *acc32;                // [T,N] int32, zero on entry
-    // finalisation (finalize != 0): Y from acc32 once a tile is complete
+    // finalisation (finalize != 0): Y from acc32 (and Yo) once a tile is complete
     int finalize;
     int32_t *counters;             // [num_tiles * 4], zero on entry
     const float *sX, *sW;
-    const int32_t *count;
+    const int32_t *count;          // |O|
+    const int32_t *idx;            // the outlier columns, ascending
+    const __half *W16;             // [K,N] fp16 (null for the Wq-only variant)
+    int o_rows;                    // Wq-only variant: rows of the compacted, dequantised W16o
+    int wq_only;                   // no W16: outlier rows come from W16o (zeros past o_rows)
+    int obuf;                      // 1: the outlier buffer exists (else the 16-bit part is skipped)
     __half *Y;
-    const float *Yo;               // [T,N] fp32: the 16-bit outlier part (read when |O| > 0)
+    float *Yo;                     // [T,N] fp32: the 16-bit outlier part (written when |O| > 0)
 };
 
 struct Barriers {
@@ -67,13 +88,18 @@ struct Barriers {
     uint64_t empty[MAX_STAGES];
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
+    uint64_t ofull, oempty;        // the outlier buffer
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
 
-__host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes) {
-    return 1024 + static_cast<size_t>(stages) * stage_bytes + sizeof(Barriers);
+// The weight ring (stages x stage_bytes), the outlier buffer (obuf x
+// stage_bytes: 64 W16 rows of a tile = A_BYTES, and T x 64 fp16 of Xo), then
+// the barriers; 1024 bytes for aligning the base to the 128-byte swizzle's
+// 1024-byte period.
+__host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes, int obuf) {
+    return 1024 + static_cast<size_t>(stages + obuf) * stage_bytes + sizeof(Barriers);
 }
 
 // CTA c of `ctas` owns units [floor(c*U/ctas), floor((c+1)*U/ctas)).
@@ -83,6 +109,28 @@ __device__ __forceinline__ long long unit_begin(long long total, int c, int ctas
 // The CTA whose range holds unit u.
 __device__ __forceinline__ int unit_owner(long long total, long long u, int ctas) {
     return static_cast<int>(((u + 1) * ctas - 1) / total);
+}
+
+// The stages of one CTA in order, the same for all its warps:
+//   for each tile its range [u0, u1) touches, the int8 k-blocks of that tile
+//   (kind 0, j = k-block), then, if the range holds the tile's k-block 0, the
+//   tile's nob outlier blocks (kind 1, j = outlier block).
+// A run of one kind for one tile is a segment: one TMEM accumulator buffer.
+// visit(kind, tile, j, first_of_segment, last_of_segment) returns false to stop.
+template <typename Visit>
+__device__ __forceinline__ bool walk_stages(const Params &p, long long u0, long long u1, int nob, Visit &&visit) {
+    for (long long u = u0; u < u1;) {
+        const int tile = static_cast<int>(u / p.KB);
+        const long long tile_u0 = static_cast<long long>(tile) * p.KB;
+        const long long end = min(u1, tile_u0 + p.KB);
+        for (long long v = u; v < end; ++v)
+            if (!visit(0, tile, static_cast<int>(v - tile_u0), v == u, v == end - 1)) return false;
+        if (u == tile_u0)
+            for (int b = 0; b < nob; ++b)
+                if (!visit(1, tile, b, b == 0, b == nob - 1)) return false;
+        u = end;
+    }
+    return true;
 }
 
 constexpr int FIN_ROWS = 16;
@@ -121,10 +169,12 @@ __device__ __forceinline__ void finalize_columns(const Params &p, int tile, int 
 
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap map_wq, const __grid_constant__ CUtensorMap map_xq,
+                       const __grid_constant__ CUtensorMap map_xo, const __grid_constant__ CUtensorMap map_w16o,
                        const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Barriers *bars = reinterpret_cast<Barriers *>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);
+    uint8_t *ob = smem + static_cast<size_t>(p.stages) * p.stage_bytes;      // the outlier buffer
+    Barriers *bars = reinterpret_cast<Barriers *>(ob + static_cast<size_t>(p.obuf) * p.stage_bytes);
     volatile int *abort = &bars->abort;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -138,6 +188,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&bars->tmem_full[b], 1);
             mbar_init(&bars->tmem_empty[b], 4);
         }
+        mbar_init(&bars->ofull, 1);
+        mbar_init(&bars->oempty, 1);
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_mbar_init();
@@ -156,100 +208,174 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const long long u0 = unit_begin(p.total_units, blockIdx.x, gridDim.x);
     const long long u1 = unit_begin(p.total_units, blockIdx.x + 1, gridDim.x);
+    const uint32_t tx = static_cast<uint32_t>(p.stage_bytes);
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        const uint32_t tx = static_cast<uint32_t>(p.stage_bytes);
-        int pending[MAX_STAGES];
-        for (int s = 0; s < MAX_STAGES; ++s) pending[s] = -1;
-        // Weight tiles of the first stages: they do not depend on the
-        // activation kernels, so they are requested before waiting on them.
-        const int pre = static_cast<int>(min(static_cast<long long>(p.stages), u1 - u0));
-        if (lane == 0) {
-            for (int i = 0; i < pre; ++i) {
-                const long long u = u0 + i;
-                const int tile = static_cast<int>(u / p.KB);
-                const int kb = static_cast<int>(u - static_cast<long long>(tile) * p.KB);
-                uint8_t *a = smem + static_cast<size_t>(i) * p.stage_bytes;
-                mbar_arrive_expect_tx(&bars->full[i], tx);   // fresh barrier: the slot is free
-                tma_load_2d(a, &map_wq, &bars->full[i], tile * BM, kb * BK);
-                tma_load_2d(a + A_HALF, &map_wq, &bars->full[i], tile * BM + BMH, kb * BK);
-                pending[i] = 0;
-            }
-        }
-        griddep_wait();
-        if (lane == 0) {
-            for (int i = 0; i < pre; ++i) {
-                const long long u = u0 + i;
-                const int kb = static_cast<int>(u % p.KB);
-                tma_load_2d(smem + static_cast<size_t>(i) * p.stage_bytes + A_BYTES, &map_xq, &bars->full[i],
-                            kb * BK, 0);
-            }
-        }
-        __syncwarp();
-        int stage = pre % p.stages;
-        uint32_t phase = (pre == p.stages) ? 1u : 0u;
-        for (long long u = u0 + pre; u < u1; ++u) {
+    // Weight tiles of the first stages (all in the first segment, which is
+    // int8) do not depend on the activation kernels: request them first.
+    const long long first_seg = min(u1, (u0 / p.KB + 1) * p.KB) - u0;
+    const int pre = static_cast<int>(min(static_cast<long long>(p.stages), first_seg));
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < pre; ++i) {
+            const long long u = u0 + i;
             const int tile = static_cast<int>(u / p.KB);
             const int kb = static_cast<int>(u - static_cast<long long>(tile) * p.KB);
-            if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) break;
-            if (lane == 0) {
-                uint8_t *a = smem + static_cast<size_t>(stage) * p.stage_bytes;
-                mbar_arrive_expect_tx(&bars->full[stage], tx);
-                tma_load_2d(a, &map_wq, &bars->full[stage], tile * BM, kb * BK);
-                tma_load_2d(a + A_HALF, &map_wq, &bars->full[stage], tile * BM + BMH, kb * BK);
-                tma_load_2d(a + A_BYTES, &map_xq, &bars->full[stage], kb * BK, 0);
-                pending[stage] = static_cast<int>(phase);
+            uint8_t *a = smem + static_cast<size_t>(i) * p.stage_bytes;
+            mbar_arrive_expect_tx(&bars->full[i], tx);   // fresh barrier: the slot is free
+            tma_load_2d(a, &map_wq, &bars->full[i], tile * BM, kb * BK);
+            tma_load_2d(a + A_HALF, &map_wq, &bars->full[i], tile * BM + BMH, kb * BK);
+        }
+    }
+    griddep_wait();                               // activation, |O|, acc32 / counters zeroed
+    const int count = p.finalize ? *p.count : 0;
+    const int nob = p.obuf ? (count + OBK - 1) / OBK : 0;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ weight producer
+        int pending[MAX_STAGES];
+        for (int s = 0; s < MAX_STAGES; ++s) pending[s] = -1;
+        int stage = 0, n = 0;
+        uint32_t phase = 0;
+        const bool ok = walk_stages(p, u0, u1, nob, [&](int kind, int tile, int j, bool, bool) -> bool {
+            if (kind != 0) return true;                   // outlier stages: the other producer
+            uint8_t *a = smem + static_cast<size_t>(stage) * p.stage_bytes;
+            uint64_t *fb = &bars->full[stage];
+            if (n < pre) {
+                if (lane == 0) tma_load_2d(a + A_BYTES, &map_xq, fb, j * BK, 0);
+            } else {
+                if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(fb, tx);
+                    tma_load_2d(a, &map_wq, fb, tile * BM, j * BK);
+                    tma_load_2d(a + A_HALF, &map_wq, fb, tile * BM + BMH, j * BK);
+                    tma_load_2d(a + A_BYTES, &map_xq, fb, j * BK, 0);
+                }
             }
+            if (lane == 0) pending[stage] = static_cast<int>(phase);
+            ++n;
             __syncwarp();
             if (++stage == p.stages) { stage = 0; phase ^= 1u; }
-        }
-        if (*abort && lane == 0) {
+            return true;
+        });
+        if (!ok && lane == 0) {
+            // let the loads already issued land before the CTA leaves (abort only)
             volatile int never = 0;
             for (int s = 0; s < p.stages; ++s)
                 if (pending[s] >= 0) mbar_wait(&bars->full[s], static_cast<uint32_t>(pending[s]), &never, 0);
         }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ outlier producer
+        if (nob > 0 && lane == 0) {
+            if (p.wq_only) tma_prefetch_map(&map_w16o);
+            tma_prefetch_map(&map_xo);
+        }
+        uint32_t ophase = 0;
+        int pending = -1;
+        const bool ok = walk_stages(p, u0, u1, nob, [&](int kind, int tile, int j, bool, bool) -> bool {
+            if (kind != 1) return true;
+            if (!warp_wait(&bars->oempty, ophase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+            uint64_t *fb = &bars->ofull;
+            if (p.wq_only) {
+                // compacted dequantised rows; past o_rows an out-of-range box, i.e.
+                // zeros (the quantiser reports the overflow)
+                if (lane == 0) {
+                    const int y = (j + 1) * OBK <= p.o_rows ? j * OBK : p.o_rows;
+                    mbar_arrive_expect_tx(fb, tx);
+                    tma_load_2d(ob + A_BYTES, &map_xo, fb, j * OBK, 0);
+                    for (int c = 0; c < 4; ++c) tma_load_2d(ob + c * O_CHUNK, &map_w16o, fb, tile * BM + 64 * c, y);
+                }
+            } else {
+                // The W16 rows of outliers j*64 .., zero past |O| rounded up to 16
+                // (the MMAs read no further): lane l copies columns 8l .. 8l+7 of
+                // every row into the 128-byte-swizzled chunk l/8, then the rows
+                // are made visible to the tensor core (async proxy) before the
+                // stage is published with its Xo tile.
+                const int rows = min(OBK, (count - j * OBK + 15) / 16 * 16);
+                const int g0 = j * OBK + lane, g1 = j * OBK + 32 + lane;
+                const int k0 = g0 < count ? p.idx[g0] : -1;
+                const int k1 = g1 < count ? p.idx[g1] : -1;
+                const int col = tile * BM + lane * 8;
+                const uint32_t chunk = smem_u32(ob) + static_cast<uint32_t>((lane >> 3) * O_CHUNK);
+                const uint32_t unit = static_cast<uint32_t>(lane & 7);
+                for (int r = 0; r < rows; ++r) {
+                    const int k = __shfl_sync(0xFFFFFFFFu, r < 32 ? k0 : k1, r & 31);
+                    const bool have = k >= 0 && col < p.N;
+                    const __half *src = have ? p.W16 + static_cast<size_t>(k) * p.N + col : p.W16;
+                    cp_async_16(chunk + static_cast<uint32_t>(r * 128) + ((unit ^ static_cast<uint32_t>(r & 7)) << 4),
+                                src, have ? 16u : 0u);
+                }
+                cp_async_wait_all();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.TP * OBK * 2));
+                    tma_load_2d(ob + A_BYTES, &map_xo, fb, j * OBK, 0);
+                }
+            }
+            pending = static_cast<int>(ophase);
+            __syncwarp();
+            ophase ^= 1u;
+            return true;
+        });
+        if (!ok && lane == 0 && pending >= 0) {
+            volatile int never = 0;
+            mbar_wait(&bars->ofull, static_cast<uint32_t>(pending), &never, 0);
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
-        const uint32_t id = idesc_i8(BMH, p.TP, true, false);
-        int stage = 0;
-        uint32_t phase = 0;
+        const uint32_t id_i8 = idesc_i8(BMH, p.TP, true, false);
+        const uint32_t id_f16 = idesc_f16(BMH, p.TP, true, false);
+        int stage = 0, seg = 0;
+        uint32_t phase = 0, ophase = 0;
         uint32_t tph[2] = {0, 0};
-        int seg = 0;
-        bool ok = true;
-        for (long long u = u0; ok && u < u1;) {
-            const int tile = static_cast<int>(u / p.KB);
-            const long long seg_end = min(u1, static_cast<long long>(tile + 1) * p.KB);
+        walk_stages(p, u0, u1, nob, [&](int kind, int, int j, bool first, bool last) -> bool {
             const int buf = seg & 1;
-            if (!warp_wait(&bars->tmem_empty[buf], tph[buf] ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) break;
-            tc_fence_after_sync();
-            const uint32_t d0 = tmem + static_cast<uint32_t>(buf) * half_cols;
-            const uint32_t d1 = d0 + static_cast<uint32_t>(p.TP);
-            for (long long v = u; v < seg_end; ++v) {
-                if (!warp_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) { ok = false; break; }
+            if (first) {
+                if (!warp_wait(&bars->tmem_empty[buf], tph[buf] ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
                 tc_fence_after_sync();
-                if (lane == 0) {
-                    const uint32_t a = smem_u32(smem + static_cast<size_t>(stage) * p.stage_bytes);
-                    const uint32_t b = a + A_BYTES;
+            }
+            uint64_t *fb = kind == 0 ? &bars->full[stage] : &bars->ofull;
+            if (!warp_wait(fb, kind == 0 ? phase : ophase, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+            tc_fence_after_sync();
+            if (kind == 1) fence_proxy_async_smem();      // cp.async rows -> tensor core reads
+            if (lane == 0) {
+                const uint32_t d0 = tmem + static_cast<uint32_t>(buf) * half_cols;
+                const uint32_t d1 = d0 + static_cast<uint32_t>(p.TP);
+                const uint32_t a = kind == 0 ? smem_u32(smem + static_cast<size_t>(stage) * p.stage_bytes) : smem_u32(ob);
+                const uint32_t b = a + A_BYTES;
+                if (kind == 0) {
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk) {
-                        const uint32_t acc = (v != u || kk != 0) ? 1u : 0u;
+                        const uint32_t acc = (!first || kk != 0) ? 1u : 0u;
                         const uint64_t bd = smem_desc_sw128(b + kk * 32, 16, 1024);
-                        mma_i8(d0, smem_desc_sw128(a + kk * 32 * 128, A_HALF, 1024), bd, id, acc);
-                        mma_i8(d1, smem_desc_sw128(a + A_HALF + kk * 32 * 128, A_HALF, 1024), bd, id, acc);
+                        mma_i8(d0, smem_desc_sw128(a + kk * 32 * 128, A_HALF, 1024), bd, id_i8, acc);
+                        mma_i8(d1, smem_desc_sw128(a + A_HALF + kk * 32 * 128, A_HALF, 1024), bd, id_i8, acc);
                     }
-                    mma_commit(&bars->empty[stage]);
+                } else {
+                    // 16 outliers per MMA: A = 16 W16 rows (2 KB of each 64-column
+                    // chunk), B = 16 fp16 of each Xo row (32 bytes)
+                    const int nk = min(OBK / 16, (count - j * OBK + 15) / 16);
+                    for (int kk = 0; kk < nk; ++kk) {
+                        const uint32_t acc = (!first || kk != 0) ? 1u : 0u;
+                        const uint64_t bd = smem_desc_sw128(b + kk * 32, 16, 1024);
+                        mma_f16(d0, smem_desc_sw128(a + kk * 16 * 128, O_CHUNK, 1024), bd, id_f16, acc);
+                        mma_f16(d1, smem_desc_sw128(a + A_HALF + kk * 16 * 128, O_CHUNK, 1024), bd, id_f16, acc);
+                    }
                 }
-                __syncwarp();
-                if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+                mma_commit(kind == 0 ? &bars->empty[stage] : &bars->oempty);
+                if (last) mma_commit(&bars->tmem_full[buf]);
             }
-            if (!ok) break;
-            if (lane == 0) mma_commit(&bars->tmem_full[buf]);
             __syncwarp();
-            tph[buf] ^= 1u;
-            ++seg;
-            u = seg_end;
-        }
+            if (last) {
+                tph[buf] ^= 1u;
+                ++seg;
+            }
+            if (kind == 0) {
+                if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+            } else {
+                ophase ^= 1u;
+            }
+            return true;
+        });
         if (lane == 0) {
             volatile int never = 0;
             mma_commit(&bars->drain);
@@ -259,16 +385,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;
-        griddep_wait();                                   // acc32 / counters zeroed, activation ready
-        const int count = p.finalize ? *p.count : 0;
         uint32_t tph[2] = {0, 0};
         int seg = 0;
-        for (long long u = u0; u < u1;) {
-            const int tile = static_cast<int>(u / p.KB);
-            const long long tile_u0 = static_cast<long long>(tile) * p.KB;
-            const long long seg_end = min(u1, tile_u0 + p.KB);
+        walk_stages(p, u0, u1, nob, [&](int kind, int tile, int, bool, bool last) -> bool {
+            if (!last) return true;
             const int buf = seg & 1;
-            if (!warp_wait(&bars->tmem_full[buf], tph[buf], abort, I8R_DEV_TMEM_TIMEOUT)) break;
+            if (!warp_wait(&bars->tmem_full[buf], tph[buf], abort, I8R_DEV_TMEM_TIMEOUT)) return false;
             tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf) * half_cols;
 #pragma unroll
@@ -282,8 +404,13 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const int t = c + i;
-                            if (t < p.T && r[i] != 0u)
-                                atomicAdd(p.acc32 + static_cast<size_t>(t) * p.N + n, static_cast<int>(r[i]));
+                            if (t >= p.T) continue;
+                            const size_t at = static_cast<size_t>(t) * p.N + n;
+                            if (kind == 0) {
+                                if (r[i] != 0u) atomicAdd(p.acc32 + at, static_cast<int>(r[i]));
+                            } else {
+                                __stcg(p.Yo + at, __uint_as_float(r[i]));
+                            }
                         }
                     }
                 }
@@ -292,26 +419,27 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
             if (p.finalize) {
-                // publish this warp's partial sums, then count the contribution
+                // publish this warp's piece, then count it
                 __threadfence();
                 __syncwarp();
-                int last = 0;
+                int done = 0;
                 if (lane == 0) {
-                    const int contributors = unit_owner(p.total_units, tile_u0 + p.KB - 1, gridDim.x) -
-                                             unit_owner(p.total_units, tile_u0, gridDim.x) + 1;
+                    const long long tile_u0 = static_cast<long long>(tile) * p.KB;
+                    const int pieces = unit_owner(p.total_units, tile_u0 + p.KB - 1, gridDim.x) -
+                                       unit_owner(p.total_units, tile_u0, gridDim.x) + 1 + (nob > 0 ? 1 : 0);
                     const int before = atomicAdd(p.counters + tile * 4 + quad, 1);
-                    last = before == contributors - 1;
+                    done = before == pieces - 1;
                 }
-                last = __shfl_sync(0xFFFFFFFFu, last, 0);
-                if (last) {
+                done = __shfl_sync(0xFFFFFFFFu, done, 0);
+                if (done) {
                     __threadfence();
                     finalize_columns(p, tile, quad, lane, count);
                 }
             }
             tph[buf] ^= 1u;
             ++seg;
-            u = seg_end;
-        }
+            return true;
+        });
     }
 
     tc_fence_before_sync();

@@ -5,15 +5,17 @@
 //   clear_mask_kernel       zeroes the outlier column bitmask
 //   outlier_scan_kernel     X -> outlier column bitmask, atomic OR per word   (a1)
 //   quantize_rows_kernel    X -> sX, Xq (outliers zeroed), Xo gather, the
-//                           index list; for T > 128 it also compacts the
-//                           outliers' W16 rows                              (a1-a3)
+//                           index list; for T > 128 (and for the Wq-only
+//                           variant at every T) it also compacts the
+//                           outliers' W16 rows (dequantised Wq rows)        (a1-a3)
 // The scan and the quantiser are programmatic dependents of the kernel
 // before them, so each loads its rows of X before waiting for it.
 //   T > 128:  gemm_prefill_kernel (one CTA per 128 x 256 tile) or
 //             gemm_prefill_pair_kernel (CTA pairs, 256 x 256 tiles): int8 +
 //             fp16 tensor-core MMA, epilogue -> Y
-//   T <= 128: gemm_decode_kernel   split-K int8 MMA -> int32 partial sums; the
-//             last contributor of each tile applies scales + fp16 outlier part
+//   T <= 128: gemm_decode_kernel   split-K int8 MMA -> int32 partial sums, one
+//             fp16 MMA segment per tile for the outlier part; the last
+//             contributor of each tile applies the scales and adds the two
 // The GEMMs are launched as programmatic dependents of the quantiser, so their
 // prologue and first weight tiles overlap the activation kernels.
 #include <algorithm>
@@ -116,7 +118,7 @@ i8r_status device_setup(const DeviceInfo **out) {
             I8R_CUDA(cudaOccupancyMaxActiveClusters(&d.pair_clusters, prefill2::gemm_prefill_pair_kernel<false>, &cfg));
             if (d.pair_clusters < 1) return I8R_EARCH;
             I8R_CUDA(cudaFuncSetAttribute(decode::gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(decode::SMEM_BUDGET + 4096)));
+                                          static_cast<int>(decode::SMEM_MAX + 4096)));
         }
         if (!g_encode) {
             void *fn = nullptr;
@@ -218,7 +220,7 @@ Workspace ws_layout(int T, int K, int N, bool wq_only = false) {
     w.Xq = off;    off = align_up(off + static_cast<size_t>(T) * K);
     w.Xo = off;    off = align_up(off + static_cast<size_t>(T) * K * 2);
     w.W16o = off;
-    if (T > decode::MAX_T) off = align_up(off + static_cast<size_t>(compact_rows(K, wq_only)) * N * 2);
+    if (T > decode::MAX_T || wq_only) off = align_up(off + static_cast<size_t>(compact_rows(K, wq_only)) * N * 2);
     w.Yo = off;
     if (T <= decode::MAX_T) off = align_up(off + static_cast<size_t>(T) * N * 4);   // fp32 outlier part
     w.acc32 = off;
@@ -264,11 +266,8 @@ cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, s
 // The row quantiser: G compaction blocks, then one block per row, launched as
 // a programmatic dependent of the outlier scan.
 template <int kThreads, typename... Args>
-cudaError_t launch_rows(cudaStream_t s, int T, int G, size_t smem, bool product, Args &&...args) {
-    if (product)
-        return launch_dependent(quantize_rows_kernel<kThreads, true>, dim3(G + T), dim3(kThreads), smem, s, 1,
-                                std::forward<Args>(args)...);
-    return launch_dependent(quantize_rows_kernel<kThreads, false>, dim3(G + T), dim3(kThreads), smem, s, 1,
+cudaError_t launch_rows(cudaStream_t s, int T, int G, size_t smem, Args &&...args) {
+    return launch_dependent(quantize_rows_kernel<kThreads>, dim3(G + T), dim3(kThreads), smem, s, 1,
                             std::forward<Args>(args)...);
 }
 
@@ -286,14 +285,11 @@ dim3 scan_grid(int T, int K, int sms, int *rows_per_block) {
 // `zero` / `zero_bytes`: a region the scan clears on the way (may be null).
 // With W16o, the quantiser's launch also compacts the W16 rows of the first
 // compact_rows(K) outlier columns into W16o ([compact_rows(K), N]); with W16
-// null (the Wq-only variant) it dequantises those rows of Wq instead.  With
-// Yo ([T,N] fp32, decode sizes) its leading blocks also compute the 16-bit
-// outlier part of Y.
+// null (the Wq-only variant) it dequantises those rows of Wq instead.
 i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int K, float alpha, uint32_t *mask,
                              int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
                              size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
-                             __half *W16o = nullptr, const int8_t *Wq = nullptr, const float *sW = nullptr,
-                             float *Yo = nullptr) {
+                             __half *W16o = nullptr, const int8_t *Wq = nullptr, const float *sW = nullptr) {
     const int nwords = (K + 31) / 32;
     clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords);
     I8R_LAUNCHED();
@@ -316,20 +312,18 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     const int rt = row_threads(K);
     const int o_rows = W16o ? compact_rows(K, W16 == nullptr) : 0;
     const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
-    const int Gy = Yo ? 2 * dev->sms : 0;                    // outlier-product blocks (decode): two per SM still
-                                                             // leave room for a decode GEMM CTA
     const size_t smem = quantize_smem_bytes(K);
     const uint32_t *m = mask;
     uint32_t *no_mask_out = nullptr;
     if (rt == 64)
-        e = launch_rows<64>(s, T, G + Gy, smem, Gy > 0, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
-                            W16o, o_rows, G, Yo, Gy);
+        e = launch_rows<64>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
+                            W16o, o_rows, G);
     else if (rt == 128)
-        e = launch_rows<128>(s, T, G + Gy, smem, Gy > 0, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
-                             W16o, o_rows, G, Yo, Gy);
+        e = launch_rows<128>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
+                             W16o, o_rows, G);
     else
-        e = launch_rows<256>(s, T, G + Gy, smem, Gy > 0, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
-                             W16o, o_rows, G, Yo, Gy);
+        e = launch_rows<256>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
+                             W16o, o_rows, G);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;
@@ -486,9 +480,12 @@ i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half 
 
 // Decode GEMM (T <= 128): int32 partial sums added into acc32, which must be
 // zero on entry.  With `fin` (non-null) the last contributor of every tile also
-// writes Y; fin->counters must be zero on entry.
+// writes Y; fin->counters must be zero on entry.  With fin, |O| > 0 adds the
+// 16-bit part from Xo and the W16 rows fin->idx (or, fin->wq_only, from the
+// fin->o_rows compacted rows W16o).
 i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, const int8_t *Wq, int N,
-                         int32_t *acc32, const decode::Params *fin, cudaStream_t s) {
+                         int32_t *acc32, const decode::Params *fin, cudaStream_t s, const __half *Xo = nullptr,
+                         const __half *W16 = nullptr, const __half *W16o = nullptr) {
     decode::Params p = fin ? *fin : decode::Params{};
     p.finalize = fin ? 1 : 0;
     p.T = T;
@@ -501,20 +498,28 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.stage_bytes = decode::A_BYTES + p.TP * decode::BK;
     p.stages = static_cast<int>(decode::SMEM_BUDGET / p.stage_bytes);
     if (p.stages > decode::MAX_STAGES) p.stages = decode::MAX_STAGES;
+    p.obuf = (fin && fin->obuf) ? 1 : 0;
+    while (p.obuf && p.stages > 2 && static_cast<size_t>(p.stages + 1) * p.stage_bytes > decode::SMEM_MAX) --p.stages;
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(4 * p.TP)) cols <<= 1;
     p.tmem_cols = cols;
     p.acc32 = acc32;
-    CUtensorMap map_wq, map_xq;
+    CUtensorMap map_wq, map_xq, map_xo, map_w16o;
     // Two 128-column boxes per stage cover 256 contiguous bytes of every weight
     // row, so the 256-byte L2 line is used whole.
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BMH));
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, p.TP, decode::BK));
+    map_xo = map_w16o = map_xq;   // unused without a 16-bit part
+    p.W16 = W16;
+    if (fin && Xo) {
+        I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, p.TP, decode::OBK));
+        if (W16o) I8R_TRY(make_map(&map_w16o, W16o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.o_rows, N, 64, 64));
+    }
     const long long g = p.total_units < dev->sms ? p.total_units : dev->sms;
-    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes);
+    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes, p.obuf);
     record_before(s);
     cudaError_t e = launch_dependent(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(g)),
-                                     dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, p);
+                                     dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, map_xo, map_w16o, p);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;
@@ -640,13 +645,16 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
 
     // decode: the outlier scan clears the split-K accumulator and the tile counters
     const size_t zero_bytes = small_t ? w.total - w.acc32 : 0;
+    // compacted outlier rows: the prefill GEMM's first compact_rows(K), and the
+    // Wq-only variant's dequantised rows at every T (the decode GEMM gathers W16
+    // rows itself)
 #if I8R_PREFILL_PAIR
-    __half *W16o = small_t ? nullptr : reinterpret_cast<__half *>(ws + w.W16o);
+    __half *W16o = (small_t && !wq_only) ? nullptr : reinterpret_cast<__half *>(ws + w.W16o);
 #else
-    __half *W16o = nullptr;        // the single-CTA GEMM gathers the rows itself
+    __half *W16o = (small_t && wq_only) ? reinterpret_cast<__half *>(ws + w.W16o) : nullptr;
 #endif
     I8R_TRY(launch_activation(dev, x, T, K, alpha, mask, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
-                              zero_bytes, stream, w16, N, W16o, Wq, sW, Yo));
+                              zero_bytes, stream, w16, N, W16o, Wq, sW));
     if (!small_t)
         return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream, W16o);
 
@@ -655,9 +663,13 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     fin.sX = sX;
     fin.sW = sW;
     fin.count = count;
+    fin.idx = idx;
+    fin.o_rows = wq_only ? compact_rows(K, true) : 0;
+    fin.wq_only = wq_only ? 1 : 0;
+    fin.obuf = std::isinf(alpha) ? 0 : 1;          // alpha = +inf: no finite input is an outlier
     fin.Y = y;
     fin.Yo = Yo;
-    return launch_decode(dev, Xq, T, K, Wq, N, acc32, &fin, stream);
+    return launch_decode(dev, Xq, T, K, Wq, N, acc32, &fin, stream, Xo, w16, W16o);
 }
 
 }  // namespace

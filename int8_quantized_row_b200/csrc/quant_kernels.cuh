@@ -291,11 +291,10 @@ __global__ void __launch_bounds__(kIndexThreads) outlier_index_kernel(const uint
 // ---------------------------------------------------------------------------
 // Row quantisation of the non-outlier part plus the outlier gather (one
 // block per row of X, after the G blocks that compact outlier weight rows for
-// the prefill GEMM and the Gy blocks that compute the outlier part of Y for
-// the decode GEMM):
+// the GEMMs):
 //   sX[t]   = max over k not in O of |X[t,k]|
 //   Xq[t,k] = 0 for k in O, else clamp(rhaz(X[t,k] * fl32(127/sX[t])), +-127)
-//   Xo[t,j] = X[t, O_j] for j < |O|, 0 up to the next multiple of 64
+//   Xo[t,j] = X[t, O_j] for j < |O|, 0 up to the next multiple of 64 (or K)
 // ("Vector-wise quantization" and "Mixed-precision decomposition").
 // Every block ORs the partial masks of the outlier scan into shared memory
 // and ranks the outlier columns itself (prefix counts of the mask words'
@@ -410,116 +409,13 @@ __device__ __forceinline__ uint32_t pack4_s8(int q0, int q1, int q2, int q3) {
     return __byte_perm(p01, p23, 0x5410u);
 }
 
-// The 16-bit outlier part of Y for decode-sized T (<= 128), computed by the
-// leading blocks of the row quantiser's launch (at most two per SM, so the
-// decode GEMM's CTAs fit beside them and request their first weights
-// meanwhile), before the weight stream starts, which would queue every load
-// behind it:
-//   Yo[t,n] = sum_j X[t,O_j] * W[O_j,n]   (fp32; W = W16, or for the Wq-only
-//                                          variant fp16_rn(Wq * fl32(sW/127)))
-// The blocks walk work items of 16 rows; the item shape follows |O|:
-//   |O| <= 16:  as many columns as threads, one per thread, one pass;
-//   larger:     64 columns; the threads form slices of 64, slice s takes
-//               outliers 16s .. 16s+15 of every group of 16 x slices, and the
-//               slices' sums are added in slice order.
-// Either way the outliers go 16 per thread per pass through shared memory
-// (their indices from the block's ranks of the mask, the X values of the 16
-// rows), each thread holding its column's 16 weights in registers (few
-// enough that a block fits on an SM beside a decode GEMM CTA).  The result
-// does not depend on timing.
-constexpr int kOutChunk = 16;    // outliers per thread per pass
-
-template <int kThreads>
-__device__ __forceinline__ void outlier_product(const uint32_t *smask, const int *spre, int w0, int w1, int total,
-                                                const __half *__restrict__ X, int T, int K,
-                                                const __half *__restrict__ W16, const int8_t *__restrict__ Wq,
-                                                const float *__restrict__ sW, int N, float *__restrict__ Yo, int b,
-                                                int nb) {
-    constexpr int kMaxSlices = kThreads / 64;
-    __shared__ int oidx[kMaxSlices * kOutChunk];
-    __shared__ float xs[kMaxSlices][16][kOutChunk];
-    __shared__ float part[kMaxSlices > 1 ? kMaxSlices - 1 : 1][16][64];
-    if (total == 0) return;
-    const int tid = threadIdx.x;
-    const bool wide = total <= kOutChunk;
-    const int cols = wide ? kThreads : 64;             // columns per item
-    const int slices = wide ? 1 : kMaxSlices;
-    const int c = tid % cols, sl = tid / cols;
-    const int group = slices * kOutChunk;              // outliers per pass
-    const int ncb = (N + cols - 1) / cols;
-    const int items = ncb * ((T + 15) / 16);
-    for (int item = b; item < items; item += nb) {
-        const int n = (item % ncb) * cols + c;
-        const int r0 = (item / ncb) * 16;
-        const bool col_ok = n < N;
-        const float dq = (!W16 && col_ok) ? __fdiv_rn(sW[n], 127.0f) : 0.0f;
-        float acc[16];
-#pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] = 0.0f;
-        for (int J = 0; J < total; J += group) {
-            // the outlier columns of ranks J .. J+group-1, from the per-word ranks
-            for (int w = w0; w < w1; ++w) {
-                int j = spre[w];
-                if (j >= J + group) break;
-                uint32_t m = smask[w];
-                while (m) {
-                    if (j >= J && j < J + group) oidx[j - J] = w * 32 + (__ffs(m) - 1);
-                    ++j;
-                    m &= m - 1;
-                }
-            }
-            __syncthreads();
-            const int j0 = J + sl * kOutChunk;
-            const int nj = max(0, min(kOutChunk, total - j0));
-            const int *oi = oidx + sl * kOutChunk;
-            for (int e = c; e < 16 * kOutChunk; e += cols) {
-                const int rr = e / kOutChunk, j = e % kOutChunk;
-                const int t = r0 + rr;
-                xs[sl][rr][j] = (t < T && j < nj) ? __half2float(X[static_cast<size_t>(t) * K + oi[j]]) : 0.0f;
-            }
-            float wv[kOutChunk];
-#pragma unroll
-            for (int j = 0; j < kOutChunk; ++j) {
-                float v = 0.0f;
-                if (j < nj && col_ok) {
-                    const size_t at = static_cast<size_t>(oi[j]) * N + n;
-                    v = W16 ? __half2float(W16[at])
-                            : __half2float(__float2half_rn(__fmul_rn(static_cast<float>(Wq[at]), dq)));
-                }
-                wv[j] = v;
-            }
-            __syncthreads();
-#pragma unroll
-            for (int r = 0; r < 16; ++r)
-#pragma unroll
-                for (int j = 0; j < kOutChunk; ++j) acc[r] = fmaf(xs[sl][r][j], wv[j], acc[r]);
-            __syncthreads();                          // oidx and xs are rewritten by the next pass
-        }
-        if (!wide && kMaxSlices > 1) {
-            if (sl > 0)
-#pragma unroll
-                for (int r = 0; r < 16; ++r) part[sl - 1][r][c] = acc[r];
-            __syncthreads();
-            if (sl == 0)
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    for (int q = 0; q < slices - 1; ++q) acc[r] += part[q][r][c];
-            __syncthreads();                          // part is rewritten by the next item
-        }
-        if (sl == 0 && col_ok)
-#pragma unroll
-            for (int r = 0; r < 16; ++r)
-                if (r0 + r < T) Yo[static_cast<size_t>(r0 + r) * N + n] = acc[r];
-    }
-}
-
-template <int kRowThreads, bool kProduct>
+template <int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ parts, int nparts,
     float *__restrict__ sX, int8_t *__restrict__ Xq, __half *__restrict__ Xo, uint32_t *__restrict__ mask_out,
     int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out, const __half *__restrict__ W16,
     const int8_t *__restrict__ Wq, const float *__restrict__ sW, int N, __half *__restrict__ W16o, int o_rows,
-    int G, float *__restrict__ Yo, int Gy) {
+    int G) {
     constexpr int kWarps = kRowThreads / 32;
     extern __shared__ uint32_t qs[];
     __shared__ float red[kWarps];
@@ -527,7 +423,7 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     const int nwords = (K + 31) / 32;
     uint32_t *smask = qs;
     int *spre = reinterpret_cast<int *>(qs + nwords);
-    const int t = static_cast<int>(blockIdx.x) - G - Gy;        // row; < 0: compaction / outlier-product block
+    const int t = static_cast<int>(blockIdx.x) - G;             // row; < 0: compaction block
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int chunks = K / 8;
     griddep_launch_dependents();        // the GEMM may start its prologue and weight loads
@@ -578,12 +474,8 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     }
     __syncthreads();
     if (t < 0) {
-        if (static_cast<int>(blockIdx.x) < G)
-            gather_outlier_weight_rows<kRowThreads>(smask, spre, w0, w1, total, W16, Wq, sW, N, W16o, o_rows,
-                                                    static_cast<int>(blockIdx.x), G);
-        else if (kProduct)
-            outlier_product<kRowThreads>(smask, spre, w0, w1, total, X, T, K, W16, Wq, sW, N, Yo,
-                                         static_cast<int>(blockIdx.x) - G, Gy);
+        gather_outlier_weight_rows<kRowThreads>(smask, spre, w0, w1, total, W16, Wq, sW, N, W16o, o_rows,
+                                                static_cast<int>(blockIdx.x), G);
         return;
     }
     const uint8_t *mbytes = reinterpret_cast<const uint8_t *>(smask);
@@ -656,7 +548,7 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
         emit(i, v);
     }
     if (orow) {
-        const int padded = (total + 63) / 64 * 64;
+        const int padded = min((total + 63) / 64 * 64, K);   // past K the GEMMs' Xo boxes read zeros
         for (int jj = total + tid; jj < padded; jj += kRowThreads) orow[jj] = __float2half_rn(0.0f);
     }
 

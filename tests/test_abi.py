@@ -92,15 +92,18 @@ def test_wq_variant_host_checks_and_capacity(so):
     g = so.int8_mixed_linear
     assert g(_p(), 16, 1024, _p(), _p(), _null(), 1024, 6.0, _p(), _p(),
              so.int8_mixed_linear_workspace_size(16, 1024, 1024), _null()) == 1
-    # rows of dequantised outlier weights the prefill workspace holds:
+    # rows of dequantised outlier weights the workspace holds:
     # at least 256 and K/16, rounded up to 64, at most K rounded up to 64
     cap = so.int8_mixed_linear_wq_max_outliers
     assert [cap(k) for k in (16, 64, 1024, 5120, 12288, 49152)] == [64, 64, 256, 320, 768, 3072]
-    # the workspace holds exactly those rows on top of the plain one (prefill), none at decode
+    # the workspace holds exactly those rows on top of the plain one: at prefill
+    # sizes the plain one already compacts 256 W16 rows, at decode sizes none
     for T, K, N in ((2048, 12288, 49152), (300, 1024, 512)):
         extra = so.int8_mixed_linear_wq_workspace_size(T, K, N) - so.int8_mixed_linear_workspace_size(T, K, N)
         assert extra == (cap(K) - min(256, (K + 63) // 64 * 64)) * N * 2
-    assert so.int8_mixed_linear_wq_workspace_size(16, 12288, 49152) == so.int8_mixed_linear_workspace_size(16, 12288, 49152)
+    for T, K, N in ((16, 12288, 49152), (128, 1024, 512), (1, 64, 16)):
+        extra = so.int8_mixed_linear_wq_workspace_size(T, K, N) - so.int8_mixed_linear_workspace_size(T, K, N)
+        assert extra == cap(K) * N * 2
 
 
 def test_host_rejects_bad_weight_conversion(so):

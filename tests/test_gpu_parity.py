@@ -228,6 +228,38 @@ def test_prefill_schedule_matches_oracle(orc, T, K, N, cols, alpha):
     assert device_status_clean()
 
 
+DECODE_SCHEDULE_CASES = [
+    # decode shapes whose CTAs run many more stages than the weight ring holds,
+    # with outlier segments in between: the ring and the outlier buffer are
+    # each reused many times over
+    (16, 4096, 12288, list(range(5, 4096, 600)), 6.0),           # |O| = 7, ~10 stages per CTA
+    (1, 4096, 12288, list(range(0, 4096, 31)), 6.0),             # |O| = 133: three outlier blocks per tile
+    (128, 4096, 8192, list(range(3, 4096, 57)), 6.0),            # T = 128, three-stage ring, |O| = 72
+    (64, 2048, 8192, [], 0.0),                                   # alpha = 0: 32 outlier blocks per tile
+]
+
+
+@pytest.mark.parametrize("T,K,N,cols,alpha", DECODE_SCHEDULE_CASES)
+@pytest.mark.parametrize("variant", ["w16", "wq"])
+def test_decode_schedule_matches_oracle(orc, T, K, N, cols, alpha, variant):
+    rng = np.random.default_rng(T + 3 * K + N)
+    X = outlier_x(rng, T, K, cols)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    Wq_o, sW_o = orc.quantize_weight_colwise(W)
+    Wq, sW = i8.int8_quantize_weight_colwise(to_dev(W))
+    if variant == "w16":
+        Y = to_host(i8.int8_mixed_linear(to_dev(X), Wq, sW, to_dev(W), alpha))
+    else:
+        if alpha == 0.0 and K > i8.int8_mixed_linear_wq_max_outliers(K):
+            pytest.skip("more outlier columns than the Wq-only workspace holds")
+        Y = to_host(i8.int8_mixed_linear_wq(to_dev(X), Wq, sW, alpha))
+    rows = np.unique(np.r_[0:T:5, T - 1]).astype(np.int32)
+    Y_o, _, _, cnt = orc.mixed_linear(X, Wq_o, sW_o, W if variant == "w16" else None, alpha, rows=rows)
+    assert cnt == (K if alpha == 0.0 else len(cols))
+    assert_y_close(Y[rows], Y_o, f"{variant} T={T} K={K} N={N} |O|={cnt}")
+    assert device_status_clean()
+
+
 def test_exact_integer_case_is_exact(orc):
     """alpha = +inf with integer inputs whose row / column absmax is 127: the
     codes are the inputs, and Y is the exact integer product (kept within

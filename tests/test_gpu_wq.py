@@ -1,11 +1,11 @@
 """The Wq-only variant (outlier rows dequantised from Wq) against the oracle.
 
-Same tolerance on Y as the fp16-weight layer.  Shapes cover the decode
-kernel (T <= 128, finaliser dequantises the rows it reads), the prefill
-kernel (the quantiser's leading blocks write the dequantised rows into the
-workspace), outlier sets of one and several 64-column blocks, a long
-schedule, alpha = 0 at decode size, an outlier count exactly at the prefill
-workspace's capacity, and one past it (reported in the device status word).
+Same tolerance on Y as the fp16-weight layer.  At every T the quantiser's
+leading blocks write the dequantised rows into the workspace; shapes cover
+the decode kernel (T <= 128) and the prefill kernel, outlier sets of one and
+several 64-column blocks, a long schedule, alpha = 0 at decode size, an
+outlier count exactly at the workspace's capacity, and one past it at both
+kernels (reported in the device status word).
 """
 import numpy as np
 import pytest
@@ -43,7 +43,7 @@ def test_wq_variant_matches_oracle(orc, T, K, N, cols, alpha, every):
     torch.cuda.synchronize()
     rows = None if every is None else np.arange(0, T, every, dtype=np.int32)
     Y_o, _, _, cnt = orc.mixed_linear(X, Wq_o, sW_o, None, alpha, rows=rows)
-    assert cnt <= i8.int8_mixed_linear_wq_max_outliers(K) or T <= 128
+    assert cnt <= i8.int8_mixed_linear_wq_max_outliers(K)
     assert_y_close(Y if rows is None else Y[rows], Y_o, f"wq T={T} K={K} N={N} |O|={cnt}")
     assert device_status_clean()
 
@@ -67,9 +67,10 @@ def test_wq_variant_differs_from_fp16_weights_only_in_outlier_rows(orc):
     assert device_status_clean()
 
 
-def test_wq_variant_reports_more_outliers_than_its_workspace_holds():
-    # alpha = 0 at prefill size makes every column an outlier: 1024 > 256 rows
-    T, K, N = 260, 1024, 256
+@pytest.mark.parametrize("T", [260, 16])
+def test_wq_variant_reports_more_outliers_than_its_workspace_holds(T):
+    # alpha = 0 makes every column an outlier: 1024 > 256 rows (prefill and decode)
+    K, N = 1024, 256
     assert i8.int8_mixed_linear_wq_max_outliers(K) == 256
     rng = np.random.default_rng(9)
     X = rng.standard_normal((T, K)).astype(np.float16)

@@ -58,6 +58,8 @@ constexpr int O_CHUNK = 64 * OBK * 2;   // 64 columns x 64 W16 rows (one 128-byt
 constexpr int THREADS = 224;       // warp 0 weight producer, 1 MMA, 2-5 epilogue, 6 outlier producer
 constexpr int MAX_T = 128;
 constexpr int MAX_STAGES = 8;
+constexpr int MAX_BUF = 4;         // TMEM accumulator buffers: the MMA runs up to three segments
+                                   // ahead of a finalising epilogue
 constexpr size_t SMEM_BUDGET = 200 * 1024;     // the weight ring
 constexpr size_t SMEM_MAX = 220 * 1024;        // ring + outlier buffer (a row-quantiser block still fits beside)
 static_assert(4 * O_CHUNK == A_BYTES, "an outlier stage's W16 rows fill the weight slot");
@@ -67,7 +69,9 @@ struct Params {
     int KB, num_tiles;
     long long total_units;
     int stages, stage_bytes;
-    uint32_t tmem_cols;            // power of two >= 4*TP, >= 32; buffer b at b*tmem_cols/2
+    uint32_t tmem_cols;            // nbuf * buf_cols (a power of two, <= 512)
+    uint32_t buf_cols;             // columns of one accumulator buffer: a power of two >= 2*TP, >= 32
+    int nbuf;                      // accumulator buffers (2 or 4), used in turn by the segments
     int32_t *acc32;                // [T,N] int32, zero on entry
     // finalisation (finalize != 0): Y from acc32 (and Yo) once a tile is complete
     int finalize;
@@ -86,8 +90,8 @@ struct Params {
 struct Barriers {
     uint64_t full[MAX_STAGES];
     uint64_t empty[MAX_STAGES];
-    uint64_t tmem_full[2];
-    uint64_t tmem_empty[2];
+    uint64_t tmem_full[MAX_BUF];
+    uint64_t tmem_empty[MAX_BUF];
     uint64_t ofull, oempty;        // the outlier buffer
     uint64_t drain;
     uint32_t tmem_base;
@@ -111,10 +115,12 @@ __device__ __forceinline__ int unit_owner(long long total, long long u, int ctas
     return static_cast<int>(((u + 1) * ctas - 1) / total);
 }
 
-// The stages of one CTA in order, the same for all its warps:
-//   for each tile its range [u0, u1) touches, the int8 k-blocks of that tile
-//   (kind 0, j = k-block), then, if the range holds the tile's k-block 0, the
-//   tile's nob outlier blocks (kind 1, j = outlier block).
+// The stages of one CTA in order, the same for all its warps: for each tile
+// its range [u0, u1) touches, first (if the range holds the tile's k-block 0)
+// the tile's nob outlier blocks (kind 1, j = outlier block), then the int8
+// k-blocks of that tile in the range (kind 0, j = k-block).  The CTA holding a
+// tile's k-block 0 reaches that tile last, so its int8 piece is usually the
+// tile's last one, and its outlier piece is stored just before.
 // A run of one kind for one tile is a segment: one TMEM accumulator buffer.
 // visit(kind, tile, j, first_of_segment, last_of_segment) returns false to stop.
 template <typename Visit>
@@ -123,11 +129,11 @@ __device__ __forceinline__ bool walk_stages(const Params &p, long long u0, long 
         const int tile = static_cast<int>(u / p.KB);
         const long long tile_u0 = static_cast<long long>(tile) * p.KB;
         const long long end = min(u1, tile_u0 + p.KB);
-        for (long long v = u; v < end; ++v)
-            if (!visit(0, tile, static_cast<int>(v - tile_u0), v == u, v == end - 1)) return false;
         if (u == tile_u0)
             for (int b = 0; b < nob; ++b)
                 if (!visit(1, tile, b, b == 0, b == nob - 1)) return false;
+        for (long long v = u; v < end; ++v)
+            if (!visit(0, tile, static_cast<int>(v - tile_u0), v == u, v == end - 1)) return false;
         u = end;
     }
     return true;
@@ -135,34 +141,47 @@ __device__ __forceinline__ bool walk_stages(const Params &p, long long u0, long 
 
 constexpr int FIN_ROWS = 16;
 
-// Y for the columns of one finished (tile, quadrant), from the int32 sums and
-// (with outliers) Yo; 16 rows at a time with all loads of a group in flight.
-__device__ __forceinline__ void finalize_columns(const Params &p, int tile, int quad, int lane, int count) {
-    const int nbase = tile * BM + quad * 32 + lane;
+// Y for the columns of one finished (tile, quadrant), both 128-column halves
+// 16 rows at a time with all their loads in flight together:
+//   Y[t,n] = fp16( (own[t,n] + acc32[t,n]) * sX[t] * sW[n] / 127^2 + Yo[t,n] )
+// own: this warp's partial sums still in TMEM (taddr, or none), acc32 read
+// only when other pieces were added there, Yo only when |O| > 0.
+__device__ __forceinline__ void finalize_columns(const Params &p, int tile, int quad, int lane, bool own,
+                                                 uint32_t taddr, bool read_acc, bool read_yo) {
+    const int n0 = tile * BM + quad * 32 + lane;
+    const bool ok0 = n0 < p.N, ok1 = n0 + BMH < p.N;
+    const float sw0 = ok0 ? p.sW[n0] : 0.0f, sw1 = ok1 ? p.sW[n0 + BMH] : 0.0f;
     for (int t0 = 0; t0 < p.T; t0 += FIN_ROWS) {
+        uint32_t r0[FIN_ROWS], r1[FIN_ROWS];
+        if (own) {
+            tmem_ld16(taddr + t0, r0);
+            tmem_ld16(taddr + p.TP + t0, r1);
+            tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int n = nbase + h * BMH;
-            if (n >= p.N) continue;
-            const float sw = p.sW[n];
-            int a[FIN_ROWS];
-            float yo[FIN_ROWS];
+            for (int r = 0; r < FIN_ROWS; ++r) r0[r] = r1[r] = 0u;
+        }
+        int a0[FIN_ROWS], a1[FIN_ROWS];
+        float y0[FIN_ROWS], y1[FIN_ROWS];
 #pragma unroll
-            for (int r = 0; r < FIN_ROWS; ++r) {
-                const bool ok = t0 + r < p.T;
-                const size_t at = static_cast<size_t>(t0 + r) * p.N + n;
-                a[r] = ok ? __ldcg(p.acc32 + at) : 0;
-                yo[r] = (ok && count > 0) ? __ldcg(p.Yo + at) : 0.0f;
-            }
+        for (int r = 0; r < FIN_ROWS; ++r) {
+            const bool row = t0 + r < p.T;
+            const size_t at = static_cast<size_t>(t0 + r) * p.N + n0;
+            a0[r] = (row && ok0 && read_acc) ? __ldcg(p.acc32 + at) : 0;
+            a1[r] = (row && ok1 && read_acc) ? __ldcg(p.acc32 + at + BMH) : 0;
+            y0[r] = (row && ok0 && read_yo) ? __ldcg(p.Yo + at) : 0.0f;
+            y1[r] = (row && ok1 && read_yo) ? __ldcg(p.Yo + at + BMH) : 0.0f;
+        }
 #pragma unroll
-            for (int r = 0; r < FIN_ROWS; ++r) {
-                const int t = t0 + r;
-                if (t < p.T) {
-                    const float rs = p.sX[t] * (1.0f / 16129.0f);
-                    p.Y[static_cast<size_t>(t) * p.N + n] =
-                        __float2half_rn(fmaf(static_cast<float>(a[r]), rs * sw, yo[r]));
-                }
-            }
+        for (int r = 0; r < FIN_ROWS; ++r) {
+            const int t = t0 + r;
+            if (t >= p.T) continue;
+            const float rs = p.sX[t] * (1.0f / 16129.0f);
+            const size_t at = static_cast<size_t>(t) * p.N + n0;
+            if (ok0)
+                p.Y[at] = __float2half_rn(fmaf(static_cast<float>(static_cast<int>(r0[r]) + a0[r]), rs * sw0, y0[r]));
+            if (ok1)
+                p.Y[at + BMH] = __float2half_rn(fmaf(static_cast<float>(static_cast<int>(r1[r]) + a1[r]), rs * sw1, y1[r]));
         }
     }
 }
@@ -184,7 +203,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&bars->full[s], 1);
             mbar_init(&bars->empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < MAX_BUF; ++b) {
             mbar_init(&bars->tmem_full[b], 1);
             mbar_init(&bars->tmem_empty[b], 4);
         }
@@ -204,7 +223,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
-    const uint32_t half_cols = p.tmem_cols / 2;
+    const uint32_t buf_cols = p.buf_cols;
 
     const long long u0 = unit_begin(p.total_units, blockIdx.x, gridDim.x);
     const long long u1 = unit_begin(p.total_units, blockIdx.x + 1, gridDim.x);
@@ -326,11 +345,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t id_f16 = idesc_f16(BMH, p.TP, true, false);
         int stage = 0, seg = 0;
         uint32_t phase = 0, ophase = 0;
-        uint32_t tph[2] = {0, 0};
+        uint32_t tph = 0;                                 // bit b: phase of buffer b
         walk_stages(p, u0, u1, nob, [&](int kind, int, int j, bool first, bool last) -> bool {
-            const int buf = seg & 1;
+            const int buf = seg % p.nbuf;
             if (first) {
-                if (!warp_wait(&bars->tmem_empty[buf], tph[buf] ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
+                if (!warp_wait(&bars->tmem_empty[buf], ((tph >> buf) & 1u) ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
                 tc_fence_after_sync();
             }
             uint64_t *fb = kind == 0 ? &bars->full[stage] : &bars->ofull;
@@ -338,7 +357,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after_sync();
             if (kind == 1) fence_proxy_async_smem();      // cp.async rows -> tensor core reads
             if (lane == 0) {
-                const uint32_t d0 = tmem + static_cast<uint32_t>(buf) * half_cols;
+                const uint32_t d0 = tmem + static_cast<uint32_t>(buf) * buf_cols;
                 const uint32_t d1 = d0 + static_cast<uint32_t>(p.TP);
                 const uint32_t a = kind == 0 ? smem_u32(smem + static_cast<size_t>(stage) * p.stage_bytes) : smem_u32(ob);
                 const uint32_t b = a + A_BYTES;
@@ -366,7 +385,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             __syncwarp();
             if (last) {
-                tph[buf] ^= 1u;
+                tph ^= 1u << buf;
                 ++seg;
             }
             if (kind == 0) {
@@ -385,58 +404,77 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;
-        uint32_t tph[2] = {0, 0};
+        uint32_t tph = 0;
         int seg = 0;
         walk_stages(p, u0, u1, nob, [&](int kind, int tile, int, bool, bool last) -> bool {
             if (!last) return true;
-            const int buf = seg & 1;
-            if (!warp_wait(&bars->tmem_full[buf], tph[buf], abort, I8R_DEV_TMEM_TIMEOUT)) return false;
+            const int buf = seg % p.nbuf;
+            if (!warp_wait(&bars->tmem_full[buf], (tph >> buf) & 1u, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
             tc_fence_after_sync();
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf) * half_cols;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf) * buf_cols;
+            // pieces of this tile: one per CTA holding some of its k-blocks, plus
+            // the outlier piece
+            const long long tile_u0 = static_cast<long long>(tile) * p.KB;
+            const int int8_pieces = unit_owner(p.total_units, tile_u0 + p.KB - 1, gridDim.x) -
+                                    unit_owner(p.total_units, tile_u0, gridDim.x) + 1;
+            const int pieces = int8_pieces + (nob > 0 ? 1 : 0);
+            int* counter = p.counters + tile * 4 + quad;
+            // An int8 piece that finds every other piece already counted is the
+            // tile's last: it writes Y from its own sums in TMEM (plus acc32 when
+            // other CTAs added theirs there) and needs neither the atomic adds nor
+            // the re-read.  Counted pieces were published before they were counted.
+            int last_piece = 0;
+            if (kind == 0 && p.finalize) {
+                if (lane == 0) last_piece = atomicAdd(counter, 0) == pieces - 1;
+                last_piece = __shfl_sync(0xFFFFFFFFu, last_piece, 0);
+            }
+            if (last_piece) {
+                __threadfence();
+                finalize_columns(p, tile, quad, lane, true, taddr, int8_pieces > 1, nob > 0);
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
+            } else {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int n = tile * BM + h * BMH + quad * 32 + lane;   // this thread's column
-                for (int c = 0; c < p.TP; c += 16) {
-                    uint32_t r[16];
-                    tmem_ld16(taddr + h * p.TP + c, r);
-                    tmem_wait_ld();
-                    if (n < p.N) {
+                for (int h = 0; h < 2; ++h) {
+                    const int n = tile * BM + h * BMH + quad * 32 + lane;   // this thread's column
+                    for (int c = 0; c < p.TP; c += 16) {
+                        uint32_t r[16];
+                        tmem_ld16(taddr + h * p.TP + c, r);
+                        tmem_wait_ld();
+                        if (n < p.N) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int t = c + i;
-                            if (t >= p.T) continue;
-                            const size_t at = static_cast<size_t>(t) * p.N + n;
-                            if (kind == 0) {
-                                if (r[i] != 0u) atomicAdd(p.acc32 + at, static_cast<int>(r[i]));
-                            } else {
-                                __stcg(p.Yo + at, __uint_as_float(r[i]));
+                            for (int i = 0; i < 16; ++i) {
+                                const int t = c + i;
+                                if (t >= p.T) continue;
+                                const size_t at = static_cast<size_t>(t) * p.N + n;
+                                if (kind == 0) {
+                                    if (r[i] != 0u) atomicAdd(p.acc32 + at, static_cast<int>(r[i]));
+                                } else {
+                                    __stcg(p.Yo + at, __uint_as_float(r[i]));
+                                }
                             }
                         }
                     }
                 }
-            }
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
-            if (p.finalize) {
-                // publish this warp's piece, then count it
-                __threadfence();
+                tc_fence_before_sync();
                 __syncwarp();
-                int done = 0;
-                if (lane == 0) {
-                    const long long tile_u0 = static_cast<long long>(tile) * p.KB;
-                    const int pieces = unit_owner(p.total_units, tile_u0 + p.KB - 1, gridDim.x) -
-                                       unit_owner(p.total_units, tile_u0, gridDim.x) + 1 + (nob > 0 ? 1 : 0);
-                    const int before = atomicAdd(p.counters + tile * 4 + quad, 1);
-                    done = before == pieces - 1;
-                }
-                done = __shfl_sync(0xFFFFFFFFu, done, 0);
-                if (done) {
+                if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
+                if (p.finalize) {
+                    // publish this warp's piece, then count it; the piece that
+                    // completes the count writes Y from acc32 (and Yo)
                     __threadfence();
-                    finalize_columns(p, tile, quad, lane, count);
+                    __syncwarp();
+                    int done = 0;
+                    if (lane == 0) done = atomicAdd(counter, 1) == pieces - 1;
+                    done = __shfl_sync(0xFFFFFFFFu, done, 0);
+                    if (done) {
+                        __threadfence();
+                        finalize_columns(p, tile, quad, lane, false, 0u, true, nob > 0);
+                    }
                 }
             }
-            tph[buf] ^= 1u;
+            tph ^= 1u << buf;
             ++seg;
             return true;
         });

@@ -501,8 +501,10 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.obuf = (fin && fin->obuf) ? 1 : 0;
     while (p.obuf && p.stages > 2 && static_cast<size_t>(p.stages + 1) * p.stage_bytes > decode::SMEM_MAX) --p.stages;
     uint32_t cols = 32;
-    while (cols < static_cast<uint32_t>(4 * p.TP)) cols <<= 1;
-    p.tmem_cols = cols;
+    while (cols < static_cast<uint32_t>(2 * p.TP)) cols <<= 1;
+    p.buf_cols = cols;
+    p.nbuf = cols * decode::MAX_BUF <= 512 ? decode::MAX_BUF : 2;
+    p.tmem_cols = cols * static_cast<uint32_t>(p.nbuf);
     p.acc32 = acc32;
     CUtensorMap map_wq, map_xq, map_xo, map_w16o;
     // Two 128-column boxes per stage cover 256 contiguous bytes of every weight

@@ -20,12 +20,12 @@
 // with A = the W16 rows of the outliers (MN-major, copied in place by the
 // lanes with cp.async, 16 bytes each, or the dequantised rows the quantiser
 // compacted for the Wq-only variant) and B = Xo (K-major), and stores it to
-// Yo [T,N].  Those stages have a shared-memory buffer of their own, filled
-// by a second producer warp, so the row copies never hold up the weight
-// stream's requests.  Each buffer (the weight ring, the outlier buffer) has
-// exactly one producer, which waits on every use of every slot: a parity
-// wait cannot tell a phase from the one two uses later, so a producer that
-// skipped slots could get two phases ahead of the consumer.
+// Yo [T,N].  Those stages go through the same ring as the weight stages,
+// filled by the same (only) producer warp: a parity wait cannot tell a phase
+// from the one two uses later, so every slot has one producer that waits on
+// each of its uses.  The row copies do not stall that warp: each lane hands
+// its cp.async copies to the stage's barrier (cp.async.mbarrier.arrive), so
+// several outlier stages can be in flight at once.
 //
 // Finalisation: after adding its partial sums (or storing its Yo piece),
 // each epilogue warp bumps a counter for its (tile, 32-lane quadrant).  The
@@ -55,13 +55,12 @@ constexpr int A_BYTES = 2 * A_HALF;
 constexpr int OBK = 64;            // outliers per outlier stage: 64 W16 rows x 256 columns = A_BYTES,
                                    // and T x 64 fp16 of Xo = the bytes of a T x 128 Xq tile
 constexpr int O_CHUNK = 64 * OBK * 2;   // 64 columns x 64 W16 rows (one 128-byte swizzle span)
-constexpr int THREADS = 224;       // warp 0 weight producer, 1 MMA, 2-5 epilogue, 6 outlier producer
+constexpr int THREADS = 192;       // warp 0 producer, 1 MMA, 2-5 epilogue
 constexpr int MAX_T = 128;
 constexpr int MAX_STAGES = 8;
 constexpr int MAX_BUF = 4;         // TMEM accumulator buffers: the MMA runs up to three segments
                                    // ahead of a finalising epilogue
-constexpr size_t SMEM_BUDGET = 200 * 1024;     // the weight ring
-constexpr size_t SMEM_MAX = 220 * 1024;        // ring + outlier buffer (a row-quantiser block still fits beside)
+constexpr size_t SMEM_BUDGET = 200 * 1024;
 static_assert(4 * O_CHUNK == A_BYTES, "an outlier stage's W16 rows fill the weight slot");
 
 struct Params {
@@ -82,7 +81,7 @@ struct Params {
     const __half *W16;             // [K,N] fp16 (null for the Wq-only variant)
     int o_rows;                    // Wq-only variant: rows of the compacted, dequantised W16o
     int wq_only;                   // no W16: outlier rows come from W16o (zeros past o_rows)
-    int obuf;                      // 1: the outlier buffer exists (else the 16-bit part is skipped)
+    int may_outlier;               // alpha < +inf: a tile's first stage may be an outlier stage
     __half *Y;
     float *Yo;                     // [T,N] fp32: the 16-bit outlier part (written when |O| > 0)
 };
@@ -92,18 +91,16 @@ struct Barriers {
     uint64_t empty[MAX_STAGES];
     uint64_t tmem_full[MAX_BUF];
     uint64_t tmem_empty[MAX_BUF];
-    uint64_t ofull, oempty;        // the outlier buffer
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
 };
 
-// The weight ring (stages x stage_bytes), the outlier buffer (obuf x
-// stage_bytes: 64 W16 rows of a tile = A_BYTES, and T x 64 fp16 of Xo), then
-// the barriers; 1024 bytes for aligning the base to the 128-byte swizzle's
-// 1024-byte period.
-__host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes, int obuf) {
-    return 1024 + static_cast<size_t>(stages + obuf) * stage_bytes + sizeof(Barriers);
+// The ring (stages x stage_bytes; an outlier stage, 64 W16 rows of a tile and
+// T x 64 fp16 of Xo, has the size of a weight stage), then the barriers;
+// 1024 bytes for aligning the base to the 128-byte swizzle's 1024-byte period.
+__host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes) {
+    return 1024 + static_cast<size_t>(stages) * stage_bytes + sizeof(Barriers);
 }
 
 // CTA c of `ctas` owns units [floor(c*U/ctas), floor((c+1)*U/ctas)).
@@ -192,8 +189,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                        const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *ob = smem + static_cast<size_t>(p.stages) * p.stage_bytes;      // the outlier buffer
-    Barriers *bars = reinterpret_cast<Barriers *>(ob + static_cast<size_t>(p.obuf) * p.stage_bytes);
+    Barriers *bars = reinterpret_cast<Barriers *>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);
     volatile int *abort = &bars->abort;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -207,8 +203,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&bars->tmem_full[b], 1);
             mbar_init(&bars->tmem_empty[b], 4);
         }
-        mbar_init(&bars->ofull, 1);
-        mbar_init(&bars->oempty, 1);
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         fence_mbar_init();
@@ -229,10 +223,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const long long u1 = unit_begin(p.total_units, blockIdx.x + 1, gridDim.x);
     const uint32_t tx = static_cast<uint32_t>(p.stage_bytes);
 
-    // Weight tiles of the first stages (all in the first segment, which is
-    // int8) do not depend on the activation kernels: request them first.
+    // Weight tiles of the first stages do not depend on the activation kernels:
+    // request them first.  Only the first segment's, and none when the range
+    // starts a tile that may open with outlier stages (|O| is not known yet).
     const long long first_seg = min(u1, (u0 / p.KB + 1) * p.KB) - u0;
-    const int pre = static_cast<int>(min(static_cast<long long>(p.stages), first_seg));
+    const int pre = (p.may_outlier && u0 % p.KB == 0) ? 0 : static_cast<int>(min(static_cast<long long>(p.stages), first_seg));
     if (warp == 0 && lane == 0) {
         for (int i = 0; i < pre; ++i) {
             const long long u = u0 + i;
@@ -246,105 +241,87 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     griddep_wait();                               // activation, |O|, acc32 / counters zeroed
     const int count = p.finalize ? *p.count : 0;
-    const int nob = p.obuf ? (count + OBK - 1) / OBK : 0;
+    const int nob = p.may_outlier ? (count + OBK - 1) / OBK : 0;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ weight producer
+        // ------------------------------------------------------------ producer
+        if (nob > 0 && lane == 0) {
+            if (p.wq_only) tma_prefetch_map(&map_w16o);
+            tma_prefetch_map(&map_xo);
+        }
         int pending[MAX_STAGES];
         for (int s = 0; s < MAX_STAGES; ++s) pending[s] = -1;
         int stage = 0, n = 0;
         uint32_t phase = 0;
         const bool ok = walk_stages(p, u0, u1, nob, [&](int kind, int tile, int j, bool, bool) -> bool {
-            if (kind != 0) return true;                   // outlier stages: the other producer
             uint8_t *a = smem + static_cast<size_t>(stage) * p.stage_bytes;
             uint64_t *fb = &bars->full[stage];
-            if (n < pre) {
+            if (kind == 0 && n < pre) {
                 if (lane == 0) tma_load_2d(a + A_BYTES, &map_xq, fb, j * BK, 0);
             } else {
                 if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(fb, tx);
-                    tma_load_2d(a, &map_wq, fb, tile * BM, j * BK);
-                    tma_load_2d(a + A_HALF, &map_wq, fb, tile * BM + BMH, j * BK);
-                    tma_load_2d(a + A_BYTES, &map_xq, fb, j * BK, 0);
+                if (kind == 0) {
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(fb, tx);
+                        tma_load_2d(a, &map_wq, fb, tile * BM, j * BK);
+                        tma_load_2d(a + A_HALF, &map_wq, fb, tile * BM + BMH, j * BK);
+                        tma_load_2d(a + A_BYTES, &map_xq, fb, j * BK, 0);
+                    }
+                } else if (p.wq_only) {
+                    // compacted dequantised rows; past o_rows an out-of-range box, i.e.
+                    // zeros (the quantiser reports the overflow)
+                    if (lane == 0) {
+                        const int y = (j + 1) * OBK <= p.o_rows ? j * OBK : p.o_rows;
+                        mbar_arrive_expect_tx(fb, tx);
+                        tma_load_2d(a + A_BYTES, &map_xo, fb, j * OBK, 0);
+                        for (int c = 0; c < 4; ++c) tma_load_2d(a + c * O_CHUNK, &map_w16o, fb, tile * BM + 64 * c, y);
+                    }
+                } else {
+                    // The W16 rows of outliers j*64 .., zero past |O| rounded up to 16
+                    // (the MMAs read no further): lane l copies columns 8l .. 8l+7 of
+                    // every row into the 128-byte-swizzled chunk l/8 and hands the
+                    // copies to the stage's barrier; lane 0 then adds the Xo tile.
+                    // (The MMA warp fences to the async proxy before reading.)
+                    const int rows = min(OBK, (count - j * OBK + 15) / 16 * 16);
+                    const int g0 = j * OBK + lane, g1 = j * OBK + 32 + lane;
+                    const int k0 = g0 < count ? p.idx[g0] : -1;
+                    const int k1 = g1 < count ? p.idx[g1] : -1;
+                    const int col = tile * BM + lane * 8;
+                    const uint32_t chunk = smem_u32(a) + static_cast<uint32_t>((lane >> 3) * O_CHUNK);
+                    const uint32_t unit = static_cast<uint32_t>(lane & 7);
+                    for (int r = 0; r < rows; ++r) {
+                        const int k = __shfl_sync(0xFFFFFFFFu, r < 32 ? k0 : k1, r & 31);
+                        const bool have = k >= 0 && col < p.N;
+                        const __half *src = have ? p.W16 + static_cast<size_t>(k) * p.N + col : p.W16;
+                        cp_async_16(chunk + static_cast<uint32_t>(r * 128) + ((unit ^ static_cast<uint32_t>(r & 7)) << 4),
+                                    src, have ? 16u : 0u);
+                    }
+                    cp_async_mbar_arrive(fb);
+                    __syncwarp();                          // every lane's copies tracked before the arrive
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.TP * OBK * 2));
+                        tma_load_2d(a + A_BYTES, &map_xo, fb, j * OBK, 0);
+                    }
                 }
             }
             if (lane == 0) pending[stage] = static_cast<int>(phase);
-            ++n;
+            if (kind == 0) ++n;
             __syncwarp();
             if (++stage == p.stages) { stage = 0; phase ^= 1u; }
             return true;
         });
         if (!ok && lane == 0) {
-            // let the loads already issued land before the CTA leaves (abort only)
+            // let the loads and copies already issued land before the CTA leaves (abort only)
             volatile int never = 0;
             for (int s = 0; s < p.stages; ++s)
                 if (pending[s] >= 0) mbar_wait(&bars->full[s], static_cast<uint32_t>(pending[s]), &never, 0);
-        }
-    } else if (warp == 6) {
-        // ------------------------------------------------------------ outlier producer
-        if (nob > 0 && lane == 0) {
-            if (p.wq_only) tma_prefetch_map(&map_w16o);
-            tma_prefetch_map(&map_xo);
-        }
-        uint32_t ophase = 0;
-        int pending = -1;
-        const bool ok = walk_stages(p, u0, u1, nob, [&](int kind, int tile, int j, bool, bool) -> bool {
-            if (kind != 1) return true;
-            if (!warp_wait(&bars->oempty, ophase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
-            uint64_t *fb = &bars->ofull;
-            if (p.wq_only) {
-                // compacted dequantised rows; past o_rows an out-of-range box, i.e.
-                // zeros (the quantiser reports the overflow)
-                if (lane == 0) {
-                    const int y = (j + 1) * OBK <= p.o_rows ? j * OBK : p.o_rows;
-                    mbar_arrive_expect_tx(fb, tx);
-                    tma_load_2d(ob + A_BYTES, &map_xo, fb, j * OBK, 0);
-                    for (int c = 0; c < 4; ++c) tma_load_2d(ob + c * O_CHUNK, &map_w16o, fb, tile * BM + 64 * c, y);
-                }
-            } else {
-                // The W16 rows of outliers j*64 .., zero past |O| rounded up to 16
-                // (the MMAs read no further): lane l copies columns 8l .. 8l+7 of
-                // every row into the 128-byte-swizzled chunk l/8, then the rows
-                // are made visible to the tensor core (async proxy) before the
-                // stage is published with its Xo tile.
-                const int rows = min(OBK, (count - j * OBK + 15) / 16 * 16);
-                const int g0 = j * OBK + lane, g1 = j * OBK + 32 + lane;
-                const int k0 = g0 < count ? p.idx[g0] : -1;
-                const int k1 = g1 < count ? p.idx[g1] : -1;
-                const int col = tile * BM + lane * 8;
-                const uint32_t chunk = smem_u32(ob) + static_cast<uint32_t>((lane >> 3) * O_CHUNK);
-                const uint32_t unit = static_cast<uint32_t>(lane & 7);
-                for (int r = 0; r < rows; ++r) {
-                    const int k = __shfl_sync(0xFFFFFFFFu, r < 32 ? k0 : k1, r & 31);
-                    const bool have = k >= 0 && col < p.N;
-                    const __half *src = have ? p.W16 + static_cast<size_t>(k) * p.N + col : p.W16;
-                    cp_async_16(chunk + static_cast<uint32_t>(r * 128) + ((unit ^ static_cast<uint32_t>(r & 7)) << 4),
-                                src, have ? 16u : 0u);
-                }
-                cp_async_wait_all();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.TP * OBK * 2));
-                    tma_load_2d(ob + A_BYTES, &map_xo, fb, j * OBK, 0);
-                }
-            }
-            pending = static_cast<int>(ophase);
-            __syncwarp();
-            ophase ^= 1u;
-            return true;
-        });
-        if (!ok && lane == 0 && pending >= 0) {
-            volatile int never = 0;
-            mbar_wait(&bars->ofull, static_cast<uint32_t>(pending), &never, 0);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         const uint32_t id_i8 = idesc_i8(BMH, p.TP, true, false);
         const uint32_t id_f16 = idesc_f16(BMH, p.TP, true, false);
         int stage = 0, seg = 0;
-        uint32_t phase = 0, ophase = 0;
+        uint32_t phase = 0;
         uint32_t tph = 0;                                 // bit b: phase of buffer b
         walk_stages(p, u0, u1, nob, [&](int kind, int, int j, bool first, bool last) -> bool {
             const int buf = seg % p.nbuf;
@@ -352,14 +329,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!warp_wait(&bars->tmem_empty[buf], ((tph >> buf) & 1u) ^ 1u, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
                 tc_fence_after_sync();
             }
-            uint64_t *fb = kind == 0 ? &bars->full[stage] : &bars->ofull;
-            if (!warp_wait(fb, kind == 0 ? phase : ophase, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+            if (!warp_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
             tc_fence_after_sync();
             if (kind == 1) fence_proxy_async_smem();      // cp.async rows -> tensor core reads
             if (lane == 0) {
                 const uint32_t d0 = tmem + static_cast<uint32_t>(buf) * buf_cols;
                 const uint32_t d1 = d0 + static_cast<uint32_t>(p.TP);
-                const uint32_t a = kind == 0 ? smem_u32(smem + static_cast<size_t>(stage) * p.stage_bytes) : smem_u32(ob);
+                const uint32_t a = smem_u32(smem + static_cast<size_t>(stage) * p.stage_bytes);
                 const uint32_t b = a + A_BYTES;
                 if (kind == 0) {
 #pragma unroll
@@ -380,7 +356,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         mma_f16(d1, smem_desc_sw128(a + A_HALF + kk * 16 * 128, O_CHUNK, 1024), bd, id_f16, acc);
                     }
                 }
-                mma_commit(kind == 0 ? &bars->empty[stage] : &bars->oempty);
+                mma_commit(&bars->empty[stage]);
                 if (last) mma_commit(&bars->tmem_full[buf]);
             }
             __syncwarp();
@@ -388,11 +364,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tph ^= 1u << buf;
                 ++seg;
             }
-            if (kind == 0) {
-                if (++stage == p.stages) { stage = 0; phase ^= 1u; }
-            } else {
-                ophase ^= 1u;
-            }
+            if (++stage == p.stages) { stage = 0; phase ^= 1u; }
             return true;
         });
         if (lane == 0) {

@@ -118,7 +118,7 @@ i8r_status device_setup(const DeviceInfo **out) {
             I8R_CUDA(cudaOccupancyMaxActiveClusters(&d.pair_clusters, prefill2::gemm_prefill_pair_kernel<false>, &cfg));
             if (d.pair_clusters < 1) return I8R_EARCH;
             I8R_CUDA(cudaFuncSetAttribute(decode::gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(decode::SMEM_MAX + 4096)));
+                                          static_cast<int>(decode::SMEM_BUDGET + 4096)));
         }
         if (!g_encode) {
             void *fn = nullptr;
@@ -498,8 +498,7 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.stage_bytes = decode::A_BYTES + p.TP * decode::BK;
     p.stages = static_cast<int>(decode::SMEM_BUDGET / p.stage_bytes);
     if (p.stages > decode::MAX_STAGES) p.stages = decode::MAX_STAGES;
-    p.obuf = (fin && fin->obuf) ? 1 : 0;
-    while (p.obuf && p.stages > 2 && static_cast<size_t>(p.stages + 1) * p.stage_bytes > decode::SMEM_MAX) --p.stages;
+    p.may_outlier = (fin && fin->may_outlier) ? 1 : 0;
     uint32_t cols = 32;
     while (cols < static_cast<uint32_t>(2 * p.TP)) cols <<= 1;
     p.buf_cols = cols;
@@ -518,7 +517,7 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
         if (W16o) I8R_TRY(make_map(&map_w16o, W16o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.o_rows, N, 64, 64));
     }
     const long long g = p.total_units < dev->sms ? p.total_units : dev->sms;
-    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes, p.obuf);
+    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes);
     record_before(s);
     cudaError_t e = launch_dependent(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(g)),
                                      dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, map_xo, map_w16o, p);
@@ -668,7 +667,7 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     fin.idx = idx;
     fin.o_rows = wq_only ? compact_rows(K, true) : 0;
     fin.wq_only = wq_only ? 1 : 0;
-    fin.obuf = std::isinf(alpha) ? 0 : 1;          // alpha = +inf: no finite input is an outlier
+    fin.may_outlier = std::isinf(alpha) ? 0 : 1;   // alpha = +inf: no finite input is an outlier
     fin.Y = y;
     fin.Yo = Yo;
     return launch_decode(dev, Xq, T, K, Wq, N, acc32, &fin, stream, Xo, w16, W16o);

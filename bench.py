@@ -53,6 +53,11 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="time every point of the 175B decoder-layer sweep in one process (one JSON line each; "
                          "not the one-line contract run)")
+    ap.add_argument("--chain", action="store_true",
+                    help="time the 175B decoder layer's four projections (qkv, out, fc1, fc2) as one "
+                         "int8_mixed_linear_chain call replayed from a CUDA graph (one JSON line; "
+                         "not the one-line contract run)")
+    ap.add_argument("--chain-t", type=int, default=16, help="tokens per projection for --chain")
     ap.add_argument("--variant", default="w16", choices=["w16", "wq"],
                     help="w16: int8_mixed_linear (fp16 weight resident for the outlier rows); "
                          "wq: int8_mixed_linear_wq (only Wq and sW resident)")
@@ -505,10 +510,83 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_chain(args):
+    """The 175B decoder layer's projections qkv, out, fc1 and fc2 (each with its
+    own seeded input of 0.1 % outlier columns, alpha 6) as one
+    int8_mixed_linear_chain call: sixteen launches, captured once into a CUDA
+    graph and replayed.  The weights (1.8 GB of int8) exceed L2, so every
+    replay streams them from HBM.  Each layer is also timed alone, eagerly."""
+    import torch
+    import int8_quantized_row_b200 as i8
+    dev = torch.device("cuda", 0)
+    pk = peaks()
+    T, alpha, frac = args.chain_t, 6.0, 0.001
+    layers, meta = [], []
+    for seed, (name, (K, N)) in enumerate(wl.SWEEP_LAYERS.items()):
+        W = torch.from_numpy(wl.make_w(K, N, 0.01)).to(dev)
+        Wq, sW = i8.int8_quantize_weight_colwise(W)
+        n_out = int(round(frac * K))
+        X = torch.from_numpy(wl.make_x(T, K, n_out, 6.0, 60.0, 1.0, seed)).to(dev)
+        layers.append((X, Wq, sW, None if args.variant == "wq" else W, alpha,
+                       torch.empty((T, N), dtype=torch.float16, device=dev)))
+        meta.append(dict(layer=name, K=K, N=N, outlier_cols=int(i8.int8_outlier_stats(X, alpha)[0].item())))
+    ws = torch.empty(max(1, i8.int8_mixed_linear_chain_workspace_size(layers)), dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            i8.int8_mixed_linear_chain(layers, workspace_buf=ws, stream=side)
+        side.synchronize()
+        with torch.cuda.graph(graph, stream=side):
+            i8.int8_mixed_linear_chain(layers, workspace_buf=ws, stream=side)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        graph.replay()
+    torch.cuda.synchronize()
+    steps = min(args.steps, 500)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        graph.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    # each layer alone, eager calls on the same workspace
+    for m, (X, Wq, sW, W, al, Y) in zip(meta, layers):
+        for _ in range(3):
+            i8.int8_mixed_linear_chain([(X, Wq, sW, W, al, Y)], workspace_buf=ws)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(steps):
+            i8.int8_mixed_linear_chain([(X, Wq, sW, W, al, Y)], workspace_buf=ws)
+        b.record(stream)
+        torch.cuda.synchronize()
+        m["ms_eager"] = a.elapsed_time(b) / steps
+    ops = sum(2.0 * T * m["K"] * m["N"] for m in meta)
+    wbytes = sum(m["K"] * m["N"] + 4 * m["N"] + (1 if args.variant == "wq" else 2) * m["outlier_cols"] * m["N"]
+                 for m in meta)
+    io_bytes = sum(2 * T * (m["K"] + m["N"]) for m in meta)
+    line = {"metric": "175B decoder-layer projections (qkv, out, fc1, fc2) as one int8_mixed_linear_chain call, "
+                      "CUDA-graph replay",
+            "value": ops / (ms * 1e-3) / 1e12, "unit": "TOPS", "ms_per_chain": ms, "steps": steps,
+            "T": T, "alpha": alpha, "variant": args.variant, "graph": True, "launches_per_chain": 4 * len(meta),
+            "weight_bytes": wbytes, "weight_gbs": wbytes / (ms * 1e-3) / 1e9,
+            "frac_hbm": (wbytes + io_bytes) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "peak_hbm_gbs": pk["hbm_gbs"], "peak_src": pk["src"],
+            "sum_of_eager_layer_ms": sum(m["ms_eager"] for m in meta), "layers": meta,
+            "data": "synthetic, seeded", "status": i8.int8_read_and_clear_device_status()}
+    del graph
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.sweep:
         run_sweep(args)
+        return
+    if args.chain:
+        run_chain(args)
         return
     cfgs = all_configs()
     if args.workload not in cfgs:

@@ -143,6 +143,40 @@ i8r_status int8_mixed_linear_wq(const void *X, int T, int K,
                                 cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * int8_mixed_linear_chain: several int8_mixed_linear layers run in order on one
+ * stream with one shared workspace: the projections of a decoder layer (the
+ * pages' unit of use: the Int8 multiplication of the feed-forward and
+ * attention projection layers; LLM.int8() abstract).
+ *
+ *   layers  [n] host array of i8r_layer; each entry has the meaning of the
+ *           int8_mixed_linear arguments of the same names (W16 may be null
+ *           for the Wq-only variant, as in int8_mixed_linear_wq).  A layer's
+ *           X may be an earlier layer's Y: the layers run one after the
+ *           other in stream order, so each sees the Y of those before it.
+ *   workspace  at least int8_mixed_linear_chain_workspace_size(n, layers)
+ *           bytes (the largest layer's need), 256-byte aligned.
+ * Every layer is checked on the host before anything is enqueued; a bad
+ * layer returns its error and enqueues nothing.  n = 0 is a no-op.  The call
+ * is asynchronous and graph-capturable, like int8_mixed_linear.
+ * ------------------------------------------------------------------------- */
+typedef struct {
+    const void *X;            /* [T,K] fp16 */
+    int T, K;
+    const int8_t *Wq;         /* [K,N] int8 */
+    const float *sW;          /* [N] fp32 */
+    const void *W16;          /* [K,N] fp16, or null: outlier rows dequantised from Wq */
+    int N;
+    float alpha;
+    void *Y;                  /* [T,N] fp16 */
+} i8r_layer;
+
+size_t int8_mixed_linear_chain_workspace_size(int n, const i8r_layer *layers);
+
+i8r_status int8_mixed_linear_chain(int n, const i8r_layer *layers,
+                                   void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * int8_mixed_linear_noalloc: the same layer, with no workspace argument and no
  * device allocation of any kind.  The paper has no counterpart; this entry
  * point exists for callers that cannot allocate device memory where they call

@@ -58,6 +58,9 @@ def lib():
     so.int8_mixed_linear_wq_max_outliers.argtypes = [_I]
     so.int8_mixed_linear_wq_max_outliers.restype = _I
     so.int8_mixed_linear_wq.argtypes = [_P, _I, _I, _P, _P, _I, _F, _P, _P, _Z, _P]
+    so.int8_mixed_linear_chain_workspace_size.argtypes = [_I, _P]
+    so.int8_mixed_linear_chain_workspace_size.restype = _Z
+    so.int8_mixed_linear_chain.argtypes = [_I, _P, _P, _Z, _P]
     so.int8_outlier_stats_workspace_size.argtypes = [_I]
     so.int8_outlier_stats_workspace_size.restype = _Z
     so.int8_outlier_stats.argtypes = [_P, _I, _I, _F, _P, _P, _P, _P, _P, _Z, _P]
@@ -166,6 +169,46 @@ def int8_mixed_linear_wq(X, Wq, sW, alpha=6.0, Y=None, workspace_buf=None, strea
         N, float(alpha), _dev(Y, torch.float16, "Y"),
         ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(), _stream(stream)))
     return Y
+
+
+class I8rLayer(ctypes.Structure):
+    """One layer of int8_mixed_linear_chain (the C struct i8r_layer)."""
+    _fields_ = [("X", _P), ("T", _I), ("K", _I), ("Wq", _P), ("sW", _P), ("W16", _P), ("N", _I),
+                ("alpha", _F), ("Y", _P)]
+
+
+def _chain_layers(layers):
+    import torch
+    descs, outs = [], []
+    for X, Wq, sW, W16, alpha, Y in layers:
+        T, K = X.shape
+        N = Wq.shape[1]
+        Y = torch.empty((T, N), dtype=torch.float16, device=X.device) if Y is None else Y
+        w16 = _dev(W16, torch.float16, "W16", 2) if W16 is not None else _P()
+        descs.append(I8rLayer(_dev(X, torch.float16, "X", 2), T, K, _dev(Wq, torch.int8, "Wq", 2),
+                              _dev(sW, torch.float32, "sW"), w16, N, float(alpha), _dev(Y, torch.float16, "Y")))
+        outs.append(Y)
+    return (I8rLayer * max(1, len(descs)))(*descs), outs
+
+
+def int8_mixed_linear_chain_workspace_size(layers):
+    arr, _ = _chain_layers(layers)
+    return int(lib().int8_mixed_linear_chain_workspace_size(len(layers), ctypes.cast(arr, _P)))
+
+
+def int8_mixed_linear_chain(layers, workspace_buf=None, stream=None):
+    """Run layers in order on one stream with one workspace.  layers: a list of
+    (X, Wq, sW, W16 or None, alpha, Y or None); returns the list of Y."""
+    import torch
+    arr, outs = _chain_layers(layers)
+    if workspace_buf is None:
+        need = int(lib().int8_mixed_linear_chain_workspace_size(len(layers), ctypes.cast(arr, _P)))
+        dev = layers[0][0].device if layers else "cuda"
+        workspace_buf = torch.empty(max(1, need), dtype=torch.uint8, device=dev)
+    _check("int8_mixed_linear_chain", lib().int8_mixed_linear_chain(
+        len(layers), ctypes.cast(arr, _P), ctypes.c_void_p(workspace_buf.data_ptr()),
+        workspace_buf.numel() * workspace_buf.element_size(), _stream(stream)))
+    return outs
 
 
 def int8_outlier_stats_workspace_size(K):

@@ -693,6 +693,45 @@ i8r_status int8_mixed_linear_wq(const void *X, int T, int K, const int8_t *Wq, c
     return mixed_linear_impl(X, T, K, Wq, sW, nullptr, N, alpha, Y, workspace, workspace_bytes, stream);
 }
 
+size_t int8_mixed_linear_chain_workspace_size(int n, const i8r_layer *layers) {
+    if (n < 0 || (n > 0 && !layers)) return 0;
+    size_t need = 0;
+    for (int i = 0; i < n; ++i) {
+        const i8r_layer &l = layers[i];
+        if (l.T < 0 || l.K < 0 || l.N < 0) return 0;
+        need = std::max(need, ws_layout(l.T, l.K, l.N, l.W16 == nullptr).total);
+    }
+    return need;
+}
+
+i8r_status int8_mixed_linear_chain(int n, const i8r_layer *layers, void *workspace, size_t workspace_bytes,
+                                   cudaStream_t stream) {
+    if (n < 0 || (n > 0 && !layers)) return I8R_EINVAL;
+    // every layer is checked before anything is enqueued
+    for (int i = 0; i < n; ++i) {
+        const i8r_layer &l = layers[i];
+        I8R_TRY(check_shape(l.T, l.K, l.N, true));
+        if (std::isnan(l.alpha) || l.alpha < 0.0f) return I8R_EINVAL;
+        if (l.T == 0) continue;
+        I8R_TRY(check_ptr(l.X));
+        I8R_TRY(check_ptr(l.Wq));
+        I8R_TRY(check_ptr(l.sW));
+        if (l.W16) I8R_TRY(check_ptr(l.W16));
+        I8R_TRY(check_ptr(l.Y));
+#if !I8R_PREFILL_PAIR
+        if (!l.W16 && l.T > decode::MAX_T) return I8R_EARCH;
+#endif
+        if (!workspace || workspace_bytes < ws_layout(l.T, l.K, l.N, l.W16 == nullptr).total) return I8R_EWORKSPACE;
+    }
+    if (n > 0 && reinterpret_cast<uintptr_t>(workspace) % kAlign) return I8R_EALIGN;
+    for (int i = 0; i < n; ++i) {
+        const i8r_layer &l = layers[i];
+        I8R_TRY(mixed_linear_impl(l.X, l.T, l.K, l.Wq, l.sW, l.W16, l.N, l.alpha, l.Y, workspace, workspace_bytes,
+                                  stream));
+    }
+    return I8R_OK;
+}
+
 size_t int8_mixed_linear_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
 
 i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K, const int8_t *Wq, const float *sW,

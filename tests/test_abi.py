@@ -106,6 +106,45 @@ def test_wq_variant_host_checks_and_capacity(so):
         assert extra == cap(K) * N * 2
 
 
+def test_chain_host_checks_and_workspace(so):
+    from int8_quantized_row_b200 import I8rLayer
+    f = so.int8_mixed_linear_chain
+    size = so.int8_mixed_linear_chain_workspace_size
+
+    def layer(T, K, N, w16=True, alpha=6.0, x=4096):
+        return I8rLayer(ctypes.c_void_p(x), T, K, _p(), _p(), _p() if w16 else _null(), N, alpha, _p())
+
+    def arr(*layers):
+        a = (I8rLayer * len(layers))(*layers)
+        return ctypes.cast(a, ctypes.c_void_p), a
+
+    # the workspace is the largest layer's need, each layer sized for its variant
+    shapes = [(16, 12288, 36864, True), (16, 12288, 12288, True), (16, 12288, 49152, False), (300, 1024, 512, True)]
+    ptr, keep = arr(*(layer(*s) for s in shapes))
+    want = max(so.int8_mixed_linear_workspace_size(T, K, N) if w else so.int8_mixed_linear_wq_workspace_size(T, K, N)
+               for T, K, N, w in shapes)
+    assert size(len(shapes), ptr) == want
+    assert size(0, _null()) == 0
+    # n = 0 is a no-op; bad counts and pointers are rejected
+    assert f(0, _null(), _null(), 0, _null()) == 0
+    assert f(-1, ptr, _p(), want, _null()) == 1
+    assert f(2, _null(), _p(), want, _null()) == 1
+    # a bad layer anywhere returns its error before anything is enqueued
+    ok = layer(16, 1024, 1024)
+    for bad, code in ((layer(16, 1000, 1024), 2), (layer(16, 1024, 1024, alpha=float("nan")), 1),
+                      (layer(16, 1024, 1024, x=0), 1), (layer(16, 1024, 1024, x=4097), 2),
+                      (layer(16, 133152, 1024), 3)):
+        ptr2, keep2 = arr(ok, bad)
+        ws = size(1, arr(ok)[0])
+        assert f(2, ptr2, _p(), 1 << 30, _null()) == code
+    # workspace too small for the largest layer, or misaligned
+    ptr3, keep3 = arr(layer(16, 1024, 1024), layer(16, 1024, 4096))
+    need = size(2, ptr3)
+    assert need == so.int8_mixed_linear_workspace_size(16, 1024, 4096)
+    assert f(2, ptr3, _p(), need - 1, _null()) == 4
+    assert f(2, ptr3, _p(4096 + 16), need, _null()) == 2
+
+
 def test_host_rejects_bad_weight_conversion(so):
     f = so.int8_quantize_weight_colwise
     assert f(_p(), 1024, 1000, _p(), _p(), _null()) == 2

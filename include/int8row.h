@@ -232,9 +232,15 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha,
  *   sX    [T] fp32              row absmax over the non-outlier columns
  *   Xq    [T,K] int8            row codes, 0 in outlier columns
  *   Xo    [T,K] fp16 (nullable) Xo[t,j] = X[t, idx[j]] for j < |O|, 0 for
- *                               |O| <= j < 64*ceil(|O|/64); later columns untouched
+ *                               |O| <= j < min(64*ceil(|O|/64), K); later columns untouched
  *   workspace  at least int8_quantize_activation_workspace_size(T, K) bytes
- *              (currently 0: it may be NULL)
+ *              (256: a counter for the one-kernel path), 16-byte aligned
+ *
+ * int8_debug_set_activation_path: 1 (the default) runs the activation side
+ *   as one cooperative kernel whenever this batch of X (at least 8 rows)
+ *   fits in the SMs' shared memory, 0 always as the outlier scan followed by
+ *   the row quantiser.  The two give the same bits; the switch (process-wide) exists
+ *   so that tests can compare them.
  *
  * int8_gemm_i8_s32: acc [T,N] int32 = Xq [T,K] int8 x Wq [K,N] int8, exact,
  *   by the same tensor-core kernels int8_mixed_linear uses (decode-shaped for
@@ -248,6 +254,8 @@ i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha,
                                     float *sX, int8_t *Xq, void *Xo,
                                     void *workspace, size_t workspace_bytes,
                                     cudaStream_t stream);
+
+void int8_debug_set_activation_path(int fused);
 
 size_t int8_gemm_i8_s32_workspace_size(int T, int K, int N);
 

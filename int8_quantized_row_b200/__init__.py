@@ -61,6 +61,8 @@ def lib():
     so.int8_mixed_linear_chain_workspace_size.argtypes = [_I, _P]
     so.int8_mixed_linear_chain_workspace_size.restype = _Z
     so.int8_mixed_linear_chain.argtypes = [_I, _P, _P, _Z, _P]
+    so.int8_debug_set_activation_path.argtypes = [_I]
+    so.int8_debug_set_activation_path.restype = None
     so.int8_outlier_stats_workspace_size.argtypes = [_I]
     so.int8_outlier_stats_workspace_size.restype = _Z
     so.int8_outlier_stats.argtypes = [_P, _I, _I, _F, _P, _P, _P, _P, _P, _Z, _P]
@@ -230,6 +232,11 @@ def int8_outlier_stats(X, alpha=6.0, with_hits=True, stream=None):
         _dev(idx, torch.int32, "idx"), _dev(hits, torch.int32, "hits") if hits is not None else None,
         _dev(frac, torch.float32, "frac"), ctypes.c_void_p(ws.data_ptr()), ws.numel(), _stream(stream)))
     return count, idx, hits, frac
+
+
+def int8_debug_set_activation_path(fused):
+    """1: one cooperative activation kernel when X fits in shared memory (default); 0: scan + quantiser."""
+    lib().int8_debug_set_activation_path(1 if fused else 0)
 
 
 def int8_quantize_activation(X, alpha=6.0, with_xo=True, stream=None):

@@ -32,6 +32,7 @@
 #include "int8row.h"
 #include "device_common.cuh"
 #include "quant_kernels.cuh"
+#include "activation_fused.cuh"
 #include "gemm_prefill.cuh"
 #include "gemm_prefill_pair.cuh"
 #include "gemm_decode.cuh"
@@ -60,7 +61,11 @@ struct DeviceInfo {
     bool sm100 = false;
     int sms = 0;
     int pair_clusters = 0;     // CTA pairs of the prefill GEMM that fit the GPU at once
+    bool fused_ok = false;     // the one-kernel activation path can be launched (cooperative)
 };
+// 1: the activation side runs as one cooperative kernel when X fits in shared
+// memory; 0: always the scan + quantiser pair (set by int8_debug_set_activation_path)
+std::atomic<int> g_activation_fused{1};
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -119,6 +124,12 @@ i8r_status device_setup(const DeviceInfo **out) {
             if (d.pair_clusters < 1) return I8R_EARCH;
             I8R_CUDA(cudaFuncSetAttribute(decode::gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(decode::SMEM_BUDGET + 4096)));
+            I8R_CUDA(cudaFuncSetAttribute(activation_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(kFusedSmemMax)));
+            int per_sm = 0;
+            I8R_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, activation_fused_kernel, kFusedThreads,
+                                                                   kFusedSmemMax));
+            d.fused_ok = per_sm >= 1;
         }
         if (!g_encode) {
             void *fn = nullptr;
@@ -197,7 +208,7 @@ i8r_status check_ptr(const void *p) {
 
 // Workspace of int8_mixed_linear.
 struct Workspace {
-    size_t count, mask, idx, sX, Xq, Xo, W16o, Yo, acc32, counters, total;
+    size_t count, ctr, mask, idx, sX, Xq, Xo, W16o, Yo, acc32, counters, total;
 };
 
 // Rows of the compacted outlier weight rows kept for the prefill GEMM: 256
@@ -214,6 +225,7 @@ Workspace ws_layout(int T, int K, int N, bool wq_only = false) {
     Workspace w{};
     size_t off = 0;
     w.count = off; off = align_up(off + sizeof(int32_t));
+    w.ctr = off;   off = align_up(off + sizeof(uint32_t));        // the fused activation kernel's grid barrier
     w.mask = off;  off = align_up(off + static_cast<size_t>((K + 31) / 32) * 4);
     w.idx = off;   off = align_up(off + static_cast<size_t>(K) * 4);
     w.sX = off;    off = align_up(off + static_cast<size_t>(T) * 4);
@@ -234,6 +246,24 @@ Workspace ws_layout(int T, int K, int N, bool wq_only = false) {
     }
     w.total = off;
     return w;
+}
+
+// Magnitude bits of the smallest fp16 value >= alpha (alpha >= 0, not NaN);
+// 0x7C00 (infinity) when no finite fp16 reaches it.  fp16 magnitudes order
+// like their bit patterns, so |x| >= alpha <=> (bits(x) & 0x7FFF) >= this,
+// for every finite x.
+uint32_t half_threshold_bits(float alpha) {
+    auto value = [](uint32_t b) -> double {                 // exact value of a finite fp16 magnitude
+        const uint32_t e = (b >> 10) & 0x1Fu, m = b & 0x3FFu;
+        return e == 0 ? std::ldexp(static_cast<double>(m), -24) : std::ldexp(static_cast<double>(m | 0x400u), static_cast<int>(e) - 25);
+    };
+    if (!(static_cast<double>(alpha) <= value(0x7BFFu))) return 0x7C00u;
+    uint32_t lo = 0, hi = 0x7BFFu;                          // value(hi) >= alpha
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi) / 2;
+        if (value(mid) >= static_cast<double>(alpha)) hi = mid; else lo = mid + 1;
+    }
+    return lo;
 }
 
 // Launch a kernel as a programmatic dependent of the previous kernel on
@@ -289,10 +319,44 @@ dim3 scan_grid(int T, int K, int sms, int *rows_per_block) {
 i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int K, float alpha, uint32_t *mask,
                              int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
                              size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
-                             __half *W16o = nullptr, const int8_t *Wq = nullptr, const float *sW = nullptr) {
+                             __half *W16o = nullptr, const int8_t *Wq = nullptr, const float *sW = nullptr,
+                             unsigned *grid_ctr = nullptr) {
     const int nwords = (K + 31) / 32;
-    clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords);
+    // One cooperative kernel when this batch of X fits in the blocks' shared
+    // memory: one block per SM (blocks past the last row still clear their
+    // share of `zero` and take part in the barrier).  Below 8 rows the
+    // grid-wide barrier costs more than the two small kernels it replaces.
+    const int fG = std::max(1, dev->sms);
+    const int fR = (T + fG - 1) / fG;
+    const bool fused = grid_ctr && T >= kFusedMinRows && dev->fused_ok &&
+                       g_activation_fused.load(std::memory_order_relaxed) && fused_smem_bytes(fR, K) <= kFusedSmemMax;
+    clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords, fused ? grid_ctr : nullptr);
     I8R_LAUNCHED();
+    if (fused) {
+        const int o_rows = W16o ? compact_rows(K, W16 == nullptr) : 0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(fG));
+        cfg.blockDim = dim3(kFusedThreads);
+        cfg.dynamicSmemBytes = fused_smem_bytes(fR, K);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        attr[1].id = cudaLaunchAttributeCooperative;       // every block resident: the grid barrier completes
+        attr[1].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        const uint32_t thr = half_threshold_bits(alpha);
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, activation_fused_kernel, X, T, K, thr | (thr << 16), fR, mask, grid_ctr, sX,
+                                                 Xq, Xo, idx, count, W16, Wq, sW, N, W16o, o_rows,
+                                                 static_cast<int4 *>(zero), zero_bytes / 16);
+        if (e != cudaSuccess) {
+            tl_last_cuda_error = static_cast<int>(e);
+            return I8R_ECUDA;
+        }
+        I8R_LAUNCHED();
+        return I8R_OK;
+    }
     if (T == 0) {
         // no rows: an empty outlier set still has to be published
         outlier_index_kernel<<<1, kIndexThreads, 0, s>>>(mask, 1, K, mask, idx, count, nullptr);
@@ -655,7 +719,7 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     __half *W16o = (small_t && wq_only) ? reinterpret_cast<__half *>(ws + w.W16o) : nullptr;
 #endif
     I8R_TRY(launch_activation(dev, x, T, K, alpha, mask, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
-                              zero_bytes, stream, w16, N, W16o, Wq, sW));
+                              zero_bytes, stream, w16, N, W16o, Wq, sW, reinterpret_cast<unsigned *>(ws + w.ctr)));
     if (!small_t)
         return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream, W16o);
 
@@ -734,6 +798,8 @@ i8r_status int8_mixed_linear_chain(int n, const i8r_layer *layers, void *workspa
 
 size_t int8_mixed_linear_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
 
+void int8_debug_set_activation_path(int fused) { g_activation_fused.store(fused ? 1 : 0); }
+
 i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K, const int8_t *Wq, const float *sW,
                                      const void *W16, int N, float alpha, void *Y, cudaStream_t stream) {
     I8R_TRY(check_shape(T, K, N, true));
@@ -782,7 +848,7 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha, int32_t 
 size_t int8_quantize_activation_workspace_size(int T, int K) {
     (void)T;
     (void)K;
-    return 0;                      // the activation side needs no scratch of its own
+    return kAlign;                 // the one-kernel path's grid-barrier counter
 }
 
 i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha, uint32_t *mask, int32_t *idx,
@@ -799,12 +865,13 @@ i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha, ui
     I8R_TRY(check_ptr(mask));
     I8R_TRY(check_ptr(idx));
     if (!count) return I8R_EINVAL;
-    (void)workspace;
-    (void)workspace_bytes;
+    if (!workspace || workspace_bytes < kAlign) return I8R_EWORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % 16) return I8R_EALIGN;
     const DeviceInfo *dev = nullptr;
     I8R_TRY(device_setup(&dev));
     return launch_activation(dev, static_cast<const __half *>(X), T, K, alpha, mask, idx, count, sX, Xq,
-                             static_cast<__half *>(Xo), nullptr, 0, stream);
+                             static_cast<__half *>(Xo), nullptr, 0, stream, nullptr, 0, nullptr, nullptr, nullptr,
+                             static_cast<unsigned *>(workspace));
 }
 
 size_t int8_gemm_i8_s32_workspace_size(int T, int K, int N) {

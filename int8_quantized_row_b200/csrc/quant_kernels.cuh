@@ -181,9 +181,11 @@ __global__ void __launch_bounds__(kStripThreads) outlier_mask_kernel(const __hal
 constexpr int kScanThreads = 256;
 constexpr int kBandCols = kScanThreads * 8;
 
-__global__ void __launch_bounds__(256) clear_mask_kernel(uint32_t *__restrict__ mask, int nwords) {
+__global__ void __launch_bounds__(256) clear_mask_kernel(uint32_t *__restrict__ mask, int nwords,
+                                                         unsigned *__restrict__ grid_ctr) {
     griddep_launch_dependents();        // the scan may start loading rows
     for (int w = threadIdx.x; w < nwords; w += blockDim.x) mask[w] = 0u;
+    if (grid_ctr && threadIdx.x == 0) *grid_ctr = 0u;     // the fused kernel's grid barrier
 }
 
 __global__ void __launch_bounds__(kScanThreads) outlier_scan_kernel(const __half *__restrict__ X, int T, int K,
@@ -316,7 +318,8 @@ inline size_t quantize_smem_bytes(int K) { return static_cast<size_t>((K + 31) /
 // The W16 rows of the first o_rows outlier columns, compacted for the
 // prefill GEMM (its outlier stages then load two 64 x 64 boxes each instead
 // of gathering rows):  W16o[j,:] = W16[O_j,:] for j < |O|, zero rows up to the
-// next multiple of 64 (at most o_rows).  Without W16 (the Wq-only variant) the
+// next multiple of 16 (at most o_rows; the MMAs read no row past that, so the
+// rest of a 64-row box may hold anything).  Without W16 (the Wq-only variant) the
 // rows are dequantised instead, W16o[j,n] = fp16_rn(Wq[O_j,n] * fl32(sW[n]/127)),
 // and more than o_rows outlier columns is reported (I8R_DEV_OUTLIER_CAP).
 // Block e of the G compaction blocks copies rows e, e+G, ... with eight
@@ -339,7 +342,7 @@ __device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *smask
         }
     }
     __syncthreads();
-    const int rows = min((total + 63) / 64 * 64, o_rows);
+    const int rows = min((total + 15) / 16 * 16, o_rows);
     const int vec = N / 8;
     constexpr int kBatch = 8;
     for (int r = e; r < rows; r += G) {

@@ -116,6 +116,46 @@ def test_quantiser_ties_round_half_away(orc):
     assert device_status_clean()
 
 
+FUSED_CASES = ACT_CASES + [
+    (2048, 5120, [3, 900, 5000], 6.0),        # the OPT-13B prefill batch: 14 rows per block
+    (8, 49152, [7, 40000], 6.0),              # one row of 96 KB in a block
+    (128, 12288, list(range(0, 12288, 97)), 6.0),
+    (4096, 12288, [5], 6.0),                  # too big for shared memory: both calls take the two-kernel path
+    # thresholds fp16 does not hold: the one-kernel path compares fp16 bit patterns
+    # with the smallest fp16 >= alpha, the two-kernel path compares in fp32
+    (64, 1024, [], 1.0 / 3.0),
+    (64, 1024, [], 3.1),
+    (32, 2048, [], 2.0 ** -20),
+]
+
+
+@pytest.mark.parametrize("T,K,cols,alpha", FUSED_CASES)
+def test_fused_activation_equals_two_kernel_path(T, K, cols, alpha):
+    """The one-kernel activation path (X held in shared memory, grid barrier)
+    gives the same bits as the outlier scan followed by the row quantiser."""
+    rng = np.random.default_rng(T * 7 + K)
+    X = outlier_x(rng, T, K, cols)
+    if T > 2:
+        X[1] = 0
+    Xd = to_dev(X)
+    outs = []
+    try:
+        for fused in (1, 0):
+            i8.int8_debug_set_activation_path(fused)
+            outs.append({k: to_host(v).copy() for k, v in i8.int8_quantize_activation(Xd, alpha).items()})
+    finally:
+        i8.int8_debug_set_activation_path(1)
+    a, b = outs
+    cnt = int(a["count"][0])
+    assert cnt == int(b["count"][0])
+    for k in ("mask", "sX", "Xq"):
+        assert np.array_equal(a[k], b[k]), k
+    assert np.array_equal(a["idx"][:cnt], b["idx"][:cnt])
+    pad = min((cnt + 63) // 64 * 64, K)
+    assert np.array_equal(a["Xo"][:T, :pad].view(np.uint16), b["Xo"][:T, :pad].view(np.uint16))
+    assert device_status_clean()
+
+
 def test_activation_t0_is_noop():
     X = torch.zeros((0, 64), dtype=torch.float16, device="cuda")
     out = i8.int8_quantize_activation(X, 6.0)

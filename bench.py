@@ -12,6 +12,8 @@ rotated so that every step reads operands that are not in L2.
 Under torchrun (N > 1) every rank runs its own independent batch (replicas;
 the layer has no exchange step), the time is the max over ranks and the
 value is the work of all ranks divided by that time ("scaling": "weak").
+With --parallel column the ranks instead split one layer by weight columns
+and all-gather Y over NCCL ("scaling": "strong": the job's work is fixed).
 
 Prints one JSON line (rank 0).  --impl reference times the CPU oracle instead
 (the reference arm for this method: it runs the plain CPU definition on a
@@ -58,6 +60,10 @@ def parse():
                          "int8_mixed_linear_chain call replayed from a CUDA graph (one JSON line; "
                          "not the one-line contract run)")
     ap.add_argument("--chain-t", type=int, default=16, help="tokens per projection for --chain")
+    ap.add_argument("--parallel", default="replica", choices=["replica", "column"],
+                    help="N>1 ranks: replica = an independent batch per GPU (weak scaling, the default); "
+                         "column = one layer split by weight columns over the GPUs, Y all-gathered over NCCL "
+                         "(strong scaling)")
     ap.add_argument("--variant", default="w16", choices=["w16", "wq"],
                     help="w16: int8_mixed_linear (fp16 weight resident for the outlier rows); "
                          "wq: int8_mixed_linear_wq (only Wq and sW resident)")
@@ -282,15 +288,25 @@ def run_ours(args, cfg, world, rank, local, pg):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     T, K, N, alpha = cfg["T"], cfg["K"], cfg["N"], cfg["alpha"]
+    column = args.parallel == "column" and world > 1
+    if column:
+        from int8_quantized_row_b200 import column_parallel as cp
+        ca, cb = cp.column_bounds(N, world, rank)
+    else:
+        ca, cb = 0, N
+    NL = cb - ca                        # this rank's output columns
 
-    # inputs: ROTATE independent sets, each seeded per (set, rank)
+    # inputs: ROTATE independent sets, each seeded per (set, rank); with the
+    # column split every rank draws the same layer and keeps its column block
     sets = []
     host_x = []
     X0 = W0 = None
     nrot = max(1, args.rotate)
     for r in range(nrot):
-        c = dict(cfg, seed=cfg["seed"] + 1000 * rank + r)
+        c = dict(cfg, seed=cfg["seed"] + (0 if column else 1000 * rank) + r)
         X, W = wl.generate(c)
+        if column:
+            W = np.ascontiguousarray(W[:, ca:cb])
         if r == 0:
             X0, W0 = X, W
         Xd = torch.from_numpy(X).to(dev)
@@ -301,25 +317,30 @@ def run_ours(args, cfg, world, rank, local, pg):
             Wd = None                   # only Wq and sW stay resident
         sets.append((Xd, Wq, sW, Wd))
         host_x.append(torch.from_numpy(X).pin_memory())
-    Y = torch.empty((T, N), dtype=torch.float16, device=dev)
+    Y = torch.empty((T, NL), dtype=torch.float16, device=dev)
+    Y_full = Y
     Y_host = torch.empty((T, N), dtype=torch.float16).pin_memory()
     if args.variant == "wq":
-        ws = torch.empty(max(1, i8.int8_mixed_linear_wq_workspace_size(T, K, N)), dtype=torch.uint8, device=dev)
+        ws = torch.empty(max(1, i8.int8_mixed_linear_wq_workspace_size(T, K, NL)), dtype=torch.uint8, device=dev)
     else:
-        ws = i8.workspace(T, K, N, dev)
+        ws = i8.workspace(T, K, NL, dev)
     torch.cuda.synchronize()
 
     stats = i8.int8_outlier_stats(sets[0][0], alpha)
     n_out = int(stats[0].item())
     frac8 = float(stats[3].item())
-    ops, wbytes = work(cfg, n_out, args.variant)
+    ops, wbytes = work(dict(cfg, N=NL), n_out, args.variant)       # this rank's share
+    ops_job = 2.0 * T * K * N if column else world * ops               # the whole job's
 
     def step(i):
+        nonlocal Y_full
         Xd, Wq, sW, Wd = sets[i % nrot]
         if Wd is None:
             i8.int8_mixed_linear_wq(Xd, Wq, sW, alpha, Y=Y, workspace_buf=ws)
         else:
             i8.int8_mixed_linear(Xd, Wq, sW, Wd, alpha, Y=Y, workspace_buf=ws)
+        if column:
+            Y_full = cp.gather_columns(Y, N, world, rank)
 
     for i in range(args.warmup):
         step(i)
@@ -361,7 +382,7 @@ def run_ours(args, cfg, world, rank, local, pg):
     status = i8.int8_read_and_clear_device_status()
 
     ms_step = ms_max / args.steps
-    value = world * ops / (ms_step * 1e-3) / 1e12
+    value = ops_job / (ms_step * 1e-3) / 1e12
 
     # end to end through the public API with host buffers: H2D of X, the call,
     # D2H of Y, every step, all inside the timed region
@@ -369,7 +390,7 @@ def run_ours(args, cfg, world, rank, local, pg):
         Xd = sets[i % nrot][0]
         Xd.copy_(host_x[i % nrot], non_blocking=True)
         step(i)
-        Y_host.copy_(Y, non_blocking=True)
+        Y_host[:, :Y_full.shape[1]].copy_(Y_full, non_blocking=True)
     torch.cuda.synchronize()
     e_steps = max(1, min(args.steps, 200))
     barrier(pg, local)
@@ -379,12 +400,12 @@ def run_ours(args, cfg, world, rank, local, pg):
         Xd = sets[i % nrot][0]
         Xd.copy_(host_x[i % nrot], non_blocking=True)
         step(i)
-        Y_host.copy_(Y, non_blocking=True)
+        Y_host[:, :Y_full.shape[1]].copy_(Y_full, non_blocking=True)
     end.record(stream)
     torch.cuda.synchronize()
     barrier(pg, local)
     e_ms = max_over_ranks(pg, start.elapsed_time(end), dev) / e_steps
-    e_value = world * ops / (e_ms * 1e-3) / 1e12
+    e_value = ops_job / (e_ms * 1e-3) / 1e12
 
     pk = peaks()
     decode = T <= i8.DECODE_MAX_T
@@ -410,16 +431,19 @@ def run_ours(args, cfg, world, rank, local, pg):
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "strong" if column else "weak",
         "vs_baseline": None, "dtype": "i8", "data": "synthetic, seeded (N(0,1) activations with planted outlier "
         "columns, N(0,sigma) weights); no datasets or trained weights",
         "config": {"workload": args.workload, "T": T, "K": K, "N": N, "alpha": alpha, "outlier_cols": n_out,
-                   "frac_8bit": frac8, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "frac_8bit": frac8,
+                   "parallelism": (f"column-parallel x{world}: weight columns split, Y all-gathered over NCCL"
+                                   if column else f"replicas x{world}" if world > 1 else "single GPU"),
                    "l2": f"{nrot} rotating input sets" + (" (each step's operands not in L2)" if nrot >= 3 else
                                                           " (operands may be partly L2-resident)"),
                    "variant": ("wq-only: outlier rows dequantised from Wq, no fp16 weight resident"
                                if args.variant == "wq" else "w16: fp16 weight rows for the outliers"),
-                   "resident_weight_bytes": K * N + 4 * N + (0 if args.variant == "wq" else 2 * K * N)},
+                   "resident_weight_bytes": K * NL + 4 * NL + (0 if args.variant == "wq" else 2 * K * NL)},
         "weight_gbs": world * wbytes / (ms_step * 1e-3) / 1e9,
         "roofline": roof,
         "e2e": {"value": e_value, "unit": "TOPS", "h2d_bytes_per_step": 2 * T * K,

@@ -85,7 +85,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // The same wait taken by lane 0 of a warp on behalf of the whole warp; the
-// verdict is broadcast so the warp stays converged.
+// result is broadcast so the warp stays converged.
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int code) {
     int ok = 1;
     if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, code) ? 1 : 0;

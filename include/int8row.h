@@ -237,10 +237,10 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha,
  *              (256: a counter for the one-kernel path), 16-byte aligned
  *
  * int8_debug_set_activation_path: 1 (the default) runs the activation side
- *   as one cooperative kernel whenever this batch of X (at least 8 rows)
- *   fits in the SMs' shared memory, 0 always as the outlier scan followed by
- *   the row quantiser.  The two give the same bits; the switch (process-wide) exists
- *   so that tests can compare them.
+ *   as one cooperative kernel for batches of 8 to 128 rows that fit in the
+ *   SMs' shared memory, 2 as that kernel whenever the batch fits, 0 always
+ *   as the outlier scan followed by the row quantiser.  All give the same
+ *   bits; the switch (process-wide) exists so that tests can compare them.
  *
  * int8_gemm_i8_s32: acc [T,N] int32 = Xq [T,K] int8 x Wq [K,N] int8, exact,
  *   by the same tensor-core kernels int8_mixed_linear uses (decode-shaped for
@@ -255,7 +255,7 @@ i8r_status int8_quantize_activation(const void *X, int T, int K, float alpha,
                                     void *workspace, size_t workspace_bytes,
                                     cudaStream_t stream);
 
-void int8_debug_set_activation_path(int fused);
+void int8_debug_set_activation_path(int mode);
 
 size_t int8_gemm_i8_s32_workspace_size(int T, int K, int N);
 

@@ -234,9 +234,10 @@ def int8_outlier_stats(X, alpha=6.0, with_hits=True, stream=None):
     return count, idx, hits, frac
 
 
-def int8_debug_set_activation_path(fused):
-    """1: one cooperative activation kernel when X fits in shared memory (default); 0: scan + quantiser."""
-    lib().int8_debug_set_activation_path(1 if fused else 0)
+def int8_debug_set_activation_path(mode):
+    """1 (default): the one cooperative activation kernel for 8 <= T <= 128 when X fits in
+    shared memory; 2: that kernel whenever X fits; 0: scan + quantiser."""
+    lib().int8_debug_set_activation_path(int(mode))
 
 
 def int8_quantize_activation(X, alpha=6.0, with_xo=True, stream=None):

@@ -175,9 +175,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) activation_fused_kernel(
         }
         if (tid == 0) *count_out = total;
     }
+    // the compaction rows go to the blocks from the last one down: they hold
+    // the fewest rows of X (or none), so the copies stay off the longest path
     if (W16o)
         gather_outlier_weight_rows<kFusedThreads>(smask, spre, w0, w1, total, W16, Wq, sW, N, W16o, o_rows,
-                                                  static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x));
+                                                  static_cast<int>(gridDim.x - 1 - blockIdx.x),
+                                                  static_cast<int>(gridDim.x));
 
     // rows: gs warps per row (one when the block holds many rows), ng rows at a time
     int gs = kWarps / max(1, min(nrows, kWarps));

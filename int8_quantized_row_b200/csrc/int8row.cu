@@ -63,8 +63,9 @@ struct DeviceInfo {
     int pair_clusters = 0;     // CTA pairs of the prefill GEMM that fit the GPU at once
     bool fused_ok = false;     // the one-kernel activation path can be launched (cooperative)
 };
-// 1: the activation side runs as one cooperative kernel when X fits in shared
-// memory; 0: always the scan + quantiser pair (set by int8_debug_set_activation_path)
+// Which activation path runs (int8_debug_set_activation_path): 1 (default) the
+// one cooperative kernel for 8 <= T <= 128 when X fits in shared memory, 2 that
+// kernel whenever X fits, 0 always the scan + quantiser pair.
 std::atomic<int> g_activation_fused{1};
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -324,12 +325,15 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     const int nwords = (K + 31) / 32;
     // One cooperative kernel when this batch of X fits in the blocks' shared
     // memory: one block per SM (blocks past the last row still clear their
-    // share of `zero` and take part in the barrier).  Below 8 rows the
-    // grid-wide barrier costs more than the two small kernels it replaces.
+    // share of `zero` and take part in the barrier).  By default only for
+    // decode-sized batches of at least 8 rows: below that the grid-wide barrier
+    // costs more than the two small kernels it replaces, and at prefill sizes
+    // (OPT-13B fc1, 2048 rows) the two paths measured level.
     const int fG = std::max(1, dev->sms);
     const int fR = (T + fG - 1) / fG;
-    const bool fused = grid_ctr && T >= kFusedMinRows && dev->fused_ok &&
-                       g_activation_fused.load(std::memory_order_relaxed) && fused_smem_bytes(fR, K) <= kFusedSmemMax;
+    const int mode = g_activation_fused.load(std::memory_order_relaxed);
+    const bool size_ok = mode == 2 ? T >= 1 : (mode == 1 && T >= kFusedMinRows && T <= decode::MAX_T);
+    const bool fused = grid_ctr && size_ok && dev->fused_ok && fused_smem_bytes(fR, K) <= kFusedSmemMax;
     clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords, fused ? grid_ctr : nullptr);
     I8R_LAUNCHED();
     if (fused) {
@@ -798,7 +802,7 @@ i8r_status int8_mixed_linear_chain(int n, const i8r_layer *layers, void *workspa
 
 size_t int8_mixed_linear_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
 
-void int8_debug_set_activation_path(int fused) { g_activation_fused.store(fused ? 1 : 0); }
+void int8_debug_set_activation_path(int mode) { g_activation_fused.store(mode < 0 ? 0 : (mode > 2 ? 2 : mode)); }
 
 i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K, const int8_t *Wq, const float *sW,
                                      const void *W16, int N, float alpha, void *Y, cudaStream_t stream) {

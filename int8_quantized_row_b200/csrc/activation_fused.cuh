@@ -1,6 +1,8 @@
 // The activation side of the layer (a1-a3) in one cooperative kernel, for
 // batches whose X fits in the GPU's shared memory (148 SMs x ~200 KB: the
-// 2048 x 5120 fp16 OPT-13B prefill batch and every decode batch do):
+// 2048 x 5120 fp16 OPT-13B prefill batch and every decode batch do; by
+// default the library uses it for batches of 8 to 128 rows, where it is the
+// faster of the two paths):
 //
 //   1. each block copies its R rows of X into shared memory (one bulk copy
 //      per row, issued before waiting for the kernel before it) and ORs the

@@ -4,10 +4,15 @@
 
 A step is one whole int8_mixed_linear call (outlier detection, row
 quantisation, outlier gather, int8 + fp16 tensor-core GEMM, dequantise and
-merge) on one batch that is already resident in HBM.  The default workload is
-the OPT-13B-shaped FFN fc1 at prefill (T=2048, K=5120, N=20480, 6 outlier
-columns in 25% of rows, alpha = 6).  Three input sets (X, Wq, sW, W16) are
-rotated so that every step reads operands that are not in L2.
+merge) on one batch that is already resident in HBM.  The headline workload
+is the largest single-GPU configuration, the 175B-shaped QKV projection at
+prefill (T=4096, K=12288, N=36864, 0.1% outlier columns in every row,
+alpha = 6), which is bound by the int8 tensor cores.  The same JSON line
+carries, under "decode", the 175B-shaped fc1 at decode size (T=16, K=12288,
+N=49152, 7 outlier columns), which is bound by HBM: the same steps and
+warm-up, its own value, roofline, clocks and CPU baseline.  Three input sets
+(X, Wq, sW, W16) are rotated so that every step reads operands that are not
+in L2 (each set's weights alone are several times the 126 MB L2).
 
 Under torchrun (N > 1) every rank runs its own independent batch (replicas;
 the layer has no exchange step), the time is the max over ranks and the
@@ -27,6 +32,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 import numpy as np
@@ -36,18 +42,29 @@ sys.path.insert(0, ROOT)
 
 from int8_quantized_row_b200 import workloads as wl  # noqa: E402
 
-DEFAULT_WORKLOAD = "opt13b_fc1_prefill_2048x5120x20480"
+DEFAULT_WORKLOAD = "b175_qkv_prefill_4096x12288x36864"
+DECODE_WORKLOAD = "b175_fc1_decode_t16_12288x49152"
 METRIC = "int8-mixed linear effective TOPS & weight GB/s; % of B200 int8/HBM roofline"
 ROTATE = 3
 PROFILES = os.path.join(ROOT, "profiles")
+# A timed region shorter than this is a burst: the GEMM's roofline takes the
+# burst GEMM peak (the sustained one was measured over seconds under the power cap).
+BURST_WINDOW_S = 1.0
+# Sources of each GEMM kernel, for keying its committed DRAM-traffic capture.
+KERNEL_SOURCES = {
+    "gemm_prefill_pair_kernel": ("gemm_prefill_pair.cuh", "device_common.cuh"),
+    "gemm_decode_kernel": ("gemm_decode.cuh", "device_common.cuh"),
+}
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--decode-workload", default=DECODE_WORKLOAD,
+                    help="the HBM-bound point reported under \"decode\" in the same line ('none' to skip)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--rotate", type=int, default=ROTATE,
@@ -55,6 +72,8 @@ def parse():
     ap.add_argument("--sweep", action="store_true",
                     help="time every point of the 175B decoder-layer sweep in one process (one JSON line each; "
                          "not the one-line contract run)")
+    ap.add_argument("--sweep-layers", default="qkv,out,fc1,fc2", help="layers of --sweep")
+    ap.add_argument("--sweep-t", default="1,16,128,2048", help="batch sizes of --sweep")
     ap.add_argument("--chain", action="store_true",
                     help="time the 175B decoder layer's four projections (qkv, out, fc1, fc2) as one "
                          "int8_mixed_linear_chain call replayed from a CUDA graph (one JSON line; "
@@ -67,7 +86,7 @@ def parse():
     ap.add_argument("--variant", default="w16", choices=["w16", "wq"],
                     help="w16: int8_mixed_linear (fp16 weight resident for the outlier rows); "
                          "wq: int8_mixed_linear_wq (only Wq and sW resident)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def all_configs():
@@ -95,63 +114,142 @@ def peaks():
     return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, src="fallback")
 
 
-def kernel_source_sha():
+def tensor_peak(pk, region_s):
+    """Dense int8 peak for a GEMM timed over a region of `region_s` seconds:
+    the bf16 GEMM figure x 2 (B200's nominal dense int8 : bf16 ratio, 4.5 : 2.25
+    POPS), the burst figure for a region under BURST_WINDOW_S, else the
+    sustained one.  Returns (peak TOP/s, description)."""
+    if region_s < BURST_WINDOW_S or not pk["bf16_tflops_sustained"]:
+        return 2.0 * pk["bf16_tflops"], (f"{pk['src']} bf16 burst x 2 (dense int8 : bf16 nominal 4.5 : 2.25); "
+                                         f"timed region {region_s * 1e3:.1f} ms < {BURST_WINDOW_S:.0f} s")
+    return 2.0 * pk["bf16_tflops_sustained"], (f"{pk['src']} bf16 sustained x 2 (dense int8 : bf16 nominal "
+                                               f"4.5 : 2.25); timed region {region_s:.2f} s")
+
+
+def kernel_source_sha(kernel):
+    """Hash of the sources of one GEMM kernel (its header and the PTX wrappers it uses)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "int8_quantized_row_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in KERNEL_SOURCES[kernel]:
         h.update(f.encode())
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload):
-    """DRAM bytes per launch of the GEMM kernel from a committed ncu capture,
-    only while the kernel sources are unchanged since the capture."""
+def ncu_traffic(workload, kernel):
+    """DRAM bytes per launch of `kernel` on `workload` from a committed ncu
+    capture, only while that kernel's sources are unchanged since the capture."""
     p = os.path.join(PROFILES, "ncu_traffic.json")
     if not os.path.exists(p):
         return None
-    d = json.load(open(p))
-    if d.get("kernel_source_sha") != kernel_source_sha():
+    d = json.load(open(p)).get("captures", {}).get(workload)
+    if not d or d.get("kernel") != kernel or d.get("source_sha") != kernel_source_sha(kernel):
         return None
-    return d.get("workloads", {}).get(workload)
+    return d.get("bytes_per_launch")
 
 
 # ------------------------------------------------------------------ clocks
 
-class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index):
-        self.dev = device_index
-        self.proc = None
-        self.f = None
+
+def summarise_clock_samples(samples, sm_max_mhz, source):
+    """samples: (sm MHz, power W, clock-event reason bits) tuples taken under load."""
+    reasons = set()
+    for _, _, bits in samples:
+        for nm, b in REASON_BITS.items():
+            if bits & b:
+                reasons.add(nm)
+    sm = [s[0] for s in samples]
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": sm_max_mhz,
+            "samples": len(sm), "power_w_max": max((s[1] for s in samples), default=None),
+            "reasons": sorted(reasons), "source": source}
+
+
+class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU, sampled on a
+    background thread through NVML every `period_s` between start() and stop()
+    (a timed region of a few milliseconds still gets samples); nvidia-smi at
+    100 ms when NVML is unavailable."""
+
+    def __init__(self, torch_device, period_s=0.001):
+        self.period = period_s
+        self.handle = None
+        self.nvml = None
+        self.samples = []
+        self.stop_evt = threading.Event()
+        self.thread = None
+        self.smi = None
+        self.index = getattr(torch_device, "index", None) or 0
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device)
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nvml = pynvml
+            self.sm_max = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.handle = None
+
+    def _poll(self):
+        n = self.nvml
+        while not self.stop_evt.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                pw = n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                bits = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((float(sm), pw, int(bits)))
+            except Exception:
+                return
+            time.sleep(self.period)
 
     def start(self):
+        self.samples = []
+        self.stop_evt.clear()
+        if self.handle is not None:
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
         try:
             self.f = tempfile.TemporaryFile(mode="w+")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.dev)], stdout=self.f, stderr=subprocess.DEVNULL)
+            self.smi = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={SMI_FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)],
+                stdout=self.f, stderr=subprocess.DEVNULL)
         except OSError:
-            self.proc = None
+            self.smi = None
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join()
+            self.thread = None
+            return summarise_clock_samples(self.samples, self.sm_max, f"NVML every {self.period * 1e3:g} ms")
+        if self.smi is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": ["no clock source"]}
+        self.smi.terminate()
         try:
-            self.proc.wait(timeout=5)
+            self.smi.wait(timeout=5)
         except subprocess.TimeoutExpired:
-            self.proc.kill()
+            self.smi.kill()
         self.f.seek(0)
         return parse_clock_csv(self.f.read())
 
 
+SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
 def parse_clock_csv(text):
     """Median SM clock, max SM clock and the throttle reasons seen, from
-    `nvidia-smi --query-gpu=<ClockSampler.FIELDS> --format=csv,noheader,nounits` lines."""
+    `nvidia-smi --query-gpu=<SMI_FIELDS> --format=csv,noheader,nounits` lines."""
     sm, smax, reasons = [], None, set()
     names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
     for line in text.splitlines():
@@ -167,7 +265,7 @@ def parse_clock_csv(text):
             if v.lower().startswith("active"):
                 reasons.add(nm)
     return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-            "samples": len(sm), "reasons": sorted(reasons)}
+            "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi every 100 ms"}
 
 
 # ------------------------------------------------------------------ distributed
@@ -216,7 +314,7 @@ def oracle_sample(cfg, X, W, target_s=15.0, orc_state=None, variant="w16"):
     of R rows of X (the whole method, outlier scan included, on those R
     tokens) against the first C columns of the weight (a column slice is the
     same sub-problem: column scales are per column).  Returns
-    (TOPS, R, C, seconds, threads used, state)."""
+    (TOPS, R, C, seconds, threads used, state, run)."""
     import oracle
     if orc_state is None:
         orc = oracle.default()
@@ -249,12 +347,19 @@ def oracle_sample(cfg, X, W, target_s=15.0, orc_state=None, variant="w16"):
     return ops / dt / 1e12, R, C, dt, min(R, threads), orc_state, run
 
 
-def run_reference(args, cfg, world, rank, pg):
-    if rank != 0:
-        return
+def cpu_baseline(cfg, X, W, variant, target_s):
+    tops, R, C, dt, cores, _, _ = oracle_sample(cfg, X, W, target_s=target_s, variant=variant)
+    T, N = cfg["T"], cfg["N"]
+    return {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
+            "sample": f"sub-batch of {R} of {T} rows x {C} of {N} columns ({dt:.1f} s, "
+                      f"whole method incl. outlier scan); weight conversion untimed"}
+
+
+def reference_line(args, name, cfg, world, seconds):
+    """The oracle timed per step on a bounded sample of workload `name`."""
     X, W = wl.generate(cfg)
     T, K, N = cfg["T"], cfg["K"], cfg["N"]
-    per_step = 100.0 / max(1, args.steps + args.warmup)          # whole run ~2 minutes
+    per_step = seconds / max(1, args.steps + args.warmup)
     _, R, C, _, cores, state, run = oracle_sample(cfg, X, W, target_s=min(per_step, 15.0), variant=args.variant)
     times = []
     for i in range(args.warmup + args.steps):
@@ -266,25 +371,66 @@ def run_reference(args, cfg, world, rank, pg):
     value = ops / total / 1e12
     sample = (f"sub-batch of {R} of {T} rows x {C} of {N} columns per step (whole method incl. outlier "
               f"scan on the sub-batch); weight conversion untimed")
-    line = {
+    return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8",
-        "data": "synthetic, seeded", "config": {"workload": args.workload, "T": T, "K": K, "N": N,
+        "data": "synthetic, seeded", "config": {"workload": name, "T": T, "K": K, "N": N,
                                                 "alpha": cfg["alpha"], "variant": args.variant},
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    cfgs = all_configs()
+    decode = args.decode_workload != "none"
+    line = reference_line(args, args.workload, cfgs[args.workload], world, 80.0 if decode else 100.0)
+    if decode:
+        d = reference_line(args, args.decode_workload, cfgs[args.decode_workload], world, 20.0)
+        line["decode"] = {k: d[k] for k in ("metric", "value", "unit", "ms_per_step", "config", "cpu_baseline",
+                                            "e2e")}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ GPU arm
 
-def run_ours(args, cfg, world, rank, local, pg):
+def cublas_int8_tops(T, K, N, dev, iters=10):
+    """cuBLAS int8 GEMM (torch._int_mm: int8 x int8 -> int32, no outlier part,
+    no quantisation) on the same shape, as a burst: a measured int8 reference
+    point, timed outside the benchmark's timed regions."""
+    import torch
+    if T <= 16:
+        return None
+    g = torch.Generator(device=dev).manual_seed(0)
+    a = torch.randint(-127, 128, (T, K), dtype=torch.int8, device=dev, generator=g)
+    b = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=g).t()   # column-major B
+    try:
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(iters):
+            torch._int_mm(a, b)
+        e.record()
+        torch.cuda.synchronize()
+        return 2.0 * T * K * N / (s.elapsed_time(e) / iters * 1e-3) / 1e12
+    except RuntimeError:
+        return None
+    finally:
+        del a, b
+        torch.cuda.empty_cache()
+
+
+def measure(args, name, cfg, world, rank, local, pg, with_cublas):
+    """One workload on this rank: the timed steps, the GEMM-only pass, the
+    end-to-end pass and the roofline.  Returns the fields of its JSON object."""
     import torch
     import int8_quantized_row_b200 as i8
 
-    torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
     T, K, N, alpha = cfg["T"], cfg["K"], cfg["N"], cfg["alpha"]
@@ -298,8 +444,7 @@ def run_ours(args, cfg, world, rank, local, pg):
 
     # inputs: ROTATE independent sets, each seeded per (set, rank); with the
     # column split every rank draws the same layer and keeps its column block
-    sets = []
-    host_x = []
+    sets, host_x = [], []
     X0 = W0 = None
     nrot = max(1, args.rotate)
     for r in range(nrot):
@@ -346,7 +491,7 @@ def run_ours(args, cfg, world, rank, local, pg):
         step(i)
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev)
     launches0 = i8.int8_kernel_launch_count()
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
@@ -410,32 +555,31 @@ def run_ours(args, cfg, world, rank, local, pg):
     pk = peaks()
     decode = T <= i8.DECODE_MAX_T
     if decode:
+        kernel = "gemm_decode_kernel"
         achieved = (wbytes + 2 * T * K + 2 * T * N) / (gemm_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "peak_src": f"{pk['src']} HBM copy bandwidth"}
+                "frac": achieved / pk["hbm_gbs"], "peak_src": f"{pk['src']} HBM copy bandwidth",
+                "algorithmic_bytes_per_launch": wbytes + 2 * T * K + 2 * T * N}
     else:
-        # the GEMM is timed inside thousands of back-to-back steps, under the
-        # power cap: the sustained GEMM figure is the matching denominator
-        # (the burst one is reported beside it)
-        burst = 2.0 * pk["bf16_tflops"]
-        sustained = 2.0 * (pk["bf16_tflops_sustained"] or pk["bf16_tflops"])
+        kernel = "gemm_prefill_pair_kernel"
+        region_s = ms_step * args.steps * 1e-3          # the length of the GEMM-timing pass
+        peak, src = tensor_peak(pk, region_s)
         achieved = ops / (gemm_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": sustained, "unit": "TFLOP/s",
-                "frac": achieved / sustained,
-                "peak_src": f"{pk['src']} bf16 sustained x 2 (dense int8 : bf16 nominal ratio 4.5 : 2.25)",
-                "peak_burst": burst, "frac_of_burst": achieved / burst}
-    roof["traffic"] = ncu_traffic(args.workload) if args.variant == "w16" else None
-    roof["kernel"] = ("gemm_decode_kernel (split-K GEMM + fused finalisation)" if decode
-                      else "gemm_prefill_pair_kernel (CTA-pair int8 + fp16 MMA, fused epilogue)")
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_src": src, "algorithmic_ops_per_launch": ops}
+        cub = cublas_int8_tops(T, K, NL, dev) if with_cublas else None
+        if cub:
+            roof["int8_cublas_measured"] = cub
+            roof["frac_of_int8_cublas"] = achieved / cub
+            roof["int8_cublas_note"] = ("torch._int_mm (cuBLAS int8 x int8 -> int32, no outlier part, no "
+                                        "quantisation) on the same shape, 10 calls, timed in this process")
+    roof["traffic"] = ncu_traffic(name, kernel) if args.variant == "w16" else None
+    roof["kernel"] = kernel
     roof["kernel_ms"] = gemm_ms
 
-    line = {
-        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "strong" if column else "weak",
-        "vs_baseline": None, "dtype": "i8", "data": "synthetic, seeded (N(0,1) activations with planted outlier "
-        "columns, N(0,sigma) weights); no datasets or trained weights",
-        "config": {"workload": args.workload, "T": T, "K": K, "N": N, "alpha": alpha, "outlier_cols": n_out,
+    out = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "ms_per_step": ms_step,
+        "config": {"workload": name, "T": T, "K": K, "N": N, "alpha": alpha, "outlier_cols": n_out,
                    "frac_8bit": frac8,
                    "parallelism": (f"column-parallel x{world}: weight columns split, Y all-gathered over NCCL"
                                    if column else f"replicas x{world}" if world > 1 else "single GPU"),
@@ -453,10 +597,29 @@ def run_ours(args, cfg, world, rank, local, pg):
         "device_status": status,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tops, R, C, dt, cores, _, _ = oracle_sample(cfg, X0, W0, variant=args.variant)
-        line["cpu_baseline"] = {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
-                                "sample": f"sub-batch of {R} of {T} rows x {C} of {N} columns ({dt:.1f} s, "
-                                          f"whole method incl. outlier scan); weight conversion untimed"}
+        out["cpu_baseline"] = cpu_baseline(cfg, X0, W0, args.variant, 15.0 if not decode else 8.0)
+    del sets, Y, Y_full, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, world, rank, local, pg):
+    import torch
+    torch.cuda.set_device(local)
+    cfgs = all_configs()
+    head = measure(args, args.workload, cfgs[args.workload], world, rank, local, pg, with_cublas=True)
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "strong" if (args.parallel == "column" and world > 1) else "weak",
+        "vs_baseline": None, "dtype": "i8", "data": "synthetic, seeded (N(0,1) activations with planted outlier "
+        "columns, N(0,sigma) weights); no datasets or trained weights",
+    }
+    line.update({k: v for k, v in head.items() if k not in line})
+    if args.decode_workload != "none":
+        d = measure(args, args.decode_workload, cfgs[args.decode_workload], world, rank, local, pg,
+                    with_cublas=False)
+        line["decode"] = d
     if rank == 0:
         print(json.dumps(line), flush=True)
     if pg is not None:
@@ -474,7 +637,10 @@ def run_sweep(args):
     stream = torch.cuda.current_stream()
     pk = peaks()
     cfgs = wl.sweep_configs()
+    want_t = {int(t) for t in args.sweep_t.split(",")}
     for layer, (K, N) in wl.SWEEP_LAYERS.items():
+        if layer not in args.sweep_layers.split(","):
+            continue
         W = torch.from_numpy(wl.make_w(K, N, 0.01)).to(dev)
         Wq, sW = i8.int8_quantize_weight_colwise(W)
         Tmax = max(wl.SWEEP_T)
@@ -485,7 +651,7 @@ def run_sweep(args):
             ws = i8.workspace(Tmax, K, N, dev)
         Y = torch.empty((Tmax, N), dtype=torch.float16, device=dev)
         for name, cfg in cfgs.items():
-            if not name.startswith(f"b175_sweep_{layer}_"):
+            if not name.startswith(f"b175_sweep_{layer}_") or cfg["T"] not in want_t:
                 continue
             T, alpha = cfg["T"], cfg["alpha"]
             X = torch.from_numpy(wl.make_x(T, K, cfg["n_out"], cfg["lo"], cfg["hi"], cfg["row_prob"], cfg["seed"])).to(dev)
@@ -524,10 +690,12 @@ def run_sweep(args):
                     "weight_gbs": wbytes / (ms * 1e-3) / 1e9, "gemm_ms": gemm_ms,
                     "status": i8.int8_read_and_clear_device_status()}
             if T <= i8.DECODE_MAX_T:
-                line["gemm_frac_hbm"] = (wbytes + 2 * T * K + 2 * T * N) / (gemm_ms * 1e-3) / 1e9 / pk["hbm_gbs"]
+                io = 2 * T * K + 2 * T * N
+                line["gemm_frac_hbm"] = (wbytes + io) / (gemm_ms * 1e-3) / 1e9 / pk["hbm_gbs"]
+                line["call_frac_hbm"] = (wbytes + io) / (ms * 1e-3) / 1e9 / pk["hbm_gbs"]
             if T >= 128:
-                line["gemm_frac_int8_sustained"] = ops / (gemm_ms * 1e-3) / 1e12 / (
-                    2.0 * (pk["bf16_tflops_sustained"] or pk["bf16_tflops"]))
+                peak, _ = tensor_peak(pk, ms * steps * 1e-3)
+                line["gemm_frac_int8"] = ops / (gemm_ms * 1e-3) / 1e12 / peak
             print(json.dumps(line), flush=True)
             del X
         del W, Wq, sW, ws, Y
@@ -613,14 +781,14 @@ def main():
         run_chain(args)
         return
     cfgs = all_configs()
-    if args.workload not in cfgs:
-        raise SystemExit(f"unknown workload {args.workload}; known: {sorted(cfgs)[:8]} ...")
-    cfg = cfgs[args.workload]
+    for w in (args.workload, args.decode_workload):
+        if w != "none" and w not in cfgs:
+            raise SystemExit(f"unknown workload {w}; known: {sorted(cfgs)[:8]} ...")
     world, rank, local, pg = dist_setup(args)
     if args.impl == "reference":
-        run_reference(args, cfg, world, rank, pg)   # rank 0 only; other ranks exit 0
+        run_reference(args, world, rank)   # rank 0 only; other ranks exit 0
         return
-    run_ours(args, cfg, world, rank, local, pg)
+    run_ours(args, world, rank, local, pg)
 
 
 if __name__ == "__main__":

@@ -41,7 +41,9 @@
  *
  * Device-side anomalies (a pipeline wait that exceeded its time limit) do
  * not trap: the kernel records a code in a per-device status word and
- * returns early.  Read it with int8_read_and_clear_device_status().
+ * returns early.  Read it with int8_read_and_clear_device_status().  While
+ * the word is non-zero, the outputs of the calls made since it was last
+ * cleared are undefined (a kernel that gave up left part of them unwritten).
  */
 #ifndef INT8ROW_H
 #define INT8ROW_H
@@ -191,9 +193,13 @@ i8r_status int8_mixed_linear_chain(int n, const i8r_layer *layers,
  * int8_mixed_linear_workspace_size(T, K, N) exceeds that are rejected with
  * I8R_ERANGE before anything is enqueued (T <= 16 fits every 175B-sized
  * projection).  The first call on a device looks up the array's address
- * there, so make that first call before any stream capture.  Every call on a
- * device shares the one array: two calls that overlap on the GPU (different
- * streams, no ordering between them) race and corrupt each other's results.
+ * there (cudaGetSymbolAddress, with that device current), so make that first
+ * call before any stream capture; the address is looked up again when the
+ * calling thread's current context is no longer the one it was found in
+ * (after cudaDeviceReset, say), and that call too belongs outside a capture.
+ * Every call on a device shares the one array: two calls that overlap on the
+ * GPU (different streams, no ordering between them) race and corrupt each
+ * other's results.
  * Arguments, layouts, result and errors are otherwise those of
  * int8_mixed_linear.
  * ------------------------------------------------------------------------- */
@@ -239,8 +245,12 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha,
  * int8_debug_set_activation_path: 1 (the default) runs the activation side
  *   as one cooperative kernel for batches of 8 to 128 rows that fit in the
  *   SMs' shared memory, 2 as that kernel whenever the batch fits, 0 always
- *   as the outlier scan followed by the row quantiser.  All give the same
- *   bits; the switch (process-wide) exists so that tests can compare them.
+ *   as the outlier scan followed by the row quantiser.  When the runtime
+ *   refuses the cooperative launch (too few SMs or too little shared memory
+ *   free to the context), the call takes the scan + quantiser pair instead;
+ *   3 behaves as 1 with every cooperative launch treated as refused, so that
+ *   fallback can be tested.  All give the same bits; the switch
+ *   (process-wide) exists so that tests can compare them.
  *
  * int8_gemm_i8_s32: acc [T,N] int32 = Xq [T,K] int8 x Wq [K,N] int8, exact,
  *   by the same tensor-core kernels int8_mixed_linear uses (decode-shaped for

@@ -111,9 +111,12 @@ __global__ void __launch_bounds__(kFusedThreads, 1) activation_fused_kernel(
         }
     }
 
-    // 2. every block's rows are in the mask
+    // 2. every block's rows are in the mask.  A block whose rows never arrived
+    // says so (grid_ctr[1]) before it arrives, so no block goes on with a
+    // mask that lacks its rows.
     __syncthreads();
     if (tid == 0) {
+        if (!rows_ok) atomicOr(grid_ctr + 1, 1u);
         __threadfence();
         atomicAdd(grid_ctr, 1u);
         const uint64_t t0 = global_timer_ns();
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) activation_fused_kernel(
         }
         if (!done) report_status(I8R_DEV_PIPELINE_TIMEOUT);
         __threadfence();
-        ok_s = done && rows_ok;
+        ok_s = done && rows_ok && *reinterpret_cast<volatile unsigned *>(grid_ctr + 1) == 0u;
     }
     __syncthreads();
     griddep_launch_dependents();        // every block of this grid is resident: the GEMM may come in

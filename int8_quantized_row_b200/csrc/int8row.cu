@@ -10,8 +10,7 @@
 //                           outliers' W16 rows (dequantised Wq rows)        (a1-a3)
 // The scan and the quantiser are programmatic dependents of the kernel
 // before them, so each loads its rows of X before waiting for it.
-//   T > 128:  gemm_prefill_kernel (one CTA per 128 x 256 tile) or
-//             gemm_prefill_pair_kernel (CTA pairs, 256 x 256 tiles): int8 +
+//   T > 128:  gemm_prefill_pair_kernel (CTA pairs, 256 x 256 tiles): int8 +
 //             fp16 tensor-core MMA, epilogue -> Y
 //   T <= 128: gemm_decode_kernel   split-K int8 MMA -> int32 partial sums, one
 //             fp16 MMA segment per tile for the outlier part; the last
@@ -33,15 +32,8 @@
 #include "device_common.cuh"
 #include "quant_kernels.cuh"
 #include "activation_fused.cuh"
-#include "gemm_prefill.cuh"
 #include "gemm_prefill_pair.cuh"
 #include "gemm_decode.cuh"
-
-// Which prefill GEMM int8_mixed_linear / int8_gemm_i32 use for T > 128:
-// 1 = CTA pairs (cta_group::2), 0 = one CTA per tile.
-#ifndef I8R_PREFILL_PAIR
-#define I8R_PREFILL_PAIR 1
-#endif
 
 namespace {
 
@@ -58,18 +50,22 @@ thread_local cudaEvent_t tl_ev_after = nullptr;
 
 struct DeviceInfo {
     bool ready = false;
+    CUcontext ctx = nullptr;   // the context the setup below was done in
     bool sm100 = false;
     int sms = 0;
     int pair_clusters = 0;     // CTA pairs of the prefill GEMM that fit the GPU at once
     bool fused_ok = false;     // the one-kernel activation path can be launched (cooperative)
+    void *noalloc_scratch = nullptr;   // device address of the no-alloc scratch in `ctx`
 };
 // Which activation path runs (int8_debug_set_activation_path): 1 (default) the
 // one cooperative kernel for 8 <= T <= 128 when X fits in shared memory, 2 that
-// kernel whenever X fits, 0 always the scan + quantiser pair.
+// kernel whenever X fits, 0 always the scan + quantiser pair, 3 as 1 but with
+// the cooperative launch treated as refused (the fallback to the pair runs).
 std::atomic<int> g_activation_fused{1};
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
 
 #define I8R_CUDA(call)                                             \
     do {                                                           \
@@ -80,30 +76,57 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
         }                                                          \
     } while (0)
 
+#define I8R_TRY(expr)                         \
+    do {                                      \
+        i8r_status s_ = (expr);               \
+        if (s_ != I8R_OK) return s_;          \
+    } while (0)
+
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Per-device one-time setup: architecture check, SM count, kernel attributes,
-// the driver's tensor-map encoder.
+// Driver entry points the library uses (fetched once, under g_dev_mutex).
+i8r_status driver_entry_points() {
+    if (g_encode && g_ctx_current) return I8R_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    I8R_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !fn) return I8R_ECUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    fn = nullptr;
+    I8R_CUDA(cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !fn) return I8R_ECUDA;
+    g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+    return I8R_OK;
+}
+
+CUcontext current_context() {
+    CUcontext c = nullptr;
+    if (g_ctx_current && g_ctx_current(&c) != CUDA_SUCCESS) c = nullptr;
+    return c;
+}
+
+// Per-device setup: architecture check, SM count, kernel attributes, the
+// driver's entry points.  Kernel attributes and symbol addresses belong to a
+// context, so the setup is done again whenever the calling thread's current
+// context is not the one it was done in (after cudaDeviceReset, or under a
+// context the caller made current).
 i8r_status device_setup(const DeviceInfo **out) {
     int dev = 0;
     I8R_CUDA(cudaGetDevice(&dev));
     if (dev < 0 || dev >= kMaxDevices) return I8R_ERANGE;
     std::lock_guard<std::mutex> lock(g_dev_mutex);
+    I8R_TRY(driver_entry_points());
     DeviceInfo &d = g_dev[dev];
-    if (!d.ready) {
+    if (!d.ready || current_context() != d.ctx) {
+        d.ready = false;
+        d.noalloc_scratch = nullptr;
         int major = 0, minor = 0;
         I8R_CUDA(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
         I8R_CUDA(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
         I8R_CUDA(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
         d.sm100 = (major == 10 && minor == 0);
         if (d.sm100) {
-            I8R_CUDA(cudaFuncSetAttribute(prefill::gemm_prefill_kernel<false>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(prefill::SMEM_BYTES)));
-            I8R_CUDA(cudaFuncSetAttribute(prefill::gemm_prefill_kernel<true>,
-                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(prefill::SMEM_BYTES)));
             I8R_CUDA(cudaFuncSetAttribute(prefill2::gemm_prefill_pair_kernel<false>,
                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(prefill2::SMEM_BYTES)));
@@ -132,13 +155,8 @@ i8r_status device_setup(const DeviceInfo **out) {
                                                                    kFusedSmemMax));
             d.fused_ok = per_sm >= 1;
         }
-        if (!g_encode) {
-            void *fn = nullptr;
-            cudaDriverEntryPointQueryResult q;
-            I8R_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
-            if (q != cudaDriverEntryPointSuccess || !fn) return I8R_ECUDA;
-            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-        }
+        // the runtime calls above made the device's context current if it was not
+        d.ctx = current_context();
         d.ready = true;
     }
     if (!d.sm100) return I8R_EARCH;
@@ -201,11 +219,6 @@ i8r_status check_ptr(const void *p) {
     return I8R_OK;
 }
 
-#define I8R_TRY(expr)                         \
-    do {                                      \
-        i8r_status s_ = (expr);               \
-        if (s_ != I8R_OK) return s_;          \
-    } while (0)
 
 // Workspace of int8_mixed_linear.
 struct Workspace {
@@ -226,7 +239,7 @@ Workspace ws_layout(int T, int K, int N, bool wq_only = false) {
     Workspace w{};
     size_t off = 0;
     w.count = off; off = align_up(off + sizeof(int32_t));
-    w.ctr = off;   off = align_up(off + sizeof(uint32_t));        // the fused activation kernel's grid barrier
+    w.ctr = off;   off = align_up(off + 2 * sizeof(uint32_t));    // the fused activation kernel's grid barrier
     w.mask = off;  off = align_up(off + static_cast<size_t>((K + 31) / 32) * 4);
     w.idx = off;   off = align_up(off + static_cast<size_t>(K) * 4);
     w.sX = off;    off = align_up(off + static_cast<size_t>(T) * 4);
@@ -332,7 +345,7 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     const int fG = std::max(1, dev->sms);
     const int fR = (T + fG - 1) / fG;
     const int mode = g_activation_fused.load(std::memory_order_relaxed);
-    const bool size_ok = mode == 2 ? T >= 1 : (mode == 1 && T >= kFusedMinRows && T <= decode::MAX_T);
+    const bool size_ok = mode == 2 ? T >= 1 : ((mode == 1 || mode == 3) && T >= kFusedMinRows && T <= decode::MAX_T);
     const bool fused = grid_ctr && size_ok && dev->fused_ok && fused_smem_bytes(fR, K) <= kFusedSmemMax;
     clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords, fused ? grid_ctr : nullptr);
     I8R_LAUNCHED();
@@ -351,15 +364,25 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
         cfg.attrs = attr;
         cfg.numAttrs = 2;
         const uint32_t thr = half_threshold_bits(alpha);
-        const cudaError_t e = cudaLaunchKernelEx(&cfg, activation_fused_kernel, X, T, K, thr | (thr << 16), fR, mask, grid_ctr, sX,
-                                                 Xq, Xo, idx, count, W16, Wq, sW, N, W16o, o_rows,
-                                                 static_cast<int4 *>(zero), zero_bytes / 16);
-        if (e != cudaSuccess) {
+        // mode 3 (a test switch) takes the refusal path below without asking
+        const cudaError_t e =
+            mode == 3 ? cudaErrorCooperativeLaunchTooLarge
+                      : cudaLaunchKernelEx(&cfg, activation_fused_kernel, X, T, K, thr | (thr << 16), fR, mask,
+                                           grid_ctr, sX, Xq, Xo, idx, count, W16, Wq, sW, N, W16o, o_rows,
+                                           static_cast<int4 *>(zero), zero_bytes / 16);
+        if (e == cudaSuccess) {
+            I8R_LAUNCHED();
+            return I8R_OK;
+        }
+        // The cooperative launch can be refused when the context has fewer SMs
+        // or less shared memory free than at setup (another green context, MPS
+        // limits).  Nothing was enqueued; the mask is clear, so the two-kernel
+        // path below gives the same bits.  Any other error is the caller's.
+        if (e != cudaErrorCooperativeLaunchTooLarge && e != cudaErrorLaunchOutOfResources) {
             tl_last_cuda_error = static_cast<int>(e);
             return I8R_ECUDA;
         }
-        I8R_LAUNCHED();
-        return I8R_OK;
+        (void)cudaGetLastError();       // the refusal is not sticky: clear it
     }
     if (T == 0) {
         // no rows: an empty outlier set still has to be published
@@ -411,64 +434,12 @@ void record_after(cudaStream_t s) {
 }
 
 // Prefill GEMM (T > 128): Y mode when Y != nullptr, else int32 accumulators.
-// One CTA per 128 x 256 tile, persistent over the tiles.
-[[maybe_unused]] i8r_status launch_prefill_single(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
-                                 const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
-                                 const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s) {
-    CUtensorMap map_xq, map_wq, map_xo, map_y;
-    I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, prefill::BM, prefill::BK));
-    I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, prefill::BK, 128));
-    if (Xo) {
-        I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, prefill::BM, prefill::OBK));
-    } else {
-        map_xo = map_xq;   // unused: no 16-bit part
-    }
-    if (Y) {
-        // 32 x 32 output blocks, unswizzled 64-byte rows
-        I8R_TRY(make_map(&map_y, Y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, N, 32, 32,
-                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
-    } else {
-        map_y = map_xq;    // unused: int32 output mode
-    }
-    prefill::Params p{};
-    p.T = T;
-    p.K = K;
-    p.N = N;
-    p.num_m = (T + prefill::BM - 1) / prefill::BM;
-    const int num_n = (N + prefill::BN - 1) / prefill::BN;
-    p.num_tiles = p.num_m * num_n;
-    p.KB = (K + prefill::BK - 1) / prefill::BK;
-    p.count = Y ? count : nullptr;
-    p.idx = idx;
-    p.W16 = W16;
-    p.sX = sX;
-    p.sW = sW;
-    p.Y = Y;
-    p.acc_out = acc_out;
-    const int grid = p.num_tiles < dev->sms ? p.num_tiles : dev->sms;
-    record_before(s);
-    cudaError_t e;
-    if (Y)
-        e = launch_dependent(prefill::gemm_prefill_kernel<false>, dim3(grid), dim3(prefill::THREADS),
-                             prefill::SMEM_BYTES, s, 1, map_xq, map_wq, map_xo, map_y, p);
-    else
-        e = launch_dependent(prefill::gemm_prefill_kernel<true>, dim3(grid), dim3(prefill::THREADS),
-                             prefill::SMEM_BYTES, s, 1, map_xq, map_wq, map_xo, map_y, p);
-    if (e != cudaSuccess) {
-        tl_last_cuda_error = static_cast<int>(e);
-        return I8R_ECUDA;
-    }
-    I8R_LAUNCHED();
-    record_after(s);
-    return I8R_OK;
-}
-
-// Same contract; CTA pairs (clusters of 2) compute 256 x 256 tiles with
-// cta_group::2 MMAs.
-[[maybe_unused]] i8r_status launch_prefill_pair(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
-                               const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
-                               const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s,
-                               const __half *W16o) {
+// CTA pairs (clusters of 2) compute 256 x 256 tiles with cta_group::2 MMAs,
+// persistent over the tiles.
+i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
+                          const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
+                          const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s,
+                          const __half *W16o = nullptr) {
     CUtensorMap map_xq, map_wq, map_xo, map_w16, map_w16x4, map_w16o, map_y;
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, 128, prefill2::A_BOX_K));
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, prefill2::BK, 128));
@@ -533,17 +504,6 @@ void record_after(cudaStream_t s) {
     I8R_LAUNCHED();
     record_after(s);
     return I8R_OK;
-}
-
-i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half *Xo, int T, int K,
-                          const int8_t *Wq, const float *sW, const __half *W16, int N, const int32_t *count,
-                          const int32_t *idx, const float *sX, __half *Y, int32_t *acc_out, cudaStream_t s,
-                          const __half *W16o = nullptr) {
-#if I8R_PREFILL_PAIR
-    return launch_prefill_pair(dev, Xq, Xo, T, K, Wq, sW, W16, N, count, idx, sX, Y, acc_out, s, W16o);
-#else
-    return launch_prefill_single(dev, Xq, Xo, T, K, Wq, sW, W16, N, count, idx, sX, Y, acc_out, s);
-#endif
 }
 
 // Decode GEMM (T <= 128): int32 partial sums added into acc32, which must be
@@ -629,22 +589,25 @@ __global__ void zero_kernel(int4 *p, size_t n16) {
 // ---------------------------------------------------------------------------
 static constexpr size_t kNoAllocScratchBytes = 8u << 20;   // 8 MiB per GPU
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
-static void *g_noalloc_scratch_ptr[kMaxDevices];           // guarded by g_dev_mutex
 
-// Device address of g_noalloc_scratch on the current device; looked up the first
-// time a device is seen, with that device current.
+// Device address of g_noalloc_scratch on the current device, looked up with
+// that device current the first time the device is used in its current
+// context (device_setup forgets the address when the context changes, e.g.
+// after cudaDeviceReset, where the array is placed afresh).
 static i8r_status noalloc_scratch_address(void **out) {
+    const DeviceInfo *info = nullptr;
+    I8R_TRY(device_setup(&info));
     int dev = 0;
     I8R_CUDA(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= kMaxDevices) return I8R_ERANGE;
     std::lock_guard<std::mutex> lock(g_dev_mutex);
-    if (!g_noalloc_scratch_ptr[dev]) {
+    DeviceInfo &d = g_dev[dev];
+    if (!d.noalloc_scratch) {
         void *p = nullptr;
         I8R_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch));
         if (!p) return I8R_ECUDA;
-        g_noalloc_scratch_ptr[dev] = p;
+        d.noalloc_scratch = p;
     }
-    *out = g_noalloc_scratch_ptr[dev];
+    *out = d.noalloc_scratch;
     return I8R_OK;
 }
 
@@ -688,9 +651,6 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     I8R_TRY(check_ptr(sW));
     if (!wq_only) I8R_TRY(check_ptr(W16));
     I8R_TRY(check_ptr(Y));
-#if !I8R_PREFILL_PAIR
-    if (wq_only && T > decode::MAX_T) return I8R_EARCH;      // the one-CTA GEMM needs W16
-#endif
     const Workspace w = ws_layout(T, K, N, wq_only);
     if (!workspace || workspace_bytes < w.total) return I8R_EWORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return I8R_EALIGN;
@@ -717,11 +677,7 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     // compacted outlier rows: the prefill GEMM's first compact_rows(K), and the
     // Wq-only variant's dequantised rows at every T (the decode GEMM gathers W16
     // rows itself)
-#if I8R_PREFILL_PAIR
     __half *W16o = (small_t && !wq_only) ? nullptr : reinterpret_cast<__half *>(ws + w.W16o);
-#else
-    __half *W16o = (small_t && wq_only) ? reinterpret_cast<__half *>(ws + w.W16o) : nullptr;
-#endif
     I8R_TRY(launch_activation(dev, x, T, K, alpha, mask, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
                               zero_bytes, stream, w16, N, W16o, Wq, sW, reinterpret_cast<unsigned *>(ws + w.ctr)));
     if (!small_t)
@@ -786,9 +742,6 @@ i8r_status int8_mixed_linear_chain(int n, const i8r_layer *layers, void *workspa
         I8R_TRY(check_ptr(l.sW));
         if (l.W16) I8R_TRY(check_ptr(l.W16));
         I8R_TRY(check_ptr(l.Y));
-#if !I8R_PREFILL_PAIR
-        if (!l.W16 && l.T > decode::MAX_T) return I8R_EARCH;
-#endif
         if (!workspace || workspace_bytes < ws_layout(l.T, l.K, l.N, l.W16 == nullptr).total) return I8R_EWORKSPACE;
     }
     if (n > 0 && reinterpret_cast<uintptr_t>(workspace) % kAlign) return I8R_EALIGN;
@@ -802,7 +755,7 @@ i8r_status int8_mixed_linear_chain(int n, const i8r_layer *layers, void *workspa
 
 size_t int8_mixed_linear_noalloc_max_workspace(void) { return kNoAllocScratchBytes; }
 
-void int8_debug_set_activation_path(int mode) { g_activation_fused.store(mode < 0 ? 0 : (mode > 2 ? 2 : mode)); }
+void int8_debug_set_activation_path(int mode) { g_activation_fused.store(mode < 0 ? 0 : (mode > 3 ? 3 : mode)); }
 
 i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K, const int8_t *Wq, const float *sW,
                                      const void *W16, int N, float alpha, void *Y, cudaStream_t stream) {

@@ -185,7 +185,10 @@ __global__ void __launch_bounds__(256) clear_mask_kernel(uint32_t *__restrict__ 
                                                          unsigned *__restrict__ grid_ctr) {
     griddep_launch_dependents();        // the scan may start loading rows
     for (int w = threadIdx.x; w < nwords; w += blockDim.x) mask[w] = 0u;
-    if (grid_ctr && threadIdx.x == 0) *grid_ctr = 0u;     // the fused kernel's grid barrier
+    if (grid_ctr && threadIdx.x == 0) {                   // the fused kernel's grid barrier
+        grid_ctr[0] = 0u;                                 // arrivals
+        grid_ctr[1] = 0u;                                 // some block's rows did not arrive
+    }
 }
 
 __global__ void __launch_bounds__(kScanThreads) outlier_scan_kernel(const __half *__restrict__ X, int T, int K,

@@ -28,7 +28,7 @@ def _run_bench(env_extra, *args):
 
 def test_reference_arm_prints_one_json_line():
     r = _run_bench({}, "--impl", "reference", "--workload", "single_linear_16x1024x1024",
-                   "--steps", "3", "--warmup", "1")
+                   "--decode-workload", "single_linear_16x1024x1024", "--steps", "3", "--warmup", "1")
     assert r.returncode == 0, r.stderr
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
@@ -39,12 +39,14 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["config"]["workload"] == "single_linear_16x1024x1024"
+    dec = d["decode"]
+    assert dec["value"] > 0 and dec["cpu_baseline"]["kind"] == "oracle" and dec["config"]["T"] == 16
 
 
 def test_reference_arm_nonzero_rank_exits_silently():
     env = {"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"}
     r = _run_bench(env, "--impl", "reference", "--workload", "single_linear_16x1024x1024",
-                   "--steps", "2", "--warmup", "1")
+                   "--decode-workload", "none", "--steps", "2", "--warmup", "1")
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
 
@@ -103,3 +105,48 @@ def test_work_counts():
     ops, wbytes = bench.work({"T": 2, "K": 32, "N": 16}, 3)
     assert ops == 2 * 2 * 32 * 16
     assert wbytes == 32 * 16 + 4 * 16 + 2 * 3 * 16
+
+
+def test_default_workloads_are_the_largest_prefill_and_a_decode_point():
+    cfgs = bench.all_configs()
+    single_gpu = [c for n, c in wl_configs().items()]
+    biggest = max(single_gpu, key=lambda c: 2 * c["T"] * c["K"] * c["N"])
+    assert cfgs[bench.DEFAULT_WORKLOAD] == biggest
+    d = cfgs[bench.DECODE_WORKLOAD]
+    assert d["T"] <= 16 and d["K"] == 12288 and d["N"] == 49152
+
+
+def wl_configs():
+    from int8_quantized_row_b200 import workloads as wl
+    return wl.CONFIGS
+
+
+def test_nvml_clock_summary():
+    samples = [(1965.0, 700.0, 0x0), (1800.0, 990.0, 0x4), (1890.0, 950.0, 0x4 | 0x1)]
+    d = bench.summarise_clock_samples(samples, 1965.0, "test")
+    assert d["sm_mhz"] == 1890.0 and d["sm_max_mhz"] == 1965.0 and d["samples"] == 3
+    assert d["reasons"] == ["sw_power_cap"] and d["power_w_max"] == 990.0
+    d = bench.summarise_clock_samples([(1500.0, 1.0, 0x8 | 0x40)], 1965.0, "test")
+    assert d["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+    assert bench.summarise_clock_samples([], 1965.0, "test")["sm_mhz"] is None
+
+
+def test_tensor_peak_follows_the_timed_region():
+    pk = dict(hbm_gbs=1.0, bf16_tflops=1687.0, bf16_tflops_sustained=1436.0, src="measured")
+    burst, src = bench.tensor_peak(pk, 0.03)
+    assert burst == 2 * 1687.0 and "burst" in src
+    sus, src = bench.tensor_peak(pk, 5.0)
+    assert sus == 2 * 1436.0 and "sustained" in src
+
+
+def test_traffic_is_keyed_on_the_kernel_sources(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    sha = bench.kernel_source_sha("gemm_decode_kernel")
+    assert sha != bench.kernel_source_sha("gemm_prefill_pair_kernel")
+    rec = {"captures": {"w": {"kernel": "gemm_decode_kernel", "source_sha": sha, "bytes_per_launch": 123}}}
+    (tmp_path / "ncu_traffic.json").write_text(json.dumps(rec))
+    assert bench.ncu_traffic("w", "gemm_decode_kernel") == 123
+    assert bench.ncu_traffic("w", "gemm_prefill_pair_kernel") is None
+    rec["captures"]["w"]["source_sha"] = "stale"
+    (tmp_path / "ncu_traffic.json").write_text(json.dumps(rec))
+    assert bench.ncu_traffic("w", "gemm_decode_kernel") is None

@@ -77,17 +77,25 @@ def test_gather_over_gloo_reassembles_the_full_output(N, wq_only):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("T,world,wq_only", [(16, 2, False), (300, 3, False), (16, 4, True)])
-def test_column_blocks_are_bit_identical_to_the_full_layer(T, world, wq_only):
+def test_column_blocks_are_bit_identical_to_the_full_layer(orc, T, world, wq_only):
     import int8_quantized_row_b200 as i8
-    from gpu_helpers import device_status_clean, outlier_x, to_dev, to_host
+    from gpu_helpers import assert_y_close, device_status_clean, outlier_x, to_dev, to_host
     K, N = 2048, 2048 + 16 * world            # uneven blocks
     rng = np.random.default_rng(T + world)
-    X = to_dev(outlier_x(rng, T, K, [3, 700, 2000]))
-    W = to_dev((rng.standard_normal((K, N)) * 0.02).astype(np.float16))
+    Xh = outlier_x(rng, T, K, [3, 700, 2000])
+    Wh = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    X, W = to_dev(Xh), to_dev(Wh)
     Wq, sW = i8.int8_quantize_weight_colwise(W)
     full = i8.int8_mixed_linear_wq(X, Wq, sW, 6.0) if wq_only else i8.int8_mixed_linear(X, Wq, sW, W, 6.0)
     blocks = [cp.int8_mixed_linear_column_parallel(X, *cp.shard_columns(Wq, sW, None if wq_only else W, world, r), N,
                                                    6.0, world=world, rank=r, gather=False) for r in range(world)]
     torch.cuda.synchronize()
-    assert np.array_equal(to_host(torch.cat(blocks, dim=1)).view(np.uint16), to_host(full).view(np.uint16))
+    Y = to_host(torch.cat(blocks, dim=1))
+    assert np.array_equal(Y.view(np.uint16), to_host(full).view(np.uint16))
+    # and the reassembled layer is the oracle's, on sampled rows
+    Wq_o, sW_o = orc.quantize_weight_colwise(Wh)
+    rows = np.unique(np.r_[0:T:7, T - 1]).astype(np.int32)
+    Y_o, _, _, cnt = orc.mixed_linear(Xh, Wq_o, sW_o, None if wq_only else Wh, 6.0, rows=rows)
+    assert cnt == 3
+    assert_y_close(Y[rows], Y_o, f"column-parallel x{world} T={T}")
     assert device_status_clean()

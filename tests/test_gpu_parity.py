@@ -130,30 +130,70 @@ FUSED_CASES = ACT_CASES + [
 
 
 @pytest.mark.parametrize("T,K,cols,alpha", FUSED_CASES)
-def test_fused_activation_equals_two_kernel_path(T, K, cols, alpha):
-    """The one-kernel activation path (X held in shared memory, grid barrier)
-    gives the same bits as the outlier scan followed by the row quantiser."""
+def test_fused_activation_equals_two_kernel_path(orc, T, K, cols, alpha):
+    """Both activation paths, the one-kernel path (X held in shared memory,
+    grid barrier, fp16 bit-pattern threshold) and the outlier scan followed by
+    the row quantiser, each give the oracle's mask, index list, count, row
+    scales, codes and gathered outlier columns bit for bit, including at
+    thresholds fp16 cannot hold."""
     rng = np.random.default_rng(T * 7 + K)
     X = outlier_x(rng, T, K, cols)
     if T > 2:
         X[1] = 0
+    if 0.0 < alpha < float("inf"):
+        # the fp16 values next to the threshold (which fp16 may not hold exactly)
+        a = np.float16(alpha)
+        X[0, :4] = [a, np.nextafter(a, np.float16(0)), np.nextafter(a, np.float16(np.inf)), -a]
+    mask_o, idx_o = orc.outlier_columns(X, alpha)
+    Xq_o, sX_o = orc.quantize_rows(X, mask_o)
+    cnt_o = len(idx_o)
+    pad = min((cnt_o + 63) // 64 * 64, K)
     Xd = to_dev(X)
-    outs = []
     try:
         for fused in (2, 0):            # the one-kernel path wherever X fits, then the two kernels
             i8.int8_debug_set_activation_path(fused)
-            outs.append({k: to_host(v).copy() for k, v in i8.int8_quantize_activation(Xd, alpha).items()})
+            out = {k: to_host(v).copy() for k, v in i8.int8_quantize_activation(Xd, alpha).items()}
+            what = f"path {fused}"
+            cnt = int(out["count"][0])
+            assert cnt == cnt_o, what
+            words = out["mask"].view(np.uint32)
+            bits = (words[np.arange(K) // 32] >> (np.arange(K) % 32)) & 1
+            assert np.array_equal(bits.astype(bool), mask_o), what
+            assert np.array_equal(out["idx"][:cnt], idx_o), what
+            assert np.array_equal(out["sX"][:T], sX_o), what
+            assert np.array_equal(out["Xq"][:T], Xq_o), what
+            Xo = out["Xo"][:T]
+            assert np.array_equal(Xo[:, :cnt].view(np.uint16), X[:, idx_o].view(np.uint16)), what
+            assert np.all(Xo[:, cnt:pad] == 0), what
+            assert device_status_clean()
     finally:
         i8.int8_debug_set_activation_path(1)
-    a, b = outs
-    cnt = int(a["count"][0])
-    assert cnt == int(b["count"][0])
-    for k in ("mask", "sX", "Xq"):
-        assert np.array_equal(a[k], b[k]), k
-    assert np.array_equal(a["idx"][:cnt], b["idx"][:cnt])
-    pad = min((cnt + 63) // 64 * 64, K)
-    assert np.array_equal(a["Xo"][:T, :pad].view(np.uint16), b["Xo"][:T, :pad].view(np.uint16))
-    assert device_status_clean()
+
+
+@pytest.mark.parametrize("T,K", [(16, 1024), (100, 12288)])
+def test_refused_cooperative_launch_falls_back_to_two_kernels(orc, T, K):
+    """When the runtime refuses the one-kernel path's cooperative launch, the
+    call runs the outlier scan and the row quantiser instead (mode 3 treats
+    every cooperative launch as refused): one more launch, the oracle's bits."""
+    rng = np.random.default_rng(T + K)
+    X = outlier_x(rng, T, K, [1, K // 3])
+    mask_o, idx_o = orc.outlier_columns(X, 6.0)
+    Xq_o, sX_o = orc.quantize_rows(X, mask_o)
+    Xd = to_dev(X)
+    launches = {}
+    try:
+        for mode in (1, 3):
+            i8.int8_debug_set_activation_path(mode)
+            n0 = i8.int8_kernel_launch_count()
+            out = {k: to_host(v).copy() for k, v in i8.int8_quantize_activation(Xd, 6.0).items()}
+            launches[mode] = i8.int8_kernel_launch_count() - n0
+            cnt = int(out["count"][0])
+            assert cnt == len(idx_o) and np.array_equal(out["idx"][:cnt], idx_o)
+            assert np.array_equal(out["sX"][:T], sX_o) and np.array_equal(out["Xq"][:T], Xq_o)
+            assert device_status_clean()
+    finally:
+        i8.int8_debug_set_activation_path(1)
+    assert launches == {1: 2, 3: 3}     # clear + fused kernel; clear + scan + quantiser
 
 
 def test_activation_t0_is_noop():

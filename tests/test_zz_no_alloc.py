@@ -6,9 +6,10 @@ output buffers from a runtime owning the GPU's memory, or a path where
 cudaMalloc may not block or synchronise).  Its scratch is a fixed array
 inside the library.  It is called here through the C ABI, twice in a row
 (the second call finds the first call's leftovers in the shared scratch),
-and must give the workspace entry point's Y within the Y tolerance.  This
-file is collected last, so a run that stops at the first failure has already
-run every other test; it also passes on its own in a fresh process.
+and must give the workspace entry point's Y, and the oracle's, within the Y
+tolerance.  This file is collected last, so a run that stops at the first
+failure has already run every other test; it also passes on its own in a
+fresh process.
 """
 import ctypes
 
@@ -38,7 +39,7 @@ def _ptr(t):
 
 
 @pytest.mark.parametrize("T,K,N", [(16, 1024, 1024), (16, 12288, 4096), (200, 2048, 512)])
-def test_noalloc_matches_workspace_entry_point(T, K, N):
+def test_noalloc_matches_workspace_entry_point(orc, T, K, N):
     f, cap = _entry()
     assert i8.int8_mixed_linear_workspace_size(T, K, N) <= cap
     rng = np.random.default_rng(T + K + N)
@@ -47,13 +48,16 @@ def test_noalloc_matches_workspace_entry_point(T, K, N):
     Xd, Wd = to_dev(X), to_dev(W)
     Wq, sW = i8.int8_quantize_weight_colwise(Wd)
     ref = to_host(i8.int8_mixed_linear(Xd, Wq, sW, Wd, 6.0))
+    Wq_o, sW_o = orc.quantize_weight_colwise(W)
+    Y_o, _, _, _ = orc.mixed_linear(X, Wq_o, sW_o, W, 6.0)
     stream = _P(torch.cuda.current_stream().cuda_stream)
     for _ in range(2):
         Y = torch.full((T, N), float("nan"), dtype=torch.float16, device="cuda")
         rc = f(_ptr(Xd), T, K, _ptr(Wq), _ptr(sW), _ptr(Wd), N, 6.0, _ptr(Y), stream)
         assert rc == 0, i8.int8_status_string(rc)
         torch.cuda.synchronize()
-        assert_y_close(to_host(Y), ref, f"noalloc T={T} K={K} N={N}")
+        assert_y_close(to_host(Y), ref, f"noalloc vs workspace entry point T={T} K={K} N={N}")
+        assert_y_close(to_host(Y), Y_o, f"noalloc vs oracle T={T} K={K} N={N}")
     assert i8.int8_read_and_clear_device_status() == 0
 
 

@@ -57,6 +57,12 @@ def _bind(so):
     so.orc_dequantize_weight.restype = None
     so.orc_mixed_linear.argtypes = [_P, _I, _I, _P, _P, _P, _I, _F, _P, _I, _P, _P, _P]
     so.orc_mixed_linear.restype = _I
+    so.orc_int4_quantize_groupwise.argtypes = [_P, _I, _I, _I, _P, _P, _P]
+    so.orc_int4_quantize_groupwise.restype = None
+    so.orc_int4_dequantize.argtypes = [_P, _P, _P, _I, _I, _I, _P]
+    so.orc_int4_dequantize.restype = None
+    so.orc_int4_linear.argtypes = [_P, _I, _I, _P, _P, _P, _I, _I, _P, _I, _P, _P]
+    so.orc_int4_linear.restype = None
     return so
 
 
@@ -165,6 +171,46 @@ class Oracle:
         if cnt < 0:
             raise ArithmeticError("oracle: an int32 accumulator disagreed with its int64 sum")
         return Y.view(np.float16), Ypre, acc, cnt
+
+    # --- the group-wise 4-bit weight codec (FlexGen summary) ---
+    def int4_quantize_groupwise(self, W16, G=64):
+        """W16 fp16 [K,N] -> (codes uint8 [K,N] in 0..15, scale fp16 [K/G,N], lo fp16 [K/G,N])."""
+        W16 = _c(W16, np.float16)
+        K, N = W16.shape
+        if K % G:
+            raise ValueError("K must be a multiple of the group size")
+        codes = np.empty((K, N), np.uint8)
+        scale = np.empty((K // G, N), np.uint16)
+        lo = np.empty((K // G, N), np.uint16)
+        self.so.orc_int4_quantize_groupwise(_ptr(W16), K, N, G, _ptr(codes), _ptr(scale), _ptr(lo))
+        return codes, scale.view(np.float16), lo.view(np.float16)
+
+    def int4_dequantize(self, codes, scale, lo):
+        """fp16 [K,N]: the decoded 4-bit weight, binary16 of q*s + lo."""
+        codes = _c(codes, np.uint8)
+        scale = _c(scale, np.float16)
+        lo = _c(lo, np.float16)
+        K, N = codes.shape
+        G = K // scale.shape[0]
+        out = np.empty((K, N), np.uint16)
+        self.so.orc_int4_dequantize(_ptr(codes), _ptr(scale), _ptr(lo), K, N, G, _ptr(out))
+        return out.view(np.float16)
+
+    def int4_linear(self, X, codes, scale, lo, rows=None):
+        """(Y fp16 [r,N], Ypre float64 [r,N]) = X times the decoded 4-bit weight."""
+        X = _c(X, np.float16)
+        codes = _c(codes, np.uint8)
+        scale = _c(scale, np.float16)
+        lo = _c(lo, np.float16)
+        T, K = X.shape
+        N = codes.shape[1]
+        G = K // scale.shape[0]
+        rows = _c(np.arange(T) if rows is None else rows, np.int32)
+        Y = np.empty((len(rows), N), np.uint16)
+        Ypre = np.empty((len(rows), N), np.float64)
+        self.so.orc_int4_linear(_ptr(X), T, K, _ptr(codes), _ptr(scale), _ptr(lo), N, G, _ptr(rows), len(rows),
+                                _ptr(Y), _ptr(Ypre))
+        return Y.view(np.float16), Ypre
 
 
 def default():

@@ -42,6 +42,13 @@
  * take them in, so the int8 codes must match bit for bit.  Everything that
  * is not a quantisation decision is done in double.
  *
+ * The group-wise 4-bit weight codec (a second low-bit scheme on the pages:
+ * the FlexGen summary, research.elamur.ai, "sheng-2023-flexgen", which states
+ * that FlexGen compresses weights and the KV cache to 4 bits with group-wise
+ * quantization and no retraining or calibration) is at the end of this file.
+ * The page fixes neither the group, the code grid nor the rounding; the
+ * readings taken are stated there.
+ *
  * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
  */
 #include <math.h>
@@ -338,4 +345,98 @@ int orc_mixed_linear(const uint16_t *X, int T, int K,
     free(idx);
     free(is_outlier);
     return ok == 0 ? count : -1;
+}
+
+/* ------------------------------------------------------------------ */
+/* Group-wise 4-bit weight codec (FlexGen summary: weights compressed  */
+/* to 4 bits group-wise, with no retraining or calibration).           */
+/* ------------------------------------------------------------------ */
+/*
+ * Readings (the page gives no formula):
+ *   - a group is G consecutive rows k of one output column n of W [K,N]
+ *     (groups run along the reduction axis, so each inner product meets
+ *     K/G groups of its own column);
+ *   - asymmetric min-max codes: lo = min and hi = max of the group, 16 levels
+ *     lo + q*s, q in 0..15, with s = (hi - lo)/15 (nothing is calibrated);
+ *   - s is kept as binary16: s = half_rn( fl32( fl32(hi - lo) / 15 ) ), and lo,
+ *     a weight of the group, is binary16 already;
+ *   - the code: inv = fl32(1 / s) (0 when s == 0), then
+ *     q = clamp(rhaz( fl32( fl32(w - lo) * inv ) ), 0, 15), every step an IEEE
+ *     fp32 operation, so the GPU can take the same decisions bit for bit;
+ *   - the decoded weight is binary16, rounded once from the exact q*s + lo;
+ *   - the product uses the decoded weights with the activation as it is
+ *     (binary16), summed here in double and rounded once to binary16.
+ * Layout here: codes [K,N] one per byte; scale and lo [K/G,N] binary16 bits.
+ */
+
+void orc_int4_quantize_groupwise(const uint16_t *W16, int K, int N, int G,
+                                 uint8_t *codes, uint16_t *scale, uint16_t *lo_out)
+{
+    int groups = K / G;
+    #pragma omp parallel for schedule(static)
+    for (int n = 0; n < N; ++n) {
+        for (int g = 0; g < groups; ++g) {
+            float lo = INFINITY, hi = -INFINITY;
+            for (int k = g * G; k < (g + 1) * G; ++k) {
+                float w = orc_half_to_float(W16[(size_t)k * N + n]);
+                if (w < lo) lo = w;
+                if (w > hi) hi = w;
+            }
+            float range = hi - lo;                                /* fp32 subtraction */
+            uint16_t s16 = orc_double_to_half((double)(range / 15.0f));   /* fp32 division, then binary16 */
+            float s = orc_half_to_float(s16);
+            float inv = s > 0.0f ? 1.0f / s : 0.0f;               /* fp32 division */
+            scale[(size_t)g * N + n] = s16;
+            lo_out[(size_t)g * N + n] = orc_double_to_half((double)lo);   /* exact: lo is a weight */
+            for (int k = g * G; k < (g + 1) * G; ++k) {
+                float d = orc_half_to_float(W16[(size_t)k * N + n]) - lo;  /* fp32 subtraction */
+                float r = orc_rhaz(d * inv);                      /* one fp32 multiply */
+                if (r < 0.0f) r = 0.0f;
+                if (r > 15.0f) r = 15.0f;
+                codes[(size_t)k * N + n] = (uint8_t)r;
+            }
+        }
+    }
+}
+
+/* W16d[k,n] = binary16 of q*s + lo for the group of row k (q*s + lo is exact in
+ * double: every term is a multiple of 2^-24 below 2^21). */
+void orc_int4_dequantize(const uint8_t *codes, const uint16_t *scale, const uint16_t *lo,
+                         int K, int N, int G, uint16_t *W16d)
+{
+    for (int k = 0; k < K; ++k)
+        for (int n = 0; n < N; ++n) {
+            size_t gi = (size_t)(k / G) * N + n;
+            double v = (double)codes[(size_t)k * N + n] * (double)orc_half_to_float(scale[gi])
+                       + (double)orc_half_to_float(lo[gi]);
+            W16d[(size_t)k * N + n] = orc_double_to_half(v);
+        }
+}
+
+/* Y[r,n] = binary16 of sum_k X[rows[r],k] * W~[k,n] (double sums) for the listed
+ * rows, W~ the decoded 4-bit weight; Ypre (nullable) the sums before rounding. */
+void orc_int4_linear(const uint16_t *X, int T, int K, const uint8_t *codes,
+                     const uint16_t *scale, const uint16_t *lo, int N, int G,
+                     const int32_t *rows, int nrows, uint16_t *Y, double *Ypre)
+{
+    (void)T;
+    uint16_t *Wd = (uint16_t *)malloc((size_t)K * N * sizeof(uint16_t));
+    orc_int4_dequantize(codes, scale, lo, K, N, G, Wd);
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nrows; ++r) {
+        const uint16_t *xrow = X + (size_t)rows[r] * K;
+        double *y = (double *)calloc((size_t)N, sizeof(double));
+        for (int k = 0; k < K; ++k) {
+            double xv = (double)orc_half_to_float(xrow[k]);
+            if (xv == 0.0) continue;
+            const uint16_t *wrow = Wd + (size_t)k * N;
+            for (int n = 0; n < N; ++n) y[n] += xv * (double)orc_half_to_float(wrow[n]);
+        }
+        for (int n = 0; n < N; ++n) {
+            if (Ypre) Ypre[(size_t)r * N + n] = y[n];
+            Y[(size_t)r * N + n] = orc_double_to_half(y[n]);
+        }
+        free(y);
+    }
+    free(Wd);
 }

@@ -32,6 +32,14 @@ int  orc_mixed_linear(const uint16_t *X, int T, int K,
                       float alpha, const int32_t *rows, int nrows,
                       uint16_t *Y, double *Ypre, int32_t *acc_out);
 
+void orc_int4_quantize_groupwise(const uint16_t *W16, int K, int N, int G,
+                                 uint8_t *codes, uint16_t *scale, uint16_t *lo);
+void orc_int4_dequantize(const uint8_t *codes, const uint16_t *scale, const uint16_t *lo,
+                         int K, int N, int G, uint16_t *W16d);
+void orc_int4_linear(const uint16_t *X, int T, int K, const uint8_t *codes,
+                     const uint16_t *scale, const uint16_t *lo, int N, int G,
+                     const int32_t *rows, int nrows, uint16_t *Y, double *Ypre);
+
 #ifdef __cplusplus
 }
 #endif

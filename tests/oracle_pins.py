@@ -459,4 +459,146 @@ def pin_wq_only_variant_error(o):
     assert np.all(np.abs(P2 - P1) <= bound * (1 + 1e-9) + 1e-12)
     assert np.any(P2 != P1)                     # the variant really uses other rows
 
+# ---------------------------------------------------------------- group-wise 4-bit codec
+
+def _int4_grid_weights(rng, K, N, G):
+    """Weights that sit exactly on a 4-bit grid: per (group, column) a power-of-two
+    step s and a base lo (both exact in binary16), every level 0..15 present."""
+    Q = np.empty((K, N), np.int64)
+    S = np.empty((K // G, N))
+    L = np.empty((K // G, N))
+    W = np.empty((K, N))
+    for g in range(K // G):
+        for n in range(N):
+            q = np.r_[0, 15, rng.integers(0, 16, G - 2)]
+            rng.shuffle(q)
+            s = 2.0 ** int(rng.integers(-12, -2))
+            lo = float(rng.integers(-64, 64)) * s
+            Q[g * G:(g + 1) * G, n] = q
+            S[g, n], L[g, n] = s, lo
+            W[g * G:(g + 1) * G, n] = lo + q * s
+    return Q, S, L, W.astype(np.float16)
+
+
+def pin_int4_grid_exact(o):
+    """Weights already on a 16-level grid per (group of 64 rows, column) are coded
+    exactly: codes, step and base recovered, and the decoded weight is the weight
+    bit for bit.  Steps and bases differ per group and per column, so a group taken
+    along the wrong axis, or a wrong step (/16 for /15), fails here."""
+    rng = np.random.default_rng(41)
+    K, N, G = 192, 24, 64
+    Q, S, L, W = _int4_grid_weights(rng, K, N, G)
+    codes, scale, lo = o.int4_quantize_groupwise(W, G)
+    assert np.array_equal(codes.astype(np.int64), Q)
+    assert np.array_equal(scale.astype(np.float64), S)
+    assert np.array_equal(lo.astype(np.float64), L)
+    Wd = o.int4_dequantize(codes, scale, lo)
+    assert np.array_equal(Wd.view(np.uint16), W.view(np.uint16))
+
+
+def pin_int4_nearest_level(o):
+    """Brute force over the 16 levels of each group: the chosen level is the one
+    nearest the weight (exact rationals), up to the fp32 rounding of the step's
+    reciprocal, and the levels span the group (lo is its minimum, the top level
+    within rounding of its maximum)."""
+    rng = np.random.default_rng(42)
+    K, N, G = 128, 16, 64
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    W[64:128, 3] = (rng.standard_normal(64) * 3.0).astype(np.float16)     # a wide group
+    codes, scale, lo = o.int4_quantize_groupwise(W, G)
+    assert codes.max() <= 15
+    for g in range(K // G):
+        for n in range(N):
+            s, l = Fraction(float(scale[g, n])), Fraction(float(lo[g, n]))
+            grp = W[g * G:(g + 1) * G, n]
+            assert float(lo[g, n]) == float(grp.astype(np.float64).min())
+            rng_ = Fraction(float(grp.astype(np.float64).max())) - l
+            assert abs(15 * s - rng_) <= rng_ * Fraction(1, 1024) + Fraction(2.0 ** -24)   # binary16 step
+            assert codes[g * G + int(np.argmin(grp)), n] == 0
+            assert codes[g * G + int(np.argmax(grp)), n] == 15 or s == 0
+            for i, w in enumerate(grp):
+                wf = Fraction(float(w))
+                q = int(codes[g * G + i, n])
+                d = abs(wf - (l + q * s))
+                best = min(abs(wf - (l + j * s)) for j in range(16))
+                assert d <= best + s * Fraction(1, 2 ** 20), (g, n, i)
+
+
+def pin_int4_invariants(o):
+    """A constant group has step 0 and decodes exactly; scaling a column by 2^j
+    (no binary16 overflow or underflow) leaves its codes unchanged and scales step,
+    base and decoded weights by exactly 2^j."""
+    rng = np.random.default_rng(43)
+    K, N, G = 128, 8, 64
+    # magnitudes in [0.01, 0.2]: scaled by 2^-3 or 2^2 they stay normal binary16
+    W = (rng.uniform(0.01, 0.2, (K, N)) * rng.choice([-1.0, 1.0], (K, N))).astype(np.float16)
+    W[0:64, 0] = np.float16(0.375)
+    W[64:128, 1] = np.float16(-2.0)
+    codes, scale, lo = o.int4_quantize_groupwise(W, G)
+    assert scale[0, 0] == 0 and scale[1, 1] == 0
+    assert np.all(codes[0:64, 0] == 0) and np.all(codes[64:128, 1] == 0)
+    Wd = o.int4_dequantize(codes, scale, lo)
+    assert np.array_equal(Wd[:64, 0], W[:64, 0]) and np.array_equal(Wd[64:, 1], W[64:, 1])
+    for j in (-3, 2):
+        W2 = (W.astype(np.float64) * 2.0 ** j).astype(np.float16)
+        assert np.array_equal(W2.astype(np.float64), W.astype(np.float64) * 2.0 ** j)
+        c2, s2, l2 = o.int4_quantize_groupwise(W2, G)
+        assert np.array_equal(c2, codes)
+        assert np.array_equal(s2.astype(np.float64), scale.astype(np.float64) * 2.0 ** j)
+        assert np.array_equal(l2.astype(np.float64), lo.astype(np.float64) * 2.0 ** j)
+        assert np.array_equal(o.int4_dequantize(c2, s2, l2).astype(np.float64), Wd.astype(np.float64) * 2.0 ** j)
+
+
+def pin_int4_error_bound(o):
+    """|W~ - W| is at most half a step (plus the shortfall of 15 steps against the
+    group's range when the binary16 step rounded down) plus half a binary16 ulp
+    of W~, and the decoded value is binary16(q*s + lo) for the stored q, s, lo."""
+    rng = np.random.default_rng(44)
+    K, N, G = 256, 32, 64
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    codes, scale, lo = o.int4_quantize_groupwise(W, G)
+    Wd = o.int4_dequantize(codes, scale, lo)
+    s = np.repeat(scale.astype(np.float64), G, axis=0)
+    l = np.repeat(lo.astype(np.float64), G, axis=0)
+    exact = codes.astype(np.float64) * s + l                      # exact in double
+    assert np.array_equal(Wd.view(np.uint16), exact.astype(np.float16).view(np.uint16))   # numpy's RNE
+    grp = W.astype(np.float64).reshape(K // G, G, N)
+    short = np.repeat(np.maximum(grp.max(1) - grp.min(1) - 15 * scale.astype(np.float64), 0), G, axis=0)
+    bound = s / 2 * (1 + 2.0 ** -20) + short + np.array([_half_ulp(v) for v in Wd.ravel()]).reshape(K, N) / 2
+    assert np.all(np.abs(Wd.astype(np.float64) - W.astype(np.float64)) <= bound)
+
+
+def pin_int4_linear_is_the_matmul_of_the_decoded_weight(o):
+    """The 4-bit product is X times the decoded weight: numpy's float64 matmul of
+    the same operands, rounded by numpy to binary16 (equal except at exact
+    ties of the rounding); and with small integers and exact grids it is the
+    exact integer product."""
+    rng = np.random.default_rng(45)
+    T, K, N, G = 5, 192, 40, 64
+    X = rng.standard_normal((T, K)).astype(np.float16)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    codes, scale, lo = o.int4_quantize_groupwise(W, G)
+    Wd = o.int4_dequantize(codes, scale, lo)
+    Y, Ypre = o.int4_linear(X, codes, scale, lo)
+    ref = X.astype(np.float64) @ Wd.astype(np.float64)
+    mag = np.abs(X.astype(np.float64)) @ np.abs(Wd.astype(np.float64))
+    assert np.all(np.abs(Ypre - ref) <= 1e-12 * mag + 1e-300)
+    assert np.array_equal(Y.view(np.uint16), Ypre.astype(np.float16).view(np.uint16))
+    rows = np.array([4, 1], np.int32)
+    Ys, _ = o.int4_linear(X, codes, scale, lo, rows=rows)
+    assert np.array_equal(Ys.view(np.uint16), Y[rows].view(np.uint16))
+    # exact integers: X in -3..3, weights on integer grids (s = 1)
+    Q = rng.integers(0, 16, (K, N))
+    Q[0::64] = 0
+    Q[1::64] = 15
+    Wi = (Q - 7).astype(np.float16)
+    Xi = rng.integers(-3, 4, (T, K)).astype(np.float16)
+    ci, si, li = o.int4_quantize_groupwise(Wi, G)
+    assert np.array_equal(ci.astype(np.int64), Q) and np.all(si == 1) and np.all(li == -7)
+    Yi, _ = o.int4_linear(Xi, ci, si, li)
+    exact = Xi.astype(np.int64) @ (Q - 7)
+    assert np.abs(exact).max() <= 2048
+    assert np.array_equal(Yi.astype(np.int64), exact)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

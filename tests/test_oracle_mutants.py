@@ -38,6 +38,15 @@ MUTANTS = {
     "y_round_truncate": ("if (diff > 0.5) return fl + 1.0;", "if (diff > 2.0) return fl + 1.0;"),
     "scale_x_instead_of_w": ("* (double)sX[r] * (double)sW[n]", "* (double)sX[r] * (double)sX[r]"),
     "reciprocal_two_roundings": ("float v = x * inv;", "float v = (x * 127.0f) / (127.0f / inv);"),
+    # the group-wise 4-bit codec
+    "int4_step_by_16": ("(range / 15.0f)", "(range / 16.0f)"),
+    "int4_code_truncates": ("float r = orc_rhaz(d * inv);", "float r = truncf(d * inv);"),
+    "int4_group_skips_first_row": ("for (int k = g * G; k < (g + 1) * G; ++k) {\n                float w",
+                                   "for (int k = g * G + 1; k < (g + 1) * G; ++k) {\n                float w"),
+    "int4_codes_from_zero_not_lo": ("W16[(size_t)k * N + n]) - lo;", "W16[(size_t)k * N + n]) - 0.0f;"),
+    "int4_decode_drops_lo": ("+ (double)orc_half_to_float(lo[gi]);", "+ 0.0;"),
+    "int4_product_wrong_row": ("const uint16_t *wrow = Wd + (size_t)k * N;",
+                               "const uint16_t *wrow = Wd + (size_t)(k ^ 1) * N;"),
 }
 
 

@@ -83,6 +83,9 @@ def parse(argv=None):
                     help="N>1 ranks: replica = an independent batch per GPU (weak scaling, the default); "
                          "column = one layer split by weight columns over the GPUs, Y all-gathered over NCCL "
                          "(strong scaling)")
+    ap.add_argument("--codec", default="int8", choices=["int8", "int4"],
+                    help="--sweep only: int8 = the LLM.int8() layer; int4 = the group-wise 4-bit weight codec "
+                         "(int4_linear, T <= 64)")
     ap.add_argument("--variant", default="w16", choices=["w16", "wq"],
                     help="w16: int8_mixed_linear (fp16 weight resident for the outlier rows); "
                          "wq: int8_mixed_linear_wq (only Wq and sW resident)")
@@ -626,6 +629,72 @@ def run_ours(args, world, rank, local, pg):
         pg.destroy_process_group()
 
 
+def int4_bytes(T, K, N):
+    """Algorithmic bytes of one int4_linear call: the packed codes (1/2 byte per
+    weight) and the (s, lo) pairs (4 bytes per group of 64), X read, Y written."""
+    return K * N // 2 + (K // 64) * N * 4 + 2 * T * K + 2 * T * N
+
+
+def run_sweep_int4(args):
+    """The 175B decoder-layer projections with the group-wise 4-bit weight codec
+    (int4_linear): every layer's weight is drawn, packed once, and each T point
+    is timed over whole calls and over the GEMM kernel alone.  The packed
+    weights (76-302 MB) exceed L2, so every call streams them from HBM."""
+    import torch
+    import int8_quantized_row_b200 as i8
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    pk = peaks()
+    want_t = sorted(int(t) for t in args.sweep_t.split(",") if int(t) <= i8.INT4_MAX_T)
+    for layer, (K, N) in wl.SWEEP_LAYERS.items():
+        if layer not in args.sweep_layers.split(","):
+            continue
+        W = torch.from_numpy(wl.make_w(K, N, 0.01)).to(dev)
+        W4, S4 = i8.int4_quantize_weight_groupwise(W)
+        del W
+        ws = torch.empty(max(1, i8.int4_linear_workspace_size(max(want_t), K, N)), dtype=torch.uint8, device=dev)
+        for T in want_t:
+            X = torch.from_numpy(wl.make_x(T, K, 0, seed=T)).to(dev)
+            Y = torch.empty((T, N), dtype=torch.float16, device=dev)
+
+            def step():
+                i8.int4_linear(X, W4, S4, N, Y=Y, workspace_buf=ws)
+            steps = 200
+            for _ in range(5):
+                step()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(steps):
+                step()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / steps
+            gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for x, y in gev:
+                x.record(stream)
+                y.record(stream)
+            torch.cuda.synchronize()
+            for i in range(steps):
+                i8.int8_time_next_gemm(gev[i][0], gev[i][1])
+                step()
+            torch.cuda.synchronize()
+            gemm_ms = sum(x.elapsed_time(y) for x, y in gev) / steps
+            nbytes = int4_bytes(T, K, N)
+            line = {"workload": f"b175_int4_{layer}_t{T}_{K}x{N}", "codec": "int4 group-wise (64)", "T": T,
+                    "K": K, "N": N, "ms_per_call": ms, "gemm_ms": gemm_ms,
+                    "tops": 2.0 * T * K * N / (ms * 1e-3) / 1e12,
+                    "weight_gbs": (K * N // 2 + (K // 64) * N * 4) / (ms * 1e-3) / 1e9,
+                    "algorithmic_bytes": nbytes,
+                    "gemm_frac_hbm": nbytes / (gemm_ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                    "call_frac_hbm": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                    "status": i8.int8_read_and_clear_device_status()}
+            print(json.dumps(line), flush=True)
+            del X, Y
+        del W4, S4, ws
+        torch.cuda.empty_cache()
+
+
 def run_sweep(args):
     """The 175B decoder-layer sweep: each layer's weight is drawn and converted
     once, then every (T, outlier fraction, alpha) point is timed on it: whole
@@ -775,7 +844,7 @@ def run_chain(args):
 def main():
     args = parse()
     if args.sweep:
-        run_sweep(args)
+        run_sweep_int4(args) if args.codec == "int4" else run_sweep(args)
         return
     if args.chain:
         run_chain(args)

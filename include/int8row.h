@@ -210,6 +210,61 @@ i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K,
                                      float alpha, void *Y, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Group-wise 4-bit weight codec.  The FlexGen summary page (research.elamur.ai,
+ * "sheng-2023-flexgen") states that FlexGen compresses weights (and the KV
+ * cache) to 4 bits with group-wise quantization, without retraining or
+ * calibration; it gives no formula.  The reading taken here, for weights:
+ *   - a group is 64 consecutive rows k of one output column n of W [K,N];
+ *   - its 16 levels are lo + q*s, q = 0..15, with lo the group's minimum and
+ *     s = fp16_rn( fl32( fl32(hi - lo) / 15 ) ), hi the group's maximum;
+ *   - code q = clamp(rhaz( fl32( fl32(w - lo) * fl32(1 / s) ) ), 0, 15), each
+ *     step an IEEE fp32 operation (s = 0 gives q = 0);
+ *   - the decoded weight is W~ = fp16_rn(q*s + lo), rounded once;
+ *   - the product is Y = fp16( X W~ ) with fp32 accumulation; X stays fp16.
+ * K must be a multiple of 256 (>= 256) and N a multiple of 16.
+ *
+ * The packed weight is two device buffers in the layout the product streams
+ * (columns padded to a multiple of 256; KT = K / 256; both caller-owned):
+ *   W4  int4_packed_code_bytes(K, N) bytes: 32 KB blocks, block (nt, kt) at
+ *       byte (nt*KT + kt) * 32768 holds columns n = 256*nt + r (r < 256) and
+ *       rows k = 256*kt .. 256*kt + 255; column r's 128 bytes start at r*128
+ *       and hold eight 16-byte chunks, chunk c (codes k = 256*kt + 32c ..
+ *       +31) at chunk position c ^ (r % 8); in a chunk, 32-bit word i holds
+ *       codes 8i .. 8i+7, nibble j (bits 4j .. 4j+3) code 8i + 2j and nibble
+ *       j + 4 code 8i + 2j + 1, for j = 0..3;
+ *   S4  int4_packed_scale_bytes(K, N) bytes: 4 KB blocks, block (nt, kt) at
+ *       byte (nt*KT + kt) * 4096; column r's 16 bytes at r*16 are the fp16
+ *       pairs (s, lo) of groups 4*kt .. 4*kt + 3.
+ * Padding columns have codes 0 and s = lo = 0.
+ *
+ * int4_quantize_weight_groupwise: W16 [K,N] fp16 -> W4, S4.
+ * int4_dequantize_weight: W4, S4 -> W16d [K,N] fp16, the decoded weight W~
+ *   (for checking the codec; the product decodes on the fly).
+ * int4_linear: Y [T,N] fp16 = X [T,K] fp16 times W~, for 1 <= T <= 64 rows
+ *   (T = 0 is a no-op; larger T returns I8R_ERANGE).  The weight is streamed
+ *   at 0.5625 bytes per weight, decoded on the fly into the tensor cores'
+ *   operand memory.  Workspace of at least int4_linear_workspace_size(T, K, N)
+ *   bytes, 256-byte aligned (fp32 partial sums of tiles split over the SMs);
+ *   its contents on entry are ignored.  Two calls sharing a workspace must
+ *   not overlap on the GPU.  Sizes out of these rules return 0 from the size
+ *   queries and an error from the calls, before anything is enqueued.
+ * ------------------------------------------------------------------------- */
+size_t int4_packed_code_bytes(int K, int N);
+
+size_t int4_packed_scale_bytes(int K, int N);
+
+i8r_status int4_quantize_weight_groupwise(const void *W16, int K, int N, uint8_t *W4, void *S4,
+                                          cudaStream_t stream);
+
+i8r_status int4_dequantize_weight(const uint8_t *W4, const void *S4, int K, int N, void *W16d,
+                                  cudaStream_t stream);
+
+size_t int4_linear_workspace_size(int T, int K, int N);
+
+i8r_status int4_linear(const void *X, int T, int K, const uint8_t *W4, const void *S4, int N, void *Y,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Outlier statistics: the outlier feature dimensions of X and the share of
  * values that go through the 8-bit product (the pages report that share as
  * above 99.9% on large models; LLM.int8() abstract).
@@ -296,7 +351,7 @@ const char *int8_status_string(i8r_status status);
 /* The last CUDA error seen by an entry point on this host thread (cudaError_t). */
 int int8_last_cuda_error(void);
 
-/* Measurement hook: the next int8_mixed_linear or int8_gemm_i8_s32 call made
+/* Measurement hook: the next int8_mixed_linear, int8_gemm_i8_s32 or int4_linear call made
  * by this host thread records `before` (a cudaEvent_t) on its stream right
  * before its tensor-core GEMM kernel and `after` right after it, then forgets
  * both.  Pass NULL, NULL to cancel. */

@@ -18,10 +18,13 @@ __all__ = [
     "int8_gemm_i8_s32", "int8_read_and_clear_device_status", "int8_status_string",
     "int8_selftest_wait_timeout",
     "int8_time_next_gemm", "int8_kernel_launch_count", "LIB_PATH",
+    "int4_packed_code_bytes", "int4_packed_scale_bytes", "int4_quantize_weight_groupwise",
+    "int4_dequantize_weight", "int4_linear_workspace_size", "int4_linear",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libint8row.so")
 DECODE_MAX_T = 128
+INT4_MAX_T = 64
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int
@@ -81,8 +84,18 @@ def lib():
     so.int8_time_next_gemm.argtypes = [_P, _P]
     so.int8_time_next_gemm.restype = None
     so.int8_kernel_launch_count.restype = ctypes.c_uint64
+    so.int4_packed_code_bytes.argtypes = [_I, _I]
+    so.int4_packed_code_bytes.restype = _Z
+    so.int4_packed_scale_bytes.argtypes = [_I, _I]
+    so.int4_packed_scale_bytes.restype = _Z
+    so.int4_quantize_weight_groupwise.argtypes = [_P, _I, _I, _P, _P, _P]
+    so.int4_dequantize_weight.argtypes = [_P, _P, _I, _I, _P, _P]
+    so.int4_linear_workspace_size.argtypes = [_I, _I, _I]
+    so.int4_linear_workspace_size.restype = _Z
+    so.int4_linear.argtypes = [_P, _I, _I, _P, _P, _I, _P, _P, _Z, _P]
     for name in ("int8_quantize_weight_colwise", "int8_mixed_linear", "int8_outlier_stats",
-                 "int8_quantize_activation", "int8_gemm_i8_s32", "int8_read_and_clear_device_status"):
+                 "int8_quantize_activation", "int8_gemm_i8_s32", "int8_read_and_clear_device_status",
+                 "int4_quantize_weight_groupwise", "int4_dequantize_weight", "int4_linear"):
         getattr(so, name).restype = _I
     _lib = so
     return so
@@ -302,3 +315,59 @@ def int8_time_next_gemm(before, after):
 
 def int8_kernel_launch_count():
     return int(lib().int8_kernel_launch_count())
+
+
+# ---------------------------------------------------------------- group-wise 4-bit codec
+
+def int4_packed_code_bytes(K, N):
+    return int(lib().int4_packed_code_bytes(int(K), int(N)))
+
+
+def int4_packed_scale_bytes(K, N):
+    return int(lib().int4_packed_scale_bytes(int(K), int(N)))
+
+
+def int4_quantize_weight_groupwise(W16, stream=None):
+    """W16 fp16 [K,N] -> (W4 uint8, S4 uint8): the packed codes and (s, lo) pairs
+    in the layout include/int8row.h describes."""
+    import torch
+    K, N = W16.shape
+    nc, ns = int4_packed_code_bytes(K, N), int4_packed_scale_bytes(K, N)
+    if nc == 0:
+        raise I8RError("int4_quantize_weight_groupwise", 2 if K % 256 or N % 16 else 3)
+    W4 = torch.empty(nc, dtype=torch.uint8, device=W16.device)
+    S4 = torch.empty(ns, dtype=torch.uint8, device=W16.device)
+    _check("int4_quantize_weight_groupwise", lib().int4_quantize_weight_groupwise(
+        _dev(W16, torch.float16, "W16", 2), K, N, _dev(W4, torch.uint8, "W4"), _dev(S4, torch.uint8, "S4"),
+        _stream(stream)))
+    return W4, S4
+
+
+def int4_dequantize_weight(W4, S4, K, N, stream=None):
+    """The decoded weight W~ fp16 [K,N] of a packed 4-bit weight."""
+    import torch
+    out = torch.empty((K, N), dtype=torch.float16, device=W4.device)
+    _check("int4_dequantize_weight", lib().int4_dequantize_weight(
+        _dev(W4, torch.uint8, "W4"), _dev(S4, torch.uint8, "S4"), int(K), int(N), _dev(out, torch.float16, "W16d"),
+        _stream(stream)))
+    return out
+
+
+def int4_linear_workspace_size(T, K, N):
+    return int(lib().int4_linear_workspace_size(int(T), int(K), int(N)))
+
+
+def int4_linear(X, W4, S4, N, Y=None, workspace_buf=None, stream=None):
+    """Y fp16 [T,N] = X fp16 [T,K] times the decoded 4-bit weight (T <= 64)."""
+    import torch
+    T, K = X.shape
+    Y = torch.empty((T, N), dtype=torch.float16, device=X.device) if Y is None else Y
+    if workspace_buf is None:
+        workspace_buf = torch.empty(max(1, int4_linear_workspace_size(T, K, N)), dtype=torch.uint8,
+                                    device=X.device)
+    ws = workspace_buf
+    _check("int4_linear", lib().int4_linear(
+        _dev(X, torch.float16, "X", 2), T, K, _dev(W4, torch.uint8, "W4"), _dev(S4, torch.uint8, "S4"), int(N),
+        _dev(Y, torch.float16, "Y"), ctypes.c_void_p(ws.data_ptr()), ws.numel() * ws.element_size(),
+        _stream(stream)))
+    return Y

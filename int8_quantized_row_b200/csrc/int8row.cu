@@ -34,6 +34,7 @@
 #include "activation_fused.cuh"
 #include "gemm_prefill_pair.cuh"
 #include "gemm_decode.cuh"
+#include "gemm_int4.cuh"
 
 namespace {
 
@@ -148,6 +149,8 @@ i8r_status device_setup(const DeviceInfo **out) {
             if (d.pair_clusters < 1) return I8R_EARCH;
             I8R_CUDA(cudaFuncSetAttribute(decode::gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(decode::SMEM_BUDGET + 4096)));
+            I8R_CUDA(cudaFuncSetAttribute(w4::gemm_int4_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(w4::SMEM_BUDGET + 4096)));
             I8R_CUDA(cudaFuncSetAttribute(activation_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(kFusedSmemMax)));
             int per_sm = 0;
@@ -558,6 +561,27 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     return I8R_OK;
 }
 
+// The group-wise 4-bit codec: shape rules and the product's workspace.
+i8r_status check_int4_shape(int K, int N) {
+    if (K < 0 || N < 0) return I8R_EINVAL;
+    if (K < w4::BK || N < 16) return I8R_ERANGE;
+    if (K % w4::BK || N % 16) return I8R_EALIGN;
+    return I8R_OK;
+}
+
+struct Int4Workspace {
+    size_t part, counters, total;
+};
+
+Int4Workspace int4_ws_layout(int T, int N) {
+    Int4Workspace w{};
+    const int TP = (T + 15) / 16 * 16;
+    w.part = 0;
+    w.counters = align_up(static_cast<size_t>(w4::MAX_CTAS) * 2 * TP * w4::BN * 4);
+    w.total = align_up(w.counters + static_cast<size_t>(w4::padded_n(N) / w4::BN) * 4 * 4);
+    return w;
+}
+
 __global__ void wait_timeout_selftest_kernel(uint64_t limit_ns) {
     __shared__ uint64_t bar;
     __shared__ int abort_flag;
@@ -856,6 +880,102 @@ i8r_status int8_gemm_i8_s32(const int8_t *Xq, int T, int K, const int8_t *Wq, in
     zero_kernel<<<dev->sms * 4, 256, 0, stream>>>(reinterpret_cast<int4 *>(acc), n16);
     I8R_LAUNCHED();
     return launch_decode(dev, Xq, T, K, Wq, N, acc, nullptr, stream);
+}
+
+size_t int4_packed_code_bytes(int K, int N) {
+    if (check_int4_shape(K, N) != I8R_OK) return 0;
+    return w4::code_bytes(K, N);
+}
+
+size_t int4_packed_scale_bytes(int K, int N) {
+    if (check_int4_shape(K, N) != I8R_OK) return 0;
+    return w4::scale_bytes(K, N);
+}
+
+i8r_status int4_quantize_weight_groupwise(const void *W16, int K, int N, uint8_t *W4, void *S4, cudaStream_t stream) {
+    I8R_TRY(check_int4_shape(K, N));
+    I8R_TRY(check_ptr(W16));
+    I8R_TRY(check_ptr(W4));
+    I8R_TRY(check_ptr(S4));
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+    const dim3 grid(static_cast<unsigned>(w4::padded_n(N) / 256), static_cast<unsigned>(K / w4::G));
+    w4::int4_pack_kernel<<<grid, 256, 0, stream>>>(static_cast<const __half *>(W16), K, N, W4,
+                                                     static_cast<uint8_t *>(S4));
+    I8R_LAUNCHED();
+    return I8R_OK;
+}
+
+i8r_status int4_dequantize_weight(const uint8_t *W4, const void *S4, int K, int N, void *W16d, cudaStream_t stream) {
+    I8R_TRY(check_int4_shape(K, N));
+    I8R_TRY(check_ptr(W4));
+    I8R_TRY(check_ptr(S4));
+    I8R_TRY(check_ptr(W16d));
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+    const dim3 grid(static_cast<unsigned>((N + 255) / 256), static_cast<unsigned>(K / w4::G));
+    w4::int4_unpack_kernel<<<grid, 256, 0, stream>>>(W4, static_cast<const uint8_t *>(S4), K, N,
+                                                       static_cast<__half *>(W16d));
+    I8R_LAUNCHED();
+    return I8R_OK;
+}
+
+size_t int4_linear_workspace_size(int T, int K, int N) {
+    if (T < 0 || T > w4::MAX_T || check_int4_shape(K, N) != I8R_OK) return 0;
+    return int4_ws_layout(T, N).total;
+}
+
+i8r_status int4_linear(const void *X, int T, int K, const uint8_t *W4, const void *S4, int N, void *Y,
+                       void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    I8R_TRY(check_int4_shape(K, N));
+    if (T < 0) return I8R_EINVAL;
+    if (T > w4::MAX_T) return I8R_ERANGE;
+    if (T == 0) return I8R_OK;
+    I8R_TRY(check_ptr(X));
+    I8R_TRY(check_ptr(W4));
+    I8R_TRY(check_ptr(S4));
+    I8R_TRY(check_ptr(Y));
+    const Int4Workspace w = int4_ws_layout(T, N);
+    if (!workspace || workspace_bytes < w.total) return I8R_EWORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return I8R_EALIGN;
+    const DeviceInfo *dev = nullptr;
+    I8R_TRY(device_setup(&dev));
+
+    w4::Params p{};
+    p.T = T;
+    p.TP = (T + 15) / 16 * 16;
+    p.K = K;
+    p.N = N;
+    p.KB = K / w4::BK;
+    p.num_tiles = w4::padded_n(N) / w4::BN;
+    p.total_units = static_cast<long long>(p.num_tiles) * p.KB;
+    p.stage_bytes = w4::CODE_BYTES + w4::SCALE_BYTES + 4 * p.TP * 128;
+    p.stages = static_cast<int>(w4::SMEM_BUDGET / p.stage_bytes);
+    if (p.stages > w4::MAX_STAGES) p.stages = w4::MAX_STAGES;
+    p.na = (w4::MAX_NA * w4::KSUB + 4 * p.TP <= static_cast<int>(w4::TMEM_COLS)) ? w4::MAX_NA : 2;
+    p.W4 = W4;
+    p.S4 = static_cast<const uint8_t *>(S4);
+    p.Y = static_cast<__half *>(Y);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    p.part = reinterpret_cast<float *>(ws + w.part);
+    p.counters = reinterpret_cast<int *>(ws + w.counters);
+    CUtensorMap map_x;
+    I8R_TRY(make_map(&map_x, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, p.TP, 64));
+    const int ncount = p.num_tiles * 4;
+    w4::int4_clear_kernel<<<(ncount + 255) / 256, 256, 0, stream>>>(p.counters, ncount);
+    I8R_LAUNCHED();
+    const long long g = std::min<long long>(p.total_units, std::min(dev->sms, w4::MAX_CTAS));
+    record_before(stream);
+    cudaError_t e = launch_dependent(w4::gemm_int4_decode_kernel, dim3(static_cast<unsigned>(g)),
+                                     dim3(w4::THREADS), w4::smem_bytes(p.stages, p.stage_bytes), stream, 1,
+                                     map_x, p);
+    if (e != cudaSuccess) {
+        tl_last_cuda_error = static_cast<int>(e);
+        return I8R_ECUDA;
+    }
+    I8R_LAUNCHED();
+    record_after(stream);
+    return I8R_OK;
 }
 
 i8r_status int8_read_and_clear_device_status(int *code, cudaStream_t stream) {

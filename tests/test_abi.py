@@ -23,7 +23,7 @@ def so():
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(int8_\w+)\s*\(", text, flags=re.M)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(int[48]_\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
 
 
@@ -31,7 +31,9 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for required in ("int8_quantize_weight_colwise", "int8_mixed_linear", "int8_outlier_stats",
                      "int8_mixed_linear_workspace_size", "int8_quantize_activation", "int8_gemm_i8_s32",
-                     "int8_read_and_clear_device_status", "int8_status_string"):
+                     "int8_read_and_clear_device_status", "int8_status_string",
+                     "int4_quantize_weight_groupwise", "int4_dequantize_weight", "int4_linear",
+                     "int4_linear_workspace_size", "int4_packed_code_bytes", "int4_packed_scale_bytes"):
         assert required in names
 
 
@@ -181,3 +183,29 @@ def test_int8_weights_take_half_the_bytes():
     for K, N in ((5120, 20480), (12288, 49152), (49152, 12288)):
         ratio = (K * N + 4 * N) / (2 * K * N)
         assert 0.5 < ratio <= 0.5 + 2.0 / K + 1e-15
+
+
+def test_int4_host_rejections(so):
+    """The 4-bit entry points check shapes, pointers and workspace on the host."""
+    P = ctypes.c_void_p
+    so.int4_linear.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, ctypes.c_int, P, P, ctypes.c_size_t, P]
+    so.int4_linear_workspace_size.argtypes = [ctypes.c_int] * 3
+    so.int4_linear_workspace_size.restype = ctypes.c_size_t
+    so.int4_packed_code_bytes.argtypes = [ctypes.c_int] * 2
+    so.int4_packed_code_bytes.restype = ctypes.c_size_t
+    so.int4_quantize_weight_groupwise.argtypes = [P, ctypes.c_int, ctypes.c_int, P, P, P]
+    ws = so.int4_linear_workspace_size(16, 1024, 1024)
+    assert ws > 0
+    assert so.int4_linear_workspace_size(65, 1024, 1024) == 0           # T > 64
+    assert so.int4_linear_workspace_size(16, 1000, 1024) == 0           # K not a multiple of 256
+    assert so.int4_packed_code_bytes(1024, 1000) == 0                   # N not a multiple of 16
+    assert so.int4_packed_code_bytes(512, 300 * 16) == 512 * 4864 // 2  # 4800 columns padded to 19 x 256
+    a = _p()
+    assert so.int4_linear(a, 16, 1000, a, a, 1024, a, a, ws, None) == 2         # I8R_EALIGN
+    assert so.int4_linear(a, 65, 1024, a, a, 1024, a, a, ws, None) == 3         # I8R_ERANGE
+    assert so.int4_linear(a, -1, 1024, a, a, 1024, a, a, ws, None) == 1         # I8R_EINVAL
+    assert so.int4_linear(_null(), 16, 1024, a, a, 1024, a, a, ws, None) == 1   # null X
+    assert so.int4_linear(_p(4097), 16, 1024, a, a, 1024, a, a, ws, None) == 2  # misaligned X
+    assert so.int4_linear(a, 16, 1024, a, a, 1024, a, a, ws - 1, None) == 4     # workspace too small
+    assert so.int4_linear(a, 0, 1024, a, a, 1024, a, a, 0, None) == 0           # T = 0: no-op
+    assert so.int4_quantize_weight_groupwise(a, 128, 1024, a, a, None) == 3    # K < 256

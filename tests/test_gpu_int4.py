@@ -1,0 +1,131 @@
+"""The group-wise 4-bit weight codec and its decode-shaped product against the
+oracle (GPU).
+
+Bit-exact: the codes, the binary16 step s and base lo of every group (read
+back through the packed layout of include/int8row.h), and the decoded weight.
+Tolerance on Y (the same bound as the int8 layer: relative L2 <= 1e-3, max
+abs <= 2^-8 max|Y_oracle|): the oracle sums in double, the kernel in fp32.
+Shapes span several 256-column tiles, tiles split over several CTAs, ragged
+column counts (padding), T from 1 to the limit of 64, and groups that are
+constant, all zero or hold signed zeros.
+"""
+import numpy as np
+import pytest
+import torch
+
+import int8_quantized_row_b200 as i8
+import int4_layout as L
+from gpu_helpers import assert_y_close, device_status_clean, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+def _weights(rng, K, N, sigma=0.02):
+    W = (rng.standard_normal((K, N)) * sigma).astype(np.float16)
+    W[0:64, 0] = np.float16(0.5)                         # a constant group: s = 0
+    W[64:128, 1] = 0                                     # an all-zero group
+    W[0:64, 2] = np.where(np.arange(64) % 2 == 0, np.float16(0.0), np.float16(-0.0))   # signed zeros
+    W[128:192, 3] = (rng.standard_normal(64) * 40).astype(np.float16)                 # a wide group
+    return W
+
+
+@pytest.mark.parametrize("K,N", [(256, 16), (512, 272), (1024, 1024), (12288, 768)])
+def test_int4_codec_bit_exact(orc, K, N):
+    rng = np.random.default_rng(K + N)
+    W = _weights(rng, K, N)
+    codes_o, s_o, lo_o = orc.int4_quantize_groupwise(W)
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev(W))
+    torch.cuda.synchronize()
+    W4h, S4h = to_host(W4), to_host(S4)
+    codes, s, lo = L.unpack(W4h, S4h, K, N)
+    assert np.array_equal(codes, codes_o)
+    assert np.array_equal(s.view(np.uint16), s_o.view(np.uint16))
+    assert np.array_equal(lo.view(np.uint16), lo_o.view(np.uint16))
+    # padding columns are zero codes and zero (s, lo)
+    pw, ps = L.pack(codes_o, s_o, lo_o)
+    assert np.array_equal(W4h, pw) and np.array_equal(S4h, ps)
+    Wd = to_host(i8.int4_dequantize_weight(W4, S4, K, N))
+    Wd_o = orc.int4_dequantize(codes_o, s_o, lo_o)
+    assert np.array_equal(Wd.view(np.uint16), Wd_o.view(np.uint16))
+    assert device_status_clean()
+
+
+def test_int4_codec_every_fp16_value(orc):
+    """Every finite fp16 value passes through the codec (in groups of 64)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16).view(np.float16)
+    vals = bits[np.isfinite(bits)]
+    N = 64
+    K = (len(vals) + N - 1) // N // 256 * 256 + 256
+    W = np.zeros(K * N, np.float16)
+    W[:len(vals)] = vals
+    W = W.reshape(K, N)
+    codes_o, s_o, lo_o = orc.int4_quantize_groupwise(W)
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev(W))
+    codes, s, lo = L.unpack(to_host(W4), to_host(S4), K, N)
+    assert np.array_equal(codes, codes_o)
+    assert np.array_equal(s.view(np.uint16), s_o.view(np.uint16))
+    assert np.array_equal(lo.view(np.uint16), lo_o.view(np.uint16))
+    Wd = to_host(i8.int4_dequantize_weight(W4, S4, K, N))
+    assert np.array_equal(Wd.view(np.uint16), orc.int4_dequantize(codes_o, s_o, lo_o).view(np.uint16))
+
+
+LINEAR_CASES = [
+    # T, K, N
+    (1, 256, 16),
+    (3, 512, 272),          # ragged N: one padded tile
+    (16, 1024, 1024),
+    (17, 2048, 528),
+    (64, 1024, 256),        # the largest T
+    (8, 12288, 2048),       # tiles split over several CTAs
+    (1, 4096, 12288),
+    (33, 4096, 4096),
+]
+
+
+@pytest.mark.parametrize("T,K,N", LINEAR_CASES)
+def test_int4_linear_matches_oracle(orc, T, K, N):
+    rng = np.random.default_rng(T * 31 + K + N)
+    X = rng.standard_normal((T, K)).astype(np.float16)
+    W = _weights(rng, K, N)
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev(W))
+    Y = to_host(i8.int4_linear(to_dev(X), W4, S4, N))
+    codes_o, s_o, lo_o = orc.int4_quantize_groupwise(W)
+    Y_o, _ = orc.int4_linear(X, codes_o, s_o, lo_o)
+    assert_y_close(Y, Y_o, f"int4 T={T} K={K} N={N}")
+    assert device_status_clean()
+
+
+def test_int4_linear_exact_integers(orc):
+    """Integer activations and weights on exact 4-bit grids: every product and
+    partial sum is exact in fp32, so Y is the exact integer product."""
+    rng = np.random.default_rng(7)
+    T, K, N = 16, 1024, 512
+    Q = rng.integers(0, 16, (K, N))
+    Q[0::64] = 0
+    Q[1::64] = 15
+    W = (Q - 7).astype(np.float16)                       # s = 1, lo = -7 in every group
+    X = rng.integers(-2, 3, (T, K)).astype(np.float16)
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev(W))
+    Y = to_host(i8.int4_linear(to_dev(X), W4, S4, N)).astype(np.int64)
+    exact = X.astype(np.int64) @ (Q - 7)
+    assert np.abs(exact).max() <= 2048
+    assert np.array_equal(Y, exact)
+
+
+def test_int4_linear_is_deterministic():
+    rng = np.random.default_rng(11)
+    T, K, N = 16, 12288, 4096
+    X = to_dev(rng.standard_normal((T, K)).astype(np.float16))
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev((rng.standard_normal((K, N)) * 0.01).astype(np.float16)))
+    a = to_host(i8.int4_linear(X, W4, S4, N))
+    b = to_host(i8.int4_linear(X, W4, S4, N))
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
+def test_int4_linear_t0_and_limits():
+    W4 = torch.zeros(i8.int4_packed_code_bytes(256, 16), dtype=torch.uint8, device="cuda")
+    S4 = torch.zeros(i8.int4_packed_scale_bytes(256, 16), dtype=torch.uint8, device="cuda")
+    Y = i8.int4_linear(torch.zeros((0, 256), dtype=torch.float16, device="cuda"), W4, S4, 16)
+    assert Y.shape == (0, 16)
+    with pytest.raises(i8.I8RError):
+        i8.int4_linear(torch.zeros((65, 256), dtype=torch.float16, device="cuda"), W4, S4, 16)

@@ -62,6 +62,14 @@ constexpr int MAX_BUF = 4;         // TMEM accumulator buffers: the MMA runs up 
                                    // ahead of a finalising epilogue
 constexpr size_t SMEM_BUDGET = 200 * 1024;
 static_assert(4 * O_CHUNK == A_BYTES, "an outlier stage's W16 rows fill the weight slot");
+// Batches above this many rows hand their partial sums to acc32 as bulk
+// tensor reduce-adds (in L2) and leave Y to decode_finalize_kernel; smaller
+// batches finalise in the GEMM's last piece of each tile.
+constexpr int BULK_MIN_T = 65;
+constexpr int RED_ROWS = 32;                       // rows per bulk reduce (a 32 x 32 int32 box, 4 KB)
+constexpr int RED_BYTES = RED_ROWS * 32 * 4;
+constexpr int RED_SMEM = 4 * 2 * RED_BYTES;        // two staging boxes per epilogue warp
+constexpr size_t SMEM_MAX = 227 * 1024;
 
 struct Params {
     int T, TP, K, N;
@@ -82,6 +90,7 @@ struct Params {
     int o_rows;                    // Wq-only variant: rows of the compacted, dequantised W16o
     int wq_only;                   // no W16: outlier rows come from W16o (zeros past o_rows)
     int may_outlier;               // alpha < +inf: a tile's first stage may be an outlier stage
+    int bulk;                      // partial sums go to acc32 by bulk reduce-adds (T >= BULK_MIN_T)
     __half *Y;
     float *Yo;                     // [T,N] fp32: the 16-bit outlier part (written when |O| > 0)
 };
@@ -97,10 +106,14 @@ struct Barriers {
 };
 
 // The ring (stages x stage_bytes; an outlier stage, 64 W16 rows of a tile and
-// T x 64 fp16 of Xo, has the size of a weight stage), then the barriers;
-// 1024 bytes for aligning the base to the 128-byte swizzle's 1024-byte period.
-__host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes) {
-    return 1024 + static_cast<size_t>(stages) * stage_bytes + sizeof(Barriers);
+// T x 64 fp16 of Xo, has the size of a weight stage), then the barriers, then
+// (bulk mode) the epilogue warps' reduce staging boxes; 1024 bytes for aligning
+// the base to the 128-byte swizzle's 1024-byte period.
+__host__ __device__ inline size_t staging_offset(int stages, int stage_bytes) {      // from the aligned base
+    return static_cast<size_t>(stages) * stage_bytes + (sizeof(Barriers) + 127) / 128 * 128;
+}
+__host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes, int bulk) {
+    return 1024 + staging_offset(stages, stage_bytes) + (bulk ? RED_SMEM : 0);
 }
 
 // CTA c of `ctas` owns units [floor(c*U/ctas), floor((c+1)*U/ctas)).
@@ -183,10 +196,44 @@ __device__ __forceinline__ void finalize_columns(const Params &p, int tile, int 
     }
 }
 
+// Y from the reduced int32 sums (bulk mode): one thread per 8 columns of a row,
+//   Y[t,n] = fp16( acc32[t,n] * sX[t] * sW[n] / 127^2 + Yo[t,n] ),
+// the arithmetic of finalize_columns; a programmatic dependent of the GEMM.
+__global__ void __launch_bounds__(256) decode_finalize_kernel(const int32_t *__restrict__ acc32,
+                                                              const float *__restrict__ Yo,
+                                                              const int32_t *__restrict__ count,
+                                                              const float *__restrict__ sX, const float *__restrict__ sW,
+                                                              int T, int N, __half *__restrict__ Y) {
+    griddep_wait();
+    const int groups = N / 8;
+    const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (g >= static_cast<long long>(T) * groups) return;
+    const int t = static_cast<int>(g / groups), n = static_cast<int>(g % groups) * 8;
+    const bool yo = Yo && *count > 0;
+    const size_t at = static_cast<size_t>(t) * N + n;
+    const int4 a0 = __ldcg(reinterpret_cast<const int4 *>(acc32 + at));
+    const int4 a1 = __ldcg(reinterpret_cast<const int4 *>(acc32 + at + 4));
+    const float4 w0 = __ldg(reinterpret_cast<const float4 *>(sW + n));
+    const float4 w1 = __ldg(reinterpret_cast<const float4 *>(sW + n + 4));
+    float4 o0 = make_float4(0.f, 0.f, 0.f, 0.f), o1 = o0;
+    if (yo) {
+        o0 = __ldcg(reinterpret_cast<const float4 *>(Yo + at));
+        o1 = __ldcg(reinterpret_cast<const float4 *>(Yo + at + 4));
+    }
+    const float rs = sX[t] * (1.0f / 16129.0f);
+    const int av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+    const float ov[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+    __align__(16) __half y[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[e] = __float2half_rn(fmaf(static_cast<float>(av[e]), rs * wv[e], ov[e]));
+    *reinterpret_cast<uint4 *>(Y + at) = *reinterpret_cast<const uint4 *>(y);
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap map_wq, const __grid_constant__ CUtensorMap map_xq,
                        const __grid_constant__ CUtensorMap map_xo, const __grid_constant__ CUtensorMap map_w16o,
-                       const Params p) {
+                       const __grid_constant__ CUtensorMap map_acc, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Barriers *bars = reinterpret_cast<Barriers *>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);
@@ -378,6 +425,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int quad = warp & 3;
         uint32_t tph = 0;
         int seg = 0;
+        int red_n = 0;                                    // bulk reduces issued by this warp
         walk_stages(p, u0, u1, nob, [&](int kind, int tile, int, bool, bool last) -> bool {
             if (!last) return true;
             const int buf = seg % p.nbuf;
@@ -395,6 +443,43 @@ __global__ void __launch_bounds__(THREADS, 1)
             // tile's last: it writes Y from its own sums in TMEM (plus acc32 when
             // other CTAs added theirs there) and needs neither the atomic adds nor
             // the re-read.  Counted pieces were published before they were counted.
+            if (p.bulk && kind == 0) {
+                // this piece's sums into acc32: 32 x 32 boxes staged in shared
+                // memory and added in L2 by bulk tensor reduce-adds
+                uint8_t *stg = smem + staging_offset(p.stages, p.stage_bytes) + static_cast<size_t>(quad) * 2 * RED_BYTES;
+                for (int h = 0; h < 2; ++h) {
+                    const int n0 = tile * BM + h * BMH + quad * 32;
+                    for (int t0 = 0; t0 < p.T; t0 += RED_ROWS) {
+                        int32_t *box = reinterpret_cast<int32_t *>(stg + (red_n & 1) * RED_BYTES);
+                        if (red_n >= 2) {
+                            if (lane == 0) bulk_wait_group_read<1>();   // the box written two reduces ago is free
+                            __syncwarp();
+                        }
+                        uint32_t r0[16], r1[16];
+                        tmem_ld16(taddr + h * p.TP + t0, r0);
+                        tmem_ld16(taddr + h * p.TP + t0 + 16, r1);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            box[i * 32 + lane] = static_cast<int32_t>(r0[i]);
+                            box[(i + 16) * 32 + lane] = static_cast<int32_t>(r1[i]);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_reduce_add_2d(&map_acc, box, n0, t0);
+                            bulk_commit_group();
+                        }
+                        ++red_n;
+                    }
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
+                tph ^= 1u << buf;
+                ++seg;
+                return true;
+            }
             int last_piece = 0;
             if (kind == 0 && p.finalize) {
                 if (lane == 0) last_piece = atomicAdd(counter, 0) == pieces - 1;
@@ -432,7 +517,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
-                if (p.finalize) {
+                if (p.finalize && !p.bulk) {
                     // publish this warp's piece, then count it; the piece that
                     // completes the count writes Y from acc32 (and Yo)
                     __threadfence();
@@ -450,6 +535,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             ++seg;
             return true;
         });
+        if (lane == 0 && red_n > 0) bulk_wait_group_all();     // every reduce has landed in acc32
+        __syncwarp();
     }
 
     tc_fence_before_sync();

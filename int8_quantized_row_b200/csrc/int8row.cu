@@ -148,7 +148,7 @@ i8r_status device_setup(const DeviceInfo **out) {
             I8R_CUDA(cudaOccupancyMaxActiveClusters(&d.pair_clusters, prefill2::gemm_prefill_pair_kernel<false>, &cfg));
             if (d.pair_clusters < 1) return I8R_EARCH;
             I8R_CUDA(cudaFuncSetAttribute(decode::gemm_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          static_cast<int>(decode::SMEM_BUDGET + 4096)));
+                                          static_cast<int>(decode::SMEM_MAX)));
             I8R_CUDA(cudaFuncSetAttribute(w4::gemm_int4_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(w4::SMEM_BUDGET + 4096)));
             I8R_CUDA(cudaFuncSetAttribute(activation_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -527,7 +527,11 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.num_tiles = (N + decode::BM - 1) / decode::BM;
     p.total_units = static_cast<long long>(p.num_tiles) * p.KB;
     p.stage_bytes = decode::A_BYTES + p.TP * decode::BK;
-    p.stages = static_cast<int>(decode::SMEM_BUDGET / p.stage_bytes);
+    // batches of BULK_MIN_T rows and more reduce their partial sums in bulk
+    // (staging boxes in shared memory); Y is then written by decode_finalize_kernel
+    p.bulk = T >= decode::BULK_MIN_T ? 1 : 0;
+    const size_t ring = p.bulk ? decode::SMEM_MAX - decode::smem_bytes(0, 0, 1) : decode::SMEM_BUDGET;
+    p.stages = static_cast<int>(ring / p.stage_bytes);
     if (p.stages > decode::MAX_STAGES) p.stages = decode::MAX_STAGES;
     p.may_outlier = (fin && fin->may_outlier) ? 1 : 0;
     uint32_t cols = 32;
@@ -536,28 +540,44 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.nbuf = cols * decode::MAX_BUF <= 512 ? decode::MAX_BUF : 2;
     p.tmem_cols = cols * static_cast<uint32_t>(p.nbuf);
     p.acc32 = acc32;
-    CUtensorMap map_wq, map_xq, map_xo, map_w16o;
+    CUtensorMap map_wq, map_xq, map_xo, map_w16o, map_acc;
     // Two 128-column boxes per stage cover 256 contiguous bytes of every weight
     // row, so the 256-byte L2 line is used whole.
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BMH));
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, p.TP, decode::BK));
-    map_xo = map_w16o = map_xq;   // unused without a 16-bit part
+    map_xo = map_w16o = map_acc = map_xq;   // unused without a 16-bit part / in atomic mode
+    if (p.bulk) {
+        // acc32 [T, N] int32 in 32 x 32 boxes, unswizzled 128-byte rows
+        I8R_TRY(make_map(&map_acc, acc32, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, T, N, decode::RED_ROWS, 32,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
+    }
     p.W16 = W16;
     if (fin && Xo) {
         I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, p.TP, decode::OBK));
         if (W16o) I8R_TRY(make_map(&map_w16o, W16o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.o_rows, N, 64, 64));
     }
     const long long g = p.total_units < dev->sms ? p.total_units : dev->sms;
-    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes);
+    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes, p.bulk);
     record_before(s);
     cudaError_t e = launch_dependent(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(g)),
-                                     dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, map_xo, map_w16o, p);
+                                     dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, map_xo, map_w16o, map_acc, p);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;
     }
     I8R_LAUNCHED();
     record_after(s);
+    if (p.bulk && fin) {
+        const long long items = static_cast<long long>(T) * (N / 8);
+        e = launch_dependent(decode::decode_finalize_kernel, dim3(static_cast<unsigned>((items + 255) / 256)), dim3(256),
+                             0, s, 1, static_cast<const int32_t *>(acc32), static_cast<const float *>(fin->Yo),
+                             fin->count, fin->sX, fin->sW, T, N, fin->Y);
+        if (e != cudaSuccess) {
+            tl_last_cuda_error = static_cast<int>(e);
+            return I8R_ECUDA;
+        }
+        I8R_LAUNCHED();
+    }
     return I8R_OK;
 }
 

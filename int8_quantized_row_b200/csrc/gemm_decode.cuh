@@ -87,7 +87,7 @@ struct Params {
     const int32_t *count;          // |O|
     const int32_t *idx;            // the outlier columns, ascending
     const __half *W16;             // [K,N] fp16 (null for the Wq-only variant)
-    int o_rows;                    // Wq-only variant: rows of the compacted, dequantised W16o
+    int o_rows;                    // rows of the compacted outlier rows W16o (W16 rows, or dequantised Wq rows)
     int wq_only;                   // no W16: outlier rows come from W16o (zeros past o_rows)
     int may_outlier;               // alpha < +inf: a tile's first stage may be an outlier stage
     int bulk;                      // partial sums go to acc32 by bulk reduce-adds (T >= BULK_MIN_T)
@@ -233,7 +233,8 @@ __global__ void __launch_bounds__(256) decode_finalize_kernel(const int32_t *__r
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_decode_kernel(const __grid_constant__ CUtensorMap map_wq, const __grid_constant__ CUtensorMap map_xq,
                        const __grid_constant__ CUtensorMap map_xo, const __grid_constant__ CUtensorMap map_w16o,
-                       const __grid_constant__ CUtensorMap map_acc, const Params p) {
+                       const __grid_constant__ CUtensorMap map_acc, const __grid_constant__ CUtensorMap map_yo,
+                       const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Barriers *bars = reinterpret_cast<Barriers *>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (nob > 0 && lane == 0) {
-            if (p.wq_only) tma_prefetch_map(&map_w16o);
+            if (p.o_rows > 0) tma_prefetch_map(&map_w16o);
             tma_prefetch_map(&map_xo);
         }
         int pending[MAX_STAGES];
@@ -314,9 +315,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tma_load_2d(a + A_HALF, &map_wq, fb, tile * BM + BMH, j * BK);
                         tma_load_2d(a + A_BYTES, &map_xq, fb, j * BK, 0);
                     }
-                } else if (p.wq_only) {
-                    // compacted dequantised rows; past o_rows an out-of-range box, i.e.
-                    // zeros (the quantiser reports the overflow)
+                } else if (p.wq_only || (j + 1) * OBK <= p.o_rows) {
+                    // compacted rows (W16 rows, or dequantised Wq rows): four 64 x 64
+                    // boxes; for the Wq-only variant past o_rows an out-of-range box,
+                    // i.e. zeros (the quantiser reports the overflow)
                     if (lane == 0) {
                         const int y = (j + 1) * OBK <= p.o_rows ? j * OBK : p.o_rows;
                         mbar_arrive_expect_tx(fb, tx);
@@ -443,9 +445,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             // tile's last: it writes Y from its own sums in TMEM (plus acc32 when
             // other CTAs added theirs there) and needs neither the atomic adds nor
             // the re-read.  Counted pieces were published before they were counted.
-            if (p.bulk && kind == 0) {
-                // this piece's sums into acc32: 32 x 32 boxes staged in shared
-                // memory and added in L2 by bulk tensor reduce-adds
+            if (p.bulk) {
+                // this piece's int32 sums into acc32 (32 x 32 boxes staged in shared
+                // memory, added in L2 by bulk tensor reduce-adds), or the tile's
+                // outlier part into Yo (the same boxes, bulk tensor stores)
                 uint8_t *stg = smem + staging_offset(p.stages, p.stage_bytes) + static_cast<size_t>(quad) * 2 * RED_BYTES;
                 for (int h = 0; h < 2; ++h) {
                     const int n0 = tile * BM + h * BMH + quad * 32;
@@ -467,7 +470,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                         fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            tma_reduce_add_2d(&map_acc, box, n0, t0);
+                            if (kind == 0)
+                                tma_reduce_add_2d(&map_acc, box, n0, t0);
+                            else
+                                tma_store_2d(&map_yo, box, n0, t0);
                             bulk_commit_group();
                         }
                         ++red_n;

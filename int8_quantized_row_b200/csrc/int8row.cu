@@ -238,7 +238,21 @@ inline int compact_rows(int K, bool wq_only = false) {
     return std::min(all, std::max(kCompactOutlierRows, ((K + 15) / 16 + 63) / 64 * 64));
 }
 
-Workspace ws_layout(int T, int K, int N, bool wq_only = false) {
+// Rows of compacted outlier rows a call uses: the Wq-only variant's (above);
+// the prefill GEMM's 256; and at decode sizes at least 256 and K/64 (rounded
+// up to 64; 1.6 % of the columns), since there every row the GEMM gathers
+// itself costs the tile's first CTA a slow stage.
+inline int outlier_rows(int T, int K, bool wq_only) {
+    if (wq_only || T > decode::MAX_T) return compact_rows(K, wq_only);
+    const int all = (K + 63) / 64 * 64;
+    return std::min(all, std::max(kCompactOutlierRows, ((K + 63) / 64 + 63) / 64 * 64));
+}
+
+// compact_decode: decode-sized calls with W16 also compact the first
+// outlier_rows(T, K) outlier rows of W16 (the GEMM then loads them as tiles);
+// without it (the allocation-free entry point's smaller scratch) the decode
+// GEMM gathers every outlier row from W16 itself.
+Workspace ws_layout(int T, int K, int N, bool wq_only = false, bool compact_decode = true) {
     Workspace w{};
     size_t off = 0;
     w.count = off; off = align_up(off + sizeof(int32_t));
@@ -249,7 +263,8 @@ Workspace ws_layout(int T, int K, int N, bool wq_only = false) {
     w.Xq = off;    off = align_up(off + static_cast<size_t>(T) * K);
     w.Xo = off;    off = align_up(off + static_cast<size_t>(T) * K * 2);
     w.W16o = off;
-    if (T > decode::MAX_T || wq_only) off = align_up(off + static_cast<size_t>(compact_rows(K, wq_only)) * N * 2);
+    if (T > decode::MAX_T || wq_only || compact_decode)
+        off = align_up(off + static_cast<size_t>(outlier_rows(T, K, wq_only)) * N * 2);
     w.Yo = off;
     if (T <= decode::MAX_T) off = align_up(off + static_cast<size_t>(T) * N * 4);   // fp32 outlier part
     w.acc32 = off;
@@ -331,8 +346,8 @@ dim3 scan_grid(int T, int K, int sms, int *rows_per_block) {
 // a1-a3 on the stream: mask, row quantisation, index list and gather.
 // `zero` / `zero_bytes`: a region the scan clears on the way (may be null).
 // With W16o, the quantiser's launch also compacts the W16 rows of the first
-// compact_rows(K) outlier columns into W16o ([compact_rows(K), N]); with W16
-// null (the Wq-only variant) it dequantises those rows of Wq instead.
+// outlier_rows(T, K) outlier columns into W16o ([outlier_rows(T, K), N]); with
+// W16 null (the Wq-only variant) it dequantises those rows of Wq instead.
 i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int K, float alpha, uint32_t *mask,
                              int32_t *idx, int32_t *count, float *sX, int8_t *Xq, __half *Xo, void *zero,
                              size_t zero_bytes, cudaStream_t s, const __half *W16 = nullptr, int N = 0,
@@ -353,7 +368,7 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords, fused ? grid_ctr : nullptr);
     I8R_LAUNCHED();
     if (fused) {
-        const int o_rows = W16o ? compact_rows(K, W16 == nullptr) : 0;
+        const int o_rows = W16o ? outlier_rows(T, K, W16 == nullptr) : 0;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(fG));
         cfg.blockDim = dim3(kFusedThreads);
@@ -404,7 +419,7 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     I8R_LAUNCHED();
     // row 0's block of the quantiser publishes the index list and |O|
     const int rt = row_threads(K);
-    const int o_rows = W16o ? compact_rows(K, W16 == nullptr) : 0;
+    const int o_rows = W16o ? outlier_rows(T, K, W16 == nullptr) : 0;
     const int G = W16o ? std::min(o_rows, 128) : 0;     // compaction blocks
     const size_t smem = quantize_smem_bytes(K);
     const uint32_t *m = mask;
@@ -540,16 +555,19 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.nbuf = cols * decode::MAX_BUF <= 512 ? decode::MAX_BUF : 2;
     p.tmem_cols = cols * static_cast<uint32_t>(p.nbuf);
     p.acc32 = acc32;
-    CUtensorMap map_wq, map_xq, map_xo, map_w16o, map_acc;
+    CUtensorMap map_wq, map_xq, map_xo, map_w16o, map_acc, map_yo;
     // Two 128-column boxes per stage cover 256 contiguous bytes of every weight
     // row, so the 256-byte L2 line is used whole.
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BMH));
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, p.TP, decode::BK));
-    map_xo = map_w16o = map_acc = map_xq;   // unused without a 16-bit part / in atomic mode
+    map_xo = map_w16o = map_acc = map_yo = map_xq;   // unused without a 16-bit part / in atomic mode
     if (p.bulk) {
         // acc32 [T, N] int32 in 32 x 32 boxes, unswizzled 128-byte rows
         I8R_TRY(make_map(&map_acc, acc32, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, T, N, decode::RED_ROWS, 32,
                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
+        if (fin && fin->Yo)
+            I8R_TRY(make_map(&map_yo, fin->Yo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, N, decode::RED_ROWS, 32,
+                             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
     }
     p.W16 = W16;
     if (fin && Xo) {
@@ -560,7 +578,8 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes, p.bulk);
     record_before(s);
     cudaError_t e = launch_dependent(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(g)),
-                                     dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, map_xo, map_w16o, map_acc, p);
+                                     dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, map_xo, map_w16o, map_acc, map_yo,
+                                     p);
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;
@@ -685,7 +704,8 @@ namespace {
 
 // int8_mixed_linear and its Wq-only variant (W16 null).
 i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, const float *sW, const void *W16, int N,
-                             float alpha, void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+                             float alpha, void *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream,
+                             bool compact_decode = true) {
     const bool wq_only = W16 == nullptr;
     I8R_TRY(check_shape(T, K, N, true));
     if (std::isnan(alpha) || alpha < 0.0f) return I8R_EINVAL;
@@ -695,7 +715,7 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     I8R_TRY(check_ptr(sW));
     if (!wq_only) I8R_TRY(check_ptr(W16));
     I8R_TRY(check_ptr(Y));
-    const Workspace w = ws_layout(T, K, N, wq_only);
+    const Workspace w = ws_layout(T, K, N, wq_only, compact_decode);
     if (!workspace || workspace_bytes < w.total) return I8R_EWORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return I8R_EALIGN;
     const DeviceInfo *dev = nullptr;
@@ -718,10 +738,10 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
 
     // decode: the outlier scan clears the split-K accumulator and the tile counters
     const size_t zero_bytes = small_t ? w.total - w.acc32 : 0;
-    // compacted outlier rows: the prefill GEMM's first compact_rows(K), and the
-    // Wq-only variant's dequantised rows at every T (the decode GEMM gathers W16
-    // rows itself)
-    __half *W16o = (small_t && !wq_only) ? nullptr : reinterpret_cast<__half *>(ws + w.W16o);
+    // compacted outlier rows: the first outlier_rows(T, K) rows of W16 (the GEMMs
+    // gather any further rows from W16 themselves), or the Wq-only variant's
+    // dequantised rows
+    __half *W16o = (small_t && !wq_only && !compact_decode) ? nullptr : reinterpret_cast<__half *>(ws + w.W16o);
     I8R_TRY(launch_activation(dev, x, T, K, alpha, mask, idx, count, sX, Xq, Xo, small_t ? acc32 : nullptr,
                               zero_bytes, stream, w16, N, W16o, Wq, sW, reinterpret_cast<unsigned *>(ws + w.ctr)));
     if (!small_t)
@@ -733,7 +753,7 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     fin.sW = sW;
     fin.count = count;
     fin.idx = idx;
-    fin.o_rows = wq_only ? compact_rows(K, true) : 0;
+    fin.o_rows = (wq_only || compact_decode) ? outlier_rows(T, K, wq_only) : 0;
     fin.wq_only = wq_only ? 1 : 0;
     fin.may_outlier = std::isinf(alpha) ? 0 : 1;   // alpha = +inf: no finite input is an outlier
     fin.Y = y;
@@ -804,12 +824,15 @@ void int8_debug_set_activation_path(int mode) { g_activation_fused.store(mode < 
 i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K, const int8_t *Wq, const float *sW,
                                      const void *W16, int N, float alpha, void *Y, cudaStream_t stream) {
     I8R_TRY(check_shape(T, K, N, true));
-    if (ws_layout(T, K, N).total > kNoAllocScratchBytes) return I8R_ERANGE;
+    // the fixed scratch holds no compacted outlier rows at decode sizes: the
+    // GEMM gathers them from W16 (same results, and more shapes fit)
+    if (ws_layout(T, K, N, false, false).total > kNoAllocScratchBytes) return I8R_ERANGE;
+    if (!W16) return I8R_EINVAL;
     void *scratch = nullptr;
     I8R_TRY(noalloc_scratch_address(&scratch));
     // Nothing in the scratch has to start at zero: int8_mixed_linear writes
     // every region before it reads it.
-    return int8_mixed_linear(X, T, K, Wq, sW, W16, N, alpha, Y, scratch, kNoAllocScratchBytes, stream);
+    return mixed_linear_impl(X, T, K, Wq, sW, W16, N, alpha, Y, scratch, kNoAllocScratchBytes, stream, false);
 }
 
 size_t int8_outlier_stats_workspace_size(int K) {

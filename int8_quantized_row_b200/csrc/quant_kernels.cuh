@@ -326,7 +326,8 @@ inline size_t quantize_smem_bytes(int K) { return static_cast<size_t>((K + 31) /
 // rows are dequantised instead, W16o[j,n] = fp16_rn(Wq[O_j,n] * fl32(sW[n]/127)),
 // and more than o_rows outlier columns is reported (I8R_DEV_OUTLIER_CAP).
 // Block e of the G compaction blocks copies rows e, e+G, ... with eight
-// 16-byte stores in flight per thread.
+// 16-byte stores in flight per thread, 256 ranks of the index list at a time
+// (the window held in shared memory).
 constexpr int kCompactOutlierRows = 256;
 
 template <int kThreads>
@@ -336,53 +337,64 @@ __device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *smask
                                                            int N, __half *__restrict__ W16o, int o_rows, int e, int G) {
     if (!W16 && total > o_rows && e == 0 && threadIdx.x == 0) report_status(I8R_DEV_OUTLIER_CAP);
     __shared__ int oidx[kCompactOutlierRows];
-    for (int w = w0; w < w1; ++w) {
-        int j = spre[w];
-        uint32_t m = smask[w];
-        while (m && j < o_rows) {
-            oidx[j++] = w * 32 + (__ffs(m) - 1);
-            m &= m - 1;
-        }
-    }
-    __syncthreads();
     const int rows = min((total + 15) / 16 * 16, o_rows);
     const int vec = N / 8;
     constexpr int kBatch = 8;
-    for (int r = e; r < rows; r += G) {
-        uint4 *dst = reinterpret_cast<uint4 *>(W16o + static_cast<size_t>(r) * N);
-        if (!W16) {
-            // dequantised rows: 8 codes and 8 column scales per 16-byte store
-            const uint2 *q8 = r < total ? reinterpret_cast<const uint2 *>(Wq + static_cast<size_t>(oidx[r]) * N) : nullptr;
-            for (int c = static_cast<int>(threadIdx.x); c < vec; c += kThreads) {
-                Vec16 v;
-                v.u = make_uint4(0u, 0u, 0u, 0u);
-                if (q8) {
-                    const uint2 qq = __ldg(q8 + c);
-                    const float4 s0 = __ldg(reinterpret_cast<const float4 *>(sW) + 2 * c);
-                    const float4 s1 = __ldg(reinterpret_cast<const float4 *>(sW) + 2 * c + 1);
-                    const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int q = static_cast<int8_t>(((i < 4 ? qq.x : qq.y) >> (8 * (i & 3))) & 0xFFu);
-                        v.h[i] = __float2half_rn(__fmul_rn(static_cast<float>(q), __fdiv_rn(sc[i], 127.0f)));
-                    }
-                }
-                dst[c] = v.u;
+    // outlier ranks [cb, cb + 256) at a time: that window's column indices, then its rows
+    for (int cb = 0; cb < rows; cb += kCompactOutlierRows) {
+        const int ce = cb + kCompactOutlierRows;
+        if (cb > 0) __syncthreads();                 // every row of the previous window is copied
+        for (int w = w0; w < w1; ++w) {
+            int j = spre[w];
+            uint32_t m = smask[w];
+            if (j >= ce || j + __popc(m) <= cb) continue;
+            while (m && j < ce) {
+                if (j >= cb) oidx[j - cb] = w * 32 + (__ffs(m) - 1);
+                ++j;
+                m &= m - 1;
             }
-            continue;
         }
-        const uint4 *src = r < total ? reinterpret_cast<const uint4 *>(W16 + static_cast<size_t>(oidx[r]) * N) : nullptr;
-        for (int c0 = static_cast<int>(threadIdx.x); c0 < vec; c0 += kThreads * kBatch) {
-            uint4 v[kBatch];
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-                const int c = c0 + b * kThreads;
-                v[b] = (src && c < vec) ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        __syncthreads();
+        int r0 = e;                                  // the first row of this window that block e copies
+        if (r0 < cb) r0 += (cb - e + G - 1) / G * G;
+        for (int r = r0; r < min(ce, rows); r += G) {
+            uint4 *dst = reinterpret_cast<uint4 *>(W16o + static_cast<size_t>(r) * N);
+            if (!W16) {
+                // dequantised rows: 8 codes and 8 column scales per 16-byte store
+                const uint2 *q8 = r < total ? reinterpret_cast<const uint2 *>(Wq + static_cast<size_t>(oidx[r - cb]) * N)
+                                            : nullptr;
+                for (int c = static_cast<int>(threadIdx.x); c < vec; c += kThreads) {
+                    Vec16 v;
+                    v.u = make_uint4(0u, 0u, 0u, 0u);
+                    if (q8) {
+                        const uint2 qq = __ldg(q8 + c);
+                        const float4 s0 = __ldg(reinterpret_cast<const float4 *>(sW) + 2 * c);
+                        const float4 s1 = __ldg(reinterpret_cast<const float4 *>(sW) + 2 * c + 1);
+                        const float sc[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    #pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int q = static_cast<int8_t>(((i < 4 ? qq.x : qq.y) >> (8 * (i & 3))) & 0xFFu);
+                            v.h[i] = __float2half_rn(__fmul_rn(static_cast<float>(q), __fdiv_rn(sc[i], 127.0f)));
+                        }
+                    }
+                    dst[c] = v.u;
+                }
+                continue;
             }
-#pragma unroll
-            for (int b = 0; b < kBatch; ++b) {
-                const int c = c0 + b * kThreads;
-                if (c < vec) dst[c] = v[b];
+            const uint4 *src = r < total ? reinterpret_cast<const uint4 *>(W16 + static_cast<size_t>(oidx[r - cb]) * N)
+                                         : nullptr;
+            for (int c0 = static_cast<int>(threadIdx.x); c0 < vec; c0 += kThreads * kBatch) {
+                uint4 v[kBatch];
+    #pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    const int c = c0 + b * kThreads;
+                    v[b] = (src && c < vec) ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+                }
+    #pragma unroll
+                for (int b = 0; b < kBatch; ++b) {
+                    const int c = c0 + b * kThreads;
+                    if (c < vec) dst[c] = v[b];
+                }
             }
         }
     }

@@ -316,6 +316,10 @@ DECODE_SCHEDULE_CASES = [
     (1, 4096, 12288, list(range(0, 4096, 31)), 6.0),             # |O| = 133: three outlier blocks per tile
     (128, 4096, 8192, list(range(3, 4096, 57)), 6.0),            # T = 128, three-stage ring, |O| = 72
     (64, 2048, 8192, [], 0.0),                                   # alpha = 0: 32 outlier blocks per tile
+    # more outlier columns than one 256-rank window of the row compaction:
+    (16, 12288, 4096, list(range(0, 12288, 24)), 6.0),          # |O| = 512: 256 compacted rows + 4 gathered blocks
+    (8, 49152, 1024, list(range(0, 49152, 97)), 6.0),           # |O| = 507 of 768 compacted rows (two windows)
+    (1, 16384, 2048, list(range(0, 16384, 40)), 6.0),           # |O| = 410, row quantiser's compaction blocks
 ]
 
 

@@ -9,33 +9,31 @@
 // used whole.  Split-K, stream-K style: the (tile, k-block) units are cut
 // into gridDim.x equal contiguous ranges, one per CTA, so every SM streams the
 // same number of weight bytes.  A CTA accumulates each run of k-blocks of one
-// tile in TMEM (double-buffered) and adds the exact int32 partial sums into
-// acc32 [T,N] (zeroed beforehand) with red.add.
+// tile in TMEM (up to four buffers, so the MMAs run ahead of the epilogue) and
+// adds the exact int32 partial sums into acc32 [T,N] (zeroed beforehand) with
+// bulk tensor reduce-adds from shared memory, done in L2.
 //
 // The 16-bit outlier part (LLM.int8() abstract: the outlier feature
 // dimensions go through a 16-bit matrix multiplication) runs on the same
 // tensor cores: the CTA that owns k-block 0 of a tile also runs an outlier
 // segment for it, ceil(|O|/64) stages of kind::f16 MMAs
 //   Yo[t,n] = sum_j Xo[t,j] * W16[O_j,n]      (fp32 in TMEM)
-// with A = the W16 rows of the outliers (MN-major, copied in place by the
-// lanes with cp.async, 16 bytes each, or the dequantised rows the quantiser
-// compacted for the Wq-only variant) and B = Xo (K-major), and stores it to
-// Yo [T,N].  Those stages go through the same ring as the weight stages,
-// filled by the same (only) producer warp: a parity wait cannot tell a phase
-// from the one two uses later, so every slot has one producer that waits on
-// each of its uses.  The row copies do not stall that warp: each lane hands
-// its cp.async copies to the stage's barrier (cp.async.mbarrier.arrive), so
+// with A = the W16 rows of the outliers (MN-major) and B = Xo (K-major), and
+// stores it to Yo [T,N] with bulk tensor stores.  The rows of the first
+// o_rows outliers come compacted by the activation side (W16o: W16 rows, or
+// the Wq-only variant's dequantised rows) and load as four 64 x 64 boxes; any
+// further rows are copied in place by the lanes with cp.async, 16 bytes
+// each.  Those stages go through the same ring as the weight stages, filled
+// by the same (only) producer warp: a parity wait cannot tell a phase from
+// the one two uses later, so every slot has one producer that waits on each
+// of its uses.  The row copies do not stall that warp: each lane hands its
+// cp.async copies to the stage's barrier (cp.async.mbarrier.arrive), so
 // several outlier stages can be in flight at once.
 //
-// Finalisation: after adding its partial sums (or storing its Yo piece),
-// each epilogue warp bumps a counter for its (tile, 32-lane quadrant).  The
-// warp that brings the counter to the number of contributions the tile gets
-// knows every piece has landed; it writes
+// Y is written by decode_finalize_kernel, a programmatic dependent of this
+// kernel, over the whole grid:
 //   Y[t,n] = fp16( acc32[t,n] * sX[t] * sW[n] / 127^2 + Yo[t,n] )
-// for its 64 columns.  No CTA ever waits on another.  (Stream-K leaves most
-// tiles split between the end of one CTA's range and the start of the next,
-// so these finalisations run in the kernel's tail, which is why they do no
-// more than combine two loaded values per output.)
+// so no CTA waits on another at the end of its range.
 //
 // Launched as a programmatic dependent of the activation kernels: the weight
 // tiles of the first stages are requested before griddepcontrol.wait, since
@@ -60,12 +58,11 @@ constexpr int MAX_T = 128;
 constexpr int MAX_STAGES = 8;
 constexpr int MAX_BUF = 4;         // TMEM accumulator buffers: the MMA runs up to three segments
                                    // ahead of a finalising epilogue
-constexpr size_t SMEM_BUDGET = 200 * 1024;
 static_assert(4 * O_CHUNK == A_BYTES, "an outlier stage's W16 rows fill the weight slot");
-// Batches above this many rows hand their partial sums to acc32 as bulk
-// tensor reduce-adds (in L2) and leave Y to decode_finalize_kernel; smaller
-// batches finalise in the GEMM's last piece of each tile.
-constexpr int BULK_MIN_T = 65;
+// Every piece of a tile hands its int32 partial sums to acc32 as bulk tensor
+// reduce-adds (done in L2) and decode_finalize_kernel writes Y afterwards:
+// no CTA waits on another at the end (measured faster than finalising in the
+// tile's last piece at every batch size).
 constexpr int RED_ROWS = 32;                       // rows per bulk reduce (a 32 x 32 int32 box, 4 KB)
 constexpr int RED_BYTES = RED_ROWS * 32 * 4;
 constexpr int RED_SMEM = 4 * 2 * RED_BYTES;        // two staging boxes per epilogue warp
@@ -80,9 +77,8 @@ struct Params {
     uint32_t buf_cols;             // columns of one accumulator buffer: a power of two >= 2*TP, >= 32
     int nbuf;                      // accumulator buffers (2 or 4), used in turn by the segments
     int32_t *acc32;                // [T,N] int32, zero on entry
-    // finalisation (finalize != 0): Y from acc32 (and Yo) once a tile is complete
+    // the layer (finalize != 0): the outlier segments, and Y by decode_finalize_kernel
     int finalize;
-    int32_t *counters;             // [num_tiles * 4], zero on entry
     const float *sX, *sW;
     const int32_t *count;          // |O|
     const int32_t *idx;            // the outlier columns, ascending
@@ -90,7 +86,6 @@ struct Params {
     int o_rows;                    // rows of the compacted outlier rows W16o (W16 rows, or dequantised Wq rows)
     int wq_only;                   // no W16: outlier rows come from W16o (zeros past o_rows)
     int may_outlier;               // alpha < +inf: a tile's first stage may be an outlier stage
-    int bulk;                      // partial sums go to acc32 by bulk reduce-adds (T >= BULK_MIN_T)
     __half *Y;
     float *Yo;                     // [T,N] fp32: the 16-bit outlier part (written when |O| > 0)
 };
@@ -112,8 +107,8 @@ struct Barriers {
 __host__ __device__ inline size_t staging_offset(int stages, int stage_bytes) {      // from the aligned base
     return static_cast<size_t>(stages) * stage_bytes + (sizeof(Barriers) + 127) / 128 * 128;
 }
-__host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes, int bulk) {
-    return 1024 + staging_offset(stages, stage_bytes) + (bulk ? RED_SMEM : 0);
+__host__ __device__ inline size_t smem_bytes(int stages, int stage_bytes) {
+    return 1024 + staging_offset(stages, stage_bytes) + RED_SMEM;
 }
 
 // CTA c of `ctas` owns units [floor(c*U/ctas), floor((c+1)*U/ctas)).
@@ -149,56 +144,9 @@ __device__ __forceinline__ bool walk_stages(const Params &p, long long u0, long 
     return true;
 }
 
-constexpr int FIN_ROWS = 16;
-
-// Y for the columns of one finished (tile, quadrant), both 128-column halves
-// 16 rows at a time with all their loads in flight together:
-//   Y[t,n] = fp16( (own[t,n] + acc32[t,n]) * sX[t] * sW[n] / 127^2 + Yo[t,n] )
-// own: this warp's partial sums still in TMEM (taddr, or none), acc32 read
-// only when other pieces were added there, Yo only when |O| > 0.
-__device__ __forceinline__ void finalize_columns(const Params &p, int tile, int quad, int lane, bool own,
-                                                 uint32_t taddr, bool read_acc, bool read_yo) {
-    const int n0 = tile * BM + quad * 32 + lane;
-    const bool ok0 = n0 < p.N, ok1 = n0 + BMH < p.N;
-    const float sw0 = ok0 ? p.sW[n0] : 0.0f, sw1 = ok1 ? p.sW[n0 + BMH] : 0.0f;
-    for (int t0 = 0; t0 < p.T; t0 += FIN_ROWS) {
-        uint32_t r0[FIN_ROWS], r1[FIN_ROWS];
-        if (own) {
-            tmem_ld16(taddr + t0, r0);
-            tmem_ld16(taddr + p.TP + t0, r1);
-            tmem_wait_ld();
-        } else {
-#pragma unroll
-            for (int r = 0; r < FIN_ROWS; ++r) r0[r] = r1[r] = 0u;
-        }
-        int a0[FIN_ROWS], a1[FIN_ROWS];
-        float y0[FIN_ROWS], y1[FIN_ROWS];
-#pragma unroll
-        for (int r = 0; r < FIN_ROWS; ++r) {
-            const bool row = t0 + r < p.T;
-            const size_t at = static_cast<size_t>(t0 + r) * p.N + n0;
-            a0[r] = (row && ok0 && read_acc) ? __ldcg(p.acc32 + at) : 0;
-            a1[r] = (row && ok1 && read_acc) ? __ldcg(p.acc32 + at + BMH) : 0;
-            y0[r] = (row && ok0 && read_yo) ? __ldcg(p.Yo + at) : 0.0f;
-            y1[r] = (row && ok1 && read_yo) ? __ldcg(p.Yo + at + BMH) : 0.0f;
-        }
-#pragma unroll
-        for (int r = 0; r < FIN_ROWS; ++r) {
-            const int t = t0 + r;
-            if (t >= p.T) continue;
-            const float rs = p.sX[t] * (1.0f / 16129.0f);
-            const size_t at = static_cast<size_t>(t) * p.N + n0;
-            if (ok0)
-                p.Y[at] = __float2half_rn(fmaf(static_cast<float>(static_cast<int>(r0[r]) + a0[r]), rs * sw0, y0[r]));
-            if (ok1)
-                p.Y[at + BMH] = __float2half_rn(fmaf(static_cast<float>(static_cast<int>(r1[r]) + a1[r]), rs * sw1, y1[r]));
-        }
-    }
-}
-
-// Y from the reduced int32 sums (bulk mode): one thread per 8 columns of a row,
-//   Y[t,n] = fp16( acc32[t,n] * sX[t] * sW[n] / 127^2 + Yo[t,n] ),
-// the arithmetic of finalize_columns; a programmatic dependent of the GEMM.
+// Y from the reduced int32 sums: one thread per 8 columns of a row,
+//   Y[t,n] = fp16( acc32[t,n] * (sX[t] / 127^2) * sW[n] + Yo[t,n] )
+// (one fp32 fma after the scale product); a programmatic dependent of the GEMM.
 __global__ void __launch_bounds__(256) decode_finalize_kernel(const int32_t *__restrict__ acc32,
                                                               const float *__restrict__ Yo,
                                                               const int32_t *__restrict__ count,
@@ -287,7 +235,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_load_2d(a + A_HALF, &map_wq, &bars->full[i], tile * BM + BMH, kb * BK);
         }
     }
-    griddep_wait();                               // activation, |O|, acc32 / counters zeroed
+    griddep_wait();                               // activation, |O|, acc32 zeroed
     const int count = p.finalize ? *p.count : 0;
     const int nob = p.may_outlier ? (count + OBK - 1) / OBK : 0;
 
@@ -434,109 +382,46 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!warp_wait(&bars->tmem_full[buf], (tph >> buf) & 1u, abort, I8R_DEV_TMEM_TIMEOUT)) return false;
             tc_fence_after_sync();
             const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + static_cast<uint32_t>(buf) * buf_cols;
-            // pieces of this tile: one per CTA holding some of its k-blocks, plus
-            // the outlier piece
-            const long long tile_u0 = static_cast<long long>(tile) * p.KB;
-            const int int8_pieces = unit_owner(p.total_units, tile_u0 + p.KB - 1, gridDim.x) -
-                                    unit_owner(p.total_units, tile_u0, gridDim.x) + 1;
-            const int pieces = int8_pieces + (nob > 0 ? 1 : 0);
-            int* counter = p.counters + tile * 4 + quad;
-            // An int8 piece that finds every other piece already counted is the
-            // tile's last: it writes Y from its own sums in TMEM (plus acc32 when
-            // other CTAs added theirs there) and needs neither the atomic adds nor
-            // the re-read.  Counted pieces were published before they were counted.
-            if (p.bulk) {
-                // this piece's int32 sums into acc32 (32 x 32 boxes staged in shared
-                // memory, added in L2 by bulk tensor reduce-adds), or the tile's
-                // outlier part into Yo (the same boxes, bulk tensor stores)
-                uint8_t *stg = smem + staging_offset(p.stages, p.stage_bytes) + static_cast<size_t>(quad) * 2 * RED_BYTES;
-                for (int h = 0; h < 2; ++h) {
-                    const int n0 = tile * BM + h * BMH + quad * 32;
-                    for (int t0 = 0; t0 < p.T; t0 += RED_ROWS) {
-                        int32_t *box = reinterpret_cast<int32_t *>(stg + (red_n & 1) * RED_BYTES);
-                        if (red_n >= 2) {
-                            if (lane == 0) bulk_wait_group_read<1>();   // the box written two reduces ago is free
-                            __syncwarp();
-                        }
-                        uint32_t r0[16], r1[16];
-                        tmem_ld16(taddr + h * p.TP + t0, r0);
-                        tmem_ld16(taddr + h * p.TP + t0 + 16, r1);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            box[i * 32 + lane] = static_cast<int32_t>(r0[i]);
-                            box[(i + 16) * 32 + lane] = static_cast<int32_t>(r1[i]);
-                        }
-                        fence_proxy_async_smem();
+            // This piece's int32 sums go into acc32 (32 x 32 boxes staged in shared
+            // memory, added in L2 by bulk tensor reduce-adds; exact and order-free),
+            // or the tile's outlier part into Yo (the same boxes, bulk tensor
+            // stores).  Box rows past T are not written by the bulk operations,
+            // and tensor-memory rows past TP are not read.
+            uint8_t *stg = smem + staging_offset(p.stages, p.stage_bytes) + static_cast<size_t>(quad) * 2 * RED_BYTES;
+            for (int h = 0; h < 2; ++h) {
+                const int n0 = tile * BM + h * BMH + quad * 32;
+                for (int t0 = 0; t0 < p.T; t0 += RED_ROWS) {
+                    int32_t *box = reinterpret_cast<int32_t *>(stg + (red_n & 1) * RED_BYTES);
+                    if (red_n >= 2) {
+                        if (lane == 0) bulk_wait_group_read<1>();   // the box written two bulk ops ago is free
                         __syncwarp();
-                        if (lane == 0) {
-                            if (kind == 0)
-                                tma_reduce_add_2d(&map_acc, box, n0, t0);
-                            else
-                                tma_store_2d(&map_yo, box, n0, t0);
-                            bulk_commit_group();
-                        }
-                        ++red_n;
                     }
-                }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
-                tph ^= 1u << buf;
-                ++seg;
-                return true;
-            }
-            int last_piece = 0;
-            if (kind == 0 && p.finalize) {
-                if (lane == 0) last_piece = atomicAdd(counter, 0) == pieces - 1;
-                last_piece = __shfl_sync(0xFFFFFFFFu, last_piece, 0);
-            }
-            if (last_piece) {
-                __threadfence();
-                finalize_columns(p, tile, quad, lane, true, taddr, int8_pieces > 1, nob > 0);
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
-            } else {
+                    uint32_t r0[16], r1[16];
+                    const bool second = t0 + 16 < p.TP;
+                    tmem_ld16(taddr + h * p.TP + t0, r0);
+                    if (second) tmem_ld16(taddr + h * p.TP + t0 + 16, r1);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int n = tile * BM + h * BMH + quad * 32 + lane;   // this thread's column
-                    for (int c = 0; c < p.TP; c += 16) {
-                        uint32_t r[16];
-                        tmem_ld16(taddr + h * p.TP + c, r);
-                        tmem_wait_ld();
-                        if (n < p.N) {
+                    for (int i = 0; i < 16; ++i) box[i * 32 + lane] = static_cast<int32_t>(r0[i]);
+                    if (second) {
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                const int t = c + i;
-                                if (t >= p.T) continue;
-                                const size_t at = static_cast<size_t>(t) * p.N + n;
-                                if (kind == 0) {
-                                    if (r[i] != 0u) atomicAdd(p.acc32 + at, static_cast<int>(r[i]));
-                                } else {
-                                    __stcg(p.Yo + at, __uint_as_float(r[i]));
-                                }
-                            }
-                        }
+                        for (int i = 0; i < 16; ++i) box[(i + 16) * 32 + lane] = static_cast<int32_t>(r1[i]);
                     }
-                }
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
-                if (p.finalize && !p.bulk) {
-                    // publish this warp's piece, then count it; the piece that
-                    // completes the count writes Y from acc32 (and Yo)
-                    __threadfence();
+                    fence_proxy_async_smem();
                     __syncwarp();
-                    int done = 0;
-                    if (lane == 0) done = atomicAdd(counter, 1) == pieces - 1;
-                    done = __shfl_sync(0xFFFFFFFFu, done, 0);
-                    if (done) {
-                        __threadfence();
-                        finalize_columns(p, tile, quad, lane, false, 0u, true, nob > 0);
+                    if (lane == 0) {
+                        if (kind == 0)
+                            tma_reduce_add_2d(&map_acc, box, n0, t0);
+                        else
+                            tma_store_2d(&map_yo, box, n0, t0);
+                        bulk_commit_group();
                     }
+                    ++red_n;
                 }
             }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->tmem_empty[buf]);
             tph ^= 1u << buf;
             ++seg;
             return true;

@@ -225,7 +225,7 @@ i8r_status check_ptr(const void *p) {
 
 // Workspace of int8_mixed_linear.
 struct Workspace {
-    size_t count, ctr, mask, idx, sX, Xq, Xo, W16o, Yo, acc32, counters, total;
+    size_t count, ctr, mask, idx, sX, Xq, Xo, W16o, Yo, acc32, total;
 };
 
 // Rows of the compacted outlier weight rows kept for the prefill GEMM: 256
@@ -268,14 +268,7 @@ Workspace ws_layout(int T, int K, int N, bool wq_only = false, bool compact_deco
     w.Yo = off;
     if (T <= decode::MAX_T) off = align_up(off + static_cast<size_t>(T) * N * 4);   // fp32 outlier part
     w.acc32 = off;
-    w.counters = off;
-    if (T <= decode::MAX_T) {
-        // split-K accumulator and per-(tile, quadrant) completion counters,
-        // contiguous so one pass of 16-byte stores clears both
-        off += static_cast<size_t>(T) * N * 4;
-        w.counters = off;
-        off = align_up(off + static_cast<size_t>((N + decode::BM - 1) / decode::BM) * 4 * 4);
-    }
+    if (T <= decode::MAX_T) off = align_up(off + static_cast<size_t>(T) * N * 4);   // split-K accumulator
     w.total = off;
     return w;
 }
@@ -525,10 +518,9 @@ i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half 
 }
 
 // Decode GEMM (T <= 128): int32 partial sums added into acc32, which must be
-// zero on entry.  With `fin` (non-null) the last contributor of every tile also
-// writes Y; fin->counters must be zero on entry.  With fin, |O| > 0 adds the
-// 16-bit part from Xo and the W16 rows fin->idx (or, fin->wq_only, from the
-// fin->o_rows compacted rows W16o).
+// zero on entry.  With `fin` (non-null) it also runs the 16-bit part (|O| > 0:
+// Xo times the rows of the first fin->o_rows outliers from W16o, the rest from
+// W16 by fin->idx) into fin->Yo, and decode_finalize_kernel then writes Y.
 i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, const int8_t *Wq, int N,
                          int32_t *acc32, const decode::Params *fin, cudaStream_t s, const __half *Xo = nullptr,
                          const __half *W16 = nullptr, const __half *W16o = nullptr) {
@@ -542,11 +534,8 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     p.num_tiles = (N + decode::BM - 1) / decode::BM;
     p.total_units = static_cast<long long>(p.num_tiles) * p.KB;
     p.stage_bytes = decode::A_BYTES + p.TP * decode::BK;
-    // batches of BULK_MIN_T rows and more reduce their partial sums in bulk
-    // (staging boxes in shared memory); Y is then written by decode_finalize_kernel
-    p.bulk = T >= decode::BULK_MIN_T ? 1 : 0;
-    const size_t ring = p.bulk ? decode::SMEM_MAX - decode::smem_bytes(0, 0, 1) : decode::SMEM_BUDGET;
-    p.stages = static_cast<int>(ring / p.stage_bytes);
+    // the ring takes what shared memory the reduce staging boxes leave
+    p.stages = static_cast<int>((decode::SMEM_MAX - decode::smem_bytes(0, 0)) / p.stage_bytes);
     if (p.stages > decode::MAX_STAGES) p.stages = decode::MAX_STAGES;
     p.may_outlier = (fin && fin->may_outlier) ? 1 : 0;
     uint32_t cols = 32;
@@ -560,22 +549,20 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     // row, so the 256-byte L2 line is used whole.
     I8R_TRY(make_map(&map_wq, Wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, decode::BK, decode::BMH));
     I8R_TRY(make_map(&map_xq, Xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, T, K, p.TP, decode::BK));
-    map_xo = map_w16o = map_acc = map_yo = map_xq;   // unused without a 16-bit part / in atomic mode
-    if (p.bulk) {
-        // acc32 [T, N] int32 in 32 x 32 boxes, unswizzled 128-byte rows
-        I8R_TRY(make_map(&map_acc, acc32, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, T, N, decode::RED_ROWS, 32,
+    map_xo = map_w16o = map_yo = map_xq;   // unused without a 16-bit part
+    // acc32 (and Yo) [T, N] in 32 x 32 boxes, unswizzled 128-byte rows
+    I8R_TRY(make_map(&map_acc, acc32, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, T, N, decode::RED_ROWS, 32,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
+    if (fin && fin->Yo)
+        I8R_TRY(make_map(&map_yo, fin->Yo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, N, decode::RED_ROWS, 32,
                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
-        if (fin && fin->Yo)
-            I8R_TRY(make_map(&map_yo, fin->Yo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, N, decode::RED_ROWS, 32,
-                             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
-    }
     p.W16 = W16;
     if (fin && Xo) {
         I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, p.TP, decode::OBK));
         if (W16o) I8R_TRY(make_map(&map_w16o, W16o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.o_rows, N, 64, 64));
     }
     const long long g = p.total_units < dev->sms ? p.total_units : dev->sms;
-    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes, p.bulk);
+    const size_t smem = decode::smem_bytes(p.stages, p.stage_bytes);
     record_before(s);
     cudaError_t e = launch_dependent(decode::gemm_decode_kernel, dim3(static_cast<unsigned>(g)),
                                      dim3(decode::THREADS), smem, s, 1, map_wq, map_xq, map_xo, map_w16o, map_acc, map_yo,
@@ -586,7 +573,7 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     }
     I8R_LAUNCHED();
     record_after(s);
-    if (p.bulk && fin) {
+    if (fin) {
         const long long items = static_cast<long long>(T) * (N / 8);
         e = launch_dependent(decode::decode_finalize_kernel, dim3(static_cast<unsigned>((items + 255) / 256)), dim3(256),
                              0, s, 1, static_cast<const int32_t *>(acc32), static_cast<const float *>(fin->Yo),
@@ -730,13 +717,12 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
     __half *Xo = reinterpret_cast<__half *>(ws + w.Xo);
     const bool small_t = T <= decode::MAX_T;
     int32_t *acc32 = small_t ? reinterpret_cast<int32_t *>(ws + w.acc32) : nullptr;
-    int32_t *counters = small_t ? reinterpret_cast<int32_t *>(ws + w.counters) : nullptr;
     float *Yo = small_t ? reinterpret_cast<float *>(ws + w.Yo) : nullptr;
     const __half *x = static_cast<const __half *>(X);
     const __half *w16 = static_cast<const __half *>(W16);
     __half *y = static_cast<__half *>(Y);
 
-    // decode: the outlier scan clears the split-K accumulator and the tile counters
+    // decode: the activation side clears the split-K accumulator
     const size_t zero_bytes = small_t ? w.total - w.acc32 : 0;
     // compacted outlier rows: the first outlier_rows(T, K) rows of W16 (the GEMMs
     // gather any further rows from W16 themselves), or the Wq-only variant's
@@ -748,7 +734,6 @@ i8r_status mixed_linear_impl(const void *X, int T, int K, const int8_t *Wq, cons
         return launch_prefill(dev, Xq, Xo, T, K, Wq, sW, w16, N, count, idx, sX, y, nullptr, stream, W16o);
 
     decode::Params fin{};
-    fin.counters = counters;
     fin.sX = sX;
     fin.sW = sW;
     fin.count = count;

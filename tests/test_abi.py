@@ -98,14 +98,16 @@ def test_wq_variant_host_checks_and_capacity(so):
     # at least 256 and K/16, rounded up to 64, at most K rounded up to 64
     cap = so.int8_mixed_linear_wq_max_outliers
     assert [cap(k) for k in (16, 64, 1024, 5120, 12288, 49152)] == [64, 64, 256, 320, 768, 3072]
-    # the workspace holds exactly those rows on top of the plain one: at prefill
-    # sizes the plain one already compacts 256 W16 rows, at decode sizes none
+    # the workspace holds exactly those rows where the plain one holds its
+    # compacted W16 rows: 256 at prefill sizes; at decode sizes at least 256
+    # and K/64 (rounded up to 64), at most K rounded up to 64
+    k64 = lambda K: (K + 63) // 64 * 64
     for T, K, N in ((2048, 12288, 49152), (300, 1024, 512)):
         extra = so.int8_mixed_linear_wq_workspace_size(T, K, N) - so.int8_mixed_linear_workspace_size(T, K, N)
-        assert extra == (cap(K) - min(256, (K + 63) // 64 * 64)) * N * 2
-    for T, K, N in ((16, 12288, 49152), (128, 1024, 512), (1, 64, 16)):
+        assert extra == (cap(K) - min(256, k64(K))) * N * 2
+    for T, K, N in ((16, 12288, 49152), (128, 1024, 512), (1, 64, 16), (16, 49152, 12288)):
         extra = so.int8_mixed_linear_wq_workspace_size(T, K, N) - so.int8_mixed_linear_workspace_size(T, K, N)
-        assert extra == cap(K) * N * 2
+        assert extra == (cap(K) - min(k64(K), max(256, k64((K + 63) // 64)))) * N * 2
 
 
 def test_chain_host_checks_and_workspace(so):

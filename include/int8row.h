@@ -72,9 +72,6 @@ typedef enum {
 #define I8R_DEV_OK 0
 #define I8R_DEV_PIPELINE_TIMEOUT 1   /* a shared-memory pipeline wait gave up */
 #define I8R_DEV_TMEM_TIMEOUT 2       /* a tensor-memory hand-off wait gave up */
-#define I8R_DEV_OUTLIER_CAP 3        /* int8_mixed_linear_wq found more outlier columns
-                                        than its workspace holds rows for; Y lacks the
-                                        16-bit part of the excess columns */
 
 /* ---------------------------------------------------------------------------
  * Weight conversion.  The pages describe a 16/32-bit checkpoint converted to
@@ -127,12 +124,12 @@ i8r_status int8_mixed_linear(const void *X, int T, int K,
  * so Y = fp16( acc*sX[t]*sW[n]/127^2 + X[:,O] W~[O,:] ).
  * Arguments, layouts and workspace rules are those of int8_mixed_linear,
  * with workspace of at least int8_mixed_linear_wq_workspace_size(T, K, N)
- * bytes.  That workspace holds the dequantised rows of at most
+ * bytes.  That workspace holds the dequantised rows of the first
  * int8_mixed_linear_wq_max_outliers(K) outlier columns (at least 256 and
  * 1/16 of K, rounded up to a multiple of 64, and not more than K rounded
- * up to 64), at every T.  A call that finds more outlier columns than that
- * sets I8R_DEV_OUTLIER_CAP in the device status word, and its Y lacks the
- * 16-bit part of the excess columns.
+ * up to 64), at every T; the GEMM dequantises the rows of any further
+ * outlier columns itself, by index, with the same rounding (slower per row,
+ * same result).
  * ------------------------------------------------------------------------- */
 size_t int8_mixed_linear_wq_workspace_size(int T, int K, int N);
 

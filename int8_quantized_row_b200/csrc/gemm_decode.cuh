@@ -83,8 +83,9 @@ struct Params {
     const int32_t *count;          // |O|
     const int32_t *idx;            // the outlier columns, ascending
     const __half *W16;             // [K,N] fp16 (null for the Wq-only variant)
+    const int8_t *Wq;              // [K,N] int8 (the Wq-only variant's rows past the compacted ones)
     int o_rows;                    // rows of the compacted outlier rows W16o (W16 rows, or dequantised Wq rows)
-    int wq_only;                   // no W16: outlier rows come from W16o (zeros past o_rows)
+    int wq_only;                   // no W16: outlier rows from W16o, dequantised from Wq past o_rows
     int may_outlier;               // alpha < +inf: a tile's first stage may be an outlier stage
     __half *Y;
     float *Yo;                     // [T,N] fp32: the 16-bit outlier part (written when |O| > 0)
@@ -263,15 +264,50 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tma_load_2d(a + A_HALF, &map_wq, fb, tile * BM + BMH, j * BK);
                         tma_load_2d(a + A_BYTES, &map_xq, fb, j * BK, 0);
                     }
-                } else if (p.wq_only || (j + 1) * OBK <= p.o_rows) {
-                    // compacted rows (W16 rows, or dequantised Wq rows): four 64 x 64
-                    // boxes; for the Wq-only variant past o_rows an out-of-range box,
-                    // i.e. zeros (the quantiser reports the overflow)
+                } else if ((j + 1) * OBK <= p.o_rows) {
+                    // compacted rows (W16 rows, or dequantised Wq rows): four 64 x 64 boxes
                     if (lane == 0) {
-                        const int y = (j + 1) * OBK <= p.o_rows ? j * OBK : p.o_rows;
                         mbar_arrive_expect_tx(fb, tx);
                         tma_load_2d(a + A_BYTES, &map_xo, fb, j * OBK, 0);
-                        for (int c = 0; c < 4; ++c) tma_load_2d(a + c * O_CHUNK, &map_w16o, fb, tile * BM + 64 * c, y);
+                        for (int c = 0; c < 4; ++c)
+                            tma_load_2d(a + c * O_CHUNK, &map_w16o, fb, tile * BM + 64 * c, j * OBK);
+                    }
+                } else if (p.wq_only) {
+                    // Wq-only variant past the compacted rows: the lanes dequantise the
+                    // Wq rows of outliers j*64 .. by index, W~ = fp16_rn(q * fl32(sW/127))
+                    // as the quantiser's compaction does, zero past |O| rounded up to 16;
+                    // lane l writes columns 8l .. 8l+7 of every row into the
+                    // 128-byte-swizzled chunk l/8.  Generic stores: fenced to the async
+                    // proxy before the arrive (the MMA warp fences again before reading).
+                    const int rows = min(OBK, (count - j * OBK + 15) / 16 * 16);
+                    const int g0 = j * OBK + lane, g1 = j * OBK + 32 + lane;
+                    const int k0 = g0 < count ? p.idx[g0] : -1;
+                    const int k1 = g1 < count ? p.idx[g1] : -1;
+                    const int col = tile * BM + lane * 8;
+                    const bool col_ok = col < p.N;
+                    float d[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) d[e] = col_ok ? __fdiv_rn(p.sW[col + e], 127.0f) : 0.0f;
+                    uint8_t *chunk = a + (lane >> 3) * O_CHUNK;
+                    const int unit = lane & 7;
+                    for (int r = 0; r < rows; ++r) {
+                        const int k = __shfl_sync(0xFFFFFFFFu, r < 32 ? k0 : k1, r & 31);
+                        uint2 q8 = make_uint2(0u, 0u);
+                        if (k >= 0 && col_ok) q8 = __ldg(reinterpret_cast<const uint2 *>(p.Wq + static_cast<size_t>(k) * p.N + col));
+                        __align__(16) __half v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int q = static_cast<int8_t>(((e < 4 ? q8.x : q8.y) >> (8 * (e & 3))) & 0xFFu);
+                            v[e] = __float2half_rn(__fmul_rn(static_cast<float>(q), d[e]));
+                        }
+                        *reinterpret_cast<uint4 *>(chunk + r * 128 + ((unit ^ (r & 7)) << 4)) =
+                            *reinterpret_cast<const uint4 *>(v);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(fb, static_cast<uint32_t>(p.TP * OBK * 2));
+                        tma_load_2d(a + A_BYTES, &map_xo, fb, j * OBK, 0);
                     }
                 } else {
                     // The W16 rows of outliers j*64 .., zero past |O| rounded up to 16

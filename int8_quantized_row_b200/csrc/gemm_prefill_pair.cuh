@@ -73,7 +73,8 @@ struct Params {
     __half *Y;
     int32_t *acc_out;
     int o_rows;                    // outlier rows compacted into the W16o map (multiple of 64)
-    int wq_only;                   // no W16 map: blocks past o_rows read zeros (flagged upstream)
+    int wq_only;                   // no W16 map: blocks past o_rows are dequantised from Wq by index
+    const int8_t *Wq;              // [K,N] int8 (the Wq-only variant's rows past the compacted ones)
 };
 
 struct Barriers {
@@ -84,6 +85,7 @@ struct Barriers {
     uint64_t acc_final_full[2];
     uint64_t acc_empty[2];
     uint64_t drain;
+    uint64_t wq_ready[STAGES];     // leader's: both CTAs wrote their dequantised outlier rows (Wq-only)
     uint32_t tmem_base;
     int abort;
     int orow[OBK];                 // W16 row of each outlier of the stage being loaded
@@ -145,6 +147,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&bars->acc_empty[b], 8);
         }
         mbar_init(&bars->drain, 1);
+        for (int s = 0; s < STAGES; ++s) mbar_init(&bars->wq_ready[s], 2);
         bars->abort = 0;
         fence_mbar_init();
         tma_prefetch_map(&map_xq);
@@ -170,6 +173,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t lead_full = mapa_shared(smem_u32(&bars->full[0]), 0);
     const uint32_t lead_acc_conv = mapa_shared(smem_u32(&bars->acc_conv[0]), 0);
     const uint32_t lead_acc_empty = mapa_shared(smem_u32(&bars->acc_empty[0]), 0);
+    const uint32_t lead_wq_ready = mapa_shared(smem_u32(&bars->wq_ready[0]), 0);
 
     // Weight halves of this CTA's first stages do not depend on the activation
     // kernels: request them first.
@@ -231,15 +235,50 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (!compact && !p.wq_only)
                         for (int j = lane; j < rows; j += 32) bars->orow[j] = j < left ? p.idx[blk * OBK + j] : p.K;
                     __syncwarp();
-                    if (lane == 0 && (compact || p.wq_only)) {
-                        // Wq-only past the compacted rows: an out-of-range box of W16o, i.e. zeros
-                        const int y = compact ? blk * OBK : p.o_rows;
+                    if (!compact && p.wq_only) {
+                        // Wq-only past the compacted rows: the Xo tile by TMA, and this
+                        // CTA's 128 columns of the outlier rows dequantised from Wq by
+                        // index, W~ = fp16_rn(q * fl32(sW/127)) as the quantiser's
+                        // compaction does (zero past |O|), written with generic stores
+                        // into the 128-byte-swizzled chunks a box load would fill: 16
+                        // bytes per lane, two rows per pass.  Each CTA then arrives on
+                        // the leader's wq_ready, which the MMA issuer also waits for.
+                        if (lane == 0) {
+                            if (leader) mbar_arrive_expect_tx(&bars->full[stage], 2u * static_cast<uint32_t>(XO_BYTES));
+                            tma_load_2d_pair(a, &map_xo, lead_full + 8u * stage, blk * OBK, m0);
+                        }
+                        const int u16 = lane & 15;
+                        const int col = n0 + 8 * u16;
+                        const bool col_ok = col < p.N;
+                        float dq[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dq[e] = col_ok ? __fdiv_rn(p.sW[col + e], 127.0f) : 0.0f;
+                        uint8_t *chunk = a + A_BYTES + (u16 >> 3) * B_CHUNK_F16;
+                        const int unit = u16 & 7;
+                        for (int r = lane >> 4; r < rows; r += 2) {
+                            const int k = r < left ? p.idx[blk * OBK + r] : -1;
+                            uint2 q8 = make_uint2(0u, 0u);
+                            if (k >= 0 && col_ok)
+                                q8 = __ldg(reinterpret_cast<const uint2 *>(p.Wq + static_cast<size_t>(k) * p.N + col));
+                            __align__(16) __half v[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int q = static_cast<int8_t>(((e < 4 ? q8.x : q8.y) >> (8 * (e & 3))) & 0xFFu);
+                                v[e] = __float2half_rn(__fmul_rn(static_cast<float>(q), dq[e]));
+                            }
+                            *reinterpret_cast<uint4 *>(chunk + r * 128 + ((unit ^ (r & 7)) << 4)) =
+                                *reinterpret_cast<const uint4 *>(v);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(lead_wq_ready + 8u * stage);
+                    } else if (lane == 0 && compact) {
                         if (leader)
                             mbar_arrive_expect_tx(&bars->full[stage], 2u * static_cast<uint32_t>(XO_BYTES + OBK * 256));
                         const uint32_t fb = lead_full + 8u * stage;
                         tma_load_2d_pair(a, &map_xo, fb, blk * OBK, m0);
-                        tma_load_2d_pair(a + A_BYTES, &map_w16o, fb, n0, y);
-                        tma_load_2d_pair(a + A_BYTES + B_CHUNK_F16, &map_w16o, fb, n0 + 64, y);
+                        tma_load_2d_pair(a + A_BYTES, &map_w16o, fb, n0, blk * OBK);
+                        tma_load_2d_pair(a + A_BYTES + B_CHUNK_F16, &map_w16o, fb, n0 + 64, blk * OBK);
                     } else if (lane == 0) {
                         if (leader)
                             mbar_arrive_expect_tx(&bars->full[stage], 2u * static_cast<uint32_t>(XO_BYTES + rows * 256));
@@ -296,6 +335,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t own_final_c = mapa_shared(own_final, 0);
             int stage = 0;
             uint32_t phase = 0;
+            uint32_t wq_phase = 0;                       // bit s: parity of wq_ready[s]'s next phase
             walk_schedule(p, nob, cluster_id, clusters, [&](int kind, int, int it, int blk) -> bool {
                 const int buf = it & 1;
                 const uint32_t use = static_cast<uint32_t>(it >> 1) & 1u;
@@ -309,6 +349,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tc_fence_after_sync();
                 }
                 if (!mbar_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+                if (kind == 1 && p.wq_only && blk * OBK + OBK > p.o_rows) {
+                    // the dequantised rows both CTAs wrote with generic stores
+                    if (!mbar_wait_cluster(&bars->wq_ready[stage], (wq_phase >> stage) & 1u, abort,
+                                           I8R_DEV_PIPELINE_TIMEOUT))
+                        return false;
+                    wq_phase ^= 1u << stage;
+                    fence_proxy_async_smem();
+                }
                 tc_fence_after_sync();
                 {
                     const uint32_t a = smem_u32(smem + stage * STAGE_BYTES);

@@ -499,6 +499,7 @@ i8r_status launch_prefill(const DeviceInfo *dev, const int8_t *Xq, const __half 
     p.acc_out = acc_out;
     p.o_rows = o_rows;
     p.wq_only = wq_only ? 1 : 0;
+    p.Wq = Wq;
     const int clusters = p.num_tiles < dev->pair_clusters ? p.num_tiles : dev->pair_clusters;
     record_before(s);
     cudaError_t e;
@@ -557,6 +558,7 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
         I8R_TRY(make_map(&map_yo, fin->Yo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, T, N, decode::RED_ROWS, 32,
                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_SWIZZLE_NONE));
     p.W16 = W16;
+    p.Wq = Wq;
     if (fin && Xo) {
         I8R_TRY(make_map(&map_xo, Xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, p.TP, decode::OBK));
         if (W16o) I8R_TRY(make_map(&map_w16o, W16o, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.o_rows, N, 64, 64));

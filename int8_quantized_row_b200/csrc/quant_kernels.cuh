@@ -323,8 +323,8 @@ inline size_t quantize_smem_bytes(int K) { return static_cast<size_t>((K + 31) /
 // of gathering rows):  W16o[j,:] = W16[O_j,:] for j < |O|, zero rows up to the
 // next multiple of 16 (at most o_rows; the MMAs read no row past that, so the
 // rest of a 64-row box may hold anything).  Without W16 (the Wq-only variant) the
-// rows are dequantised instead, W16o[j,n] = fp16_rn(Wq[O_j,n] * fl32(sW[n]/127)),
-// and more than o_rows outlier columns is reported (I8R_DEV_OUTLIER_CAP).
+// rows are dequantised instead, W16o[j,n] = fp16_rn(Wq[O_j,n] * fl32(sW[n]/127));
+// the GEMMs dequantise any rows past o_rows themselves.
 // Block e of the G compaction blocks copies rows e, e+G, ... with eight
 // 16-byte stores in flight per thread, 256 ranks of the index list at a time
 // (the window held in shared memory).
@@ -335,7 +335,6 @@ __device__ __forceinline__ void gather_outlier_weight_rows(const uint32_t *smask
                                                            int total, const __half *__restrict__ W16,
                                                            const int8_t *__restrict__ Wq, const float *__restrict__ sW,
                                                            int N, __half *__restrict__ W16o, int o_rows, int e, int G) {
-    if (!W16 && total > o_rows && e == 0 && threadIdx.x == 0) report_status(I8R_DEV_OUTLIER_CAP);
     __shared__ int oidx[kCompactOutlierRows];
     const int rows = min((total + 15) / 16 * 16, o_rows);
     const int vec = N / 8;

@@ -4,8 +4,8 @@ Same tolerance on Y as the fp16-weight layer.  At every T the quantiser's
 leading blocks write the dequantised rows into the workspace; shapes cover
 the decode kernel (T <= 128) and the prefill kernel, outlier sets of one and
 several 64-column blocks, a long schedule, alpha = 0 at decode size, an
-outlier count exactly at the workspace's capacity, and one past it at both
-kernels (reported in the device status word).
+outlier count exactly at the workspace's capacity, and counts past it at both
+kernels, where the GEMM's producer dequantises the remaining rows by index.
 """
 import numpy as np
 import pytest
@@ -15,8 +15,6 @@ import int8_quantized_row_b200 as i8
 from gpu_helpers import assert_y_close, device_status_clean, outlier_x, to_dev, to_host
 
 pytestmark = pytest.mark.gpu
-
-I8R_DEV_OUTLIER_CAP = 3
 
 WQ_CASES = [
     # T, K, N, outlier columns, alpha, rows sampled (None: all)
@@ -29,6 +27,9 @@ WQ_CASES = [
     (300, 2048, 256, list(range(0, 2048, 31)), 6.0, None),   # |O| = 67: two outlier blocks
     (2048, 1024, 4096, list(range(0, 1024, 15)), 6.0, 7),    # long schedule, |O| = 69
     (300, 1024, 512, list(range(0, 1024, 4)), 6.0, None),    # |O| = 256 = the capacity at K = 1024
+    (300, 1024, 512, list(range(0, 1024, 3)), 6.0, None),    # |O| = 342: 86 rows past the capacity
+    (16, 1024, 1040, list(range(0, 1024, 3)), 6.0, None),    # the same at decode size, ragged N
+    (260, 1024, 256, [], 0.0, None),                          # prefill, every column an outlier
 ]
 
 
@@ -43,7 +44,6 @@ def test_wq_variant_matches_oracle(orc, T, K, N, cols, alpha, every):
     torch.cuda.synchronize()
     rows = None if every is None else np.arange(0, T, every, dtype=np.int32)
     Y_o, _, _, cnt = orc.mixed_linear(X, Wq_o, sW_o, None, alpha, rows=rows)
-    assert cnt <= i8.int8_mixed_linear_wq_max_outliers(K)
     assert_y_close(Y if rows is None else Y[rows], Y_o, f"wq T={T} K={K} N={N} |O|={cnt}")
     assert device_status_clean()
 
@@ -68,15 +68,18 @@ def test_wq_variant_differs_from_fp16_weights_only_in_outlier_rows(orc):
 
 
 @pytest.mark.parametrize("T", [260, 16])
-def test_wq_variant_reports_more_outliers_than_its_workspace_holds(T):
-    # alpha = 0 makes every column an outlier: 1024 > 256 rows (prefill and decode)
+def test_wq_variant_past_its_workspace_capacity_matches_oracle(orc, T):
+    # alpha = 0 makes every column an outlier: 1024 > 256 compacted rows (prefill
+    # and decode); the rows past them are dequantised in the GEMM, nothing is dropped
     K, N = 1024, 256
     assert i8.int8_mixed_linear_wq_max_outliers(K) == 256
     rng = np.random.default_rng(9)
     X = rng.standard_normal((T, K)).astype(np.float16)
     W = (rng.standard_normal((K, N)) * 0.02).astype(np.float16)
+    Wq_o, sW_o = orc.quantize_weight_colwise(W)
     Wq, sW = i8.int8_quantize_weight_colwise(to_dev(W))
-    i8.int8_mixed_linear_wq(to_dev(X), Wq, sW, 0.0)
-    torch.cuda.synchronize()
-    assert i8.int8_read_and_clear_device_status() == I8R_DEV_OUTLIER_CAP
-    assert device_status_clean()                               # cleared by the read
+    Y = to_host(i8.int8_mixed_linear_wq(to_dev(X), Wq, sW, 0.0))
+    Y_o, _, _, cnt = orc.mixed_linear(X, Wq_o, sW_o, None, 0.0)
+    assert cnt == K
+    assert_y_close(Y, Y_o, f"wq alpha=0 T={T}")
+    assert device_status_clean()

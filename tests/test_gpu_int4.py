@@ -129,3 +129,24 @@ def test_int4_linear_t0_and_limits():
     assert Y.shape == (0, 16)
     with pytest.raises(i8.I8RError):
         i8.int4_linear(torch.zeros((65, 256), dtype=torch.float16, device="cuda"), W4, S4, 16)
+
+
+def test_int4_full_size_fc1_decode(orc):
+    """The 175B fc1 shape at T=16 (K=12288, N=49152; 302 MB of packed codes), in
+    the launch configuration the sweep times: every group's (s, lo) bit for bit,
+    and Y on sampled rows within the tolerance."""
+    from int8_quantized_row_b200 import workloads as wl
+    T, K, N = 16, 12288, 49152
+    W = wl.make_w(K, N, 0.01)
+    X = wl.make_x(T, K, 0, seed=16)
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev(W))
+    Y = to_host(i8.int4_linear(to_dev(X), W4, S4, N))
+    codes_o, s_o, lo_o = orc.int4_quantize_groupwise(W)
+    NP, KT = L.padded_n(N), K // 256
+    sl = to_host(S4).reshape(NP // 256, KT, 256, 4, 2, 2).view("<u2")[..., 0].transpose(1, 3, 0, 2, 4).reshape(K // 64, NP, 2)
+    assert np.array_equal(sl[:, :N, 0], s_o.view(np.uint16))
+    assert np.array_equal(sl[:, :N, 1], lo_o.view(np.uint16))
+    rows = np.array([0, 7, 15], np.int32)
+    Y_o, _ = orc.int4_linear(X, codes_o, s_o, lo_o, rows=rows)
+    assert_y_close(Y[rows], Y_o, "int4 fc1 T=16 full size")
+    assert device_status_clean()

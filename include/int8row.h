@@ -295,9 +295,12 @@ i8r_status int8_outlier_stats(const void *X, int T, int K, float alpha,
  *              (256: a counter for the one-kernel path), 16-byte aligned
  *
  * int8_debug_set_activation_path: 1 (the default) runs the activation side
- *   as one cooperative kernel for batches of 8 to 128 rows that fit in the
- *   SMs' shared memory, 2 as that kernel whenever the batch fits, 0 always
- *   as the outlier scan followed by the row quantiser.  When the runtime
+ *   as one kernel wherever that pays: for batches of 1 to 7 rows with
+ *   T*K <= 32768 the row quantiser finds the outlier mask itself (every block
+ *   reads all of X), for 8 to 128 rows that fit in the SMs' shared memory one
+ *   cooperative kernel holds X and finds the mask across a grid barrier.
+ *   2 takes that cooperative kernel whenever the batch fits, 0 always the
+ *   outlier scan followed by the row quantiser.  When the runtime
  *   refuses the cooperative launch (too few SMs or too little shared memory
  *   free to the context), the call takes the scan + quantiser pair instead;
  *   3 behaves as 1 with every cooperative launch treated as refused, so that

@@ -259,7 +259,7 @@ def int8_quantize_activation(X, alpha=6.0, with_xo=True, stream=None):
     T, K = X.shape
     dev = X.device
     out = dict(
-        mask=torch.zeros((K + 31) // 32 + 3, dtype=torch.int32, device=dev),
+        mask=torch.full(((K + 31) // 32 + 3,), -1, dtype=torch.int32, device=dev),
         idx=torch.full((K,), -1, dtype=torch.int32, device=dev),
         count=torch.zeros(4, dtype=torch.int32, device=dev),
         sX=torch.empty(max(T, 1), dtype=torch.float32, device=dev),

@@ -23,11 +23,11 @@
 // bits.  Rows are processed by groups of warps: a few warps per row when a
 // block holds many rows, the whole block on one row when it holds one.
 //
-// The outlier test runs on packed fp16 pairs as an integer compare: for
-// finite x and alpha >= 0, |x| >= alpha holds exactly when the magnitude bits
-// of x (bits & 0x7FFF) are at least those of the smallest fp16 value >= alpha
-// (magnitude bit patterns order like the values), so one __vcmpgeu2 tests two
-// elements.  The host supplies that threshold.
+// The outlier test runs on packed fp16 pairs as an integer compare
+// (outlier_pair): for alpha >= 0, |x| >= alpha holds exactly when the
+// magnitude bits of x (bits & 0x7FFF) are at least those of the smallest fp16
+// value >= alpha and x is not NaN, so two compares test two elements.  The
+// host supplies that threshold.
 #pragma once
 
 #include "device_common.cuh"
@@ -37,6 +37,9 @@ namespace i8r {
 
 constexpr int kFusedThreads = 1024;
 constexpr int kFusedMinRows = 8;    // fewer rows: the scan + quantiser pair is faster
+// Fewer rows than kFusedMinRows and at most this many elements of X: the row
+// quantiser finds the mask itself (every block reads all of X), no scan.
+constexpr long long kSelfMaskElems = 1 << 15;
 constexpr size_t kFusedSmemMax = 200 * 1024;
 
 // Shared memory of activation_fused_kernel: R rows of X, the mask words and
@@ -96,10 +99,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) activation_fused_kernel(
             if (c < chunks)
                 for (int r = 0; r < nrows; ++r) {
                     const uint4 u = reinterpret_cast<const uint4 *>(rows + static_cast<size_t>(r) * K)[c];
-                    h0 |= __vcmpgeu2(u.x & 0x7FFF7FFFu, thr2);
-                    h1 |= __vcmpgeu2(u.y & 0x7FFF7FFFu, thr2);
-                    h2 |= __vcmpgeu2(u.z & 0x7FFF7FFFu, thr2);
-                    h3 |= __vcmpgeu2(u.w & 0x7FFF7FFFu, thr2);
+                    h0 |= outlier_pair(u.x, thr2);
+                    h1 |= outlier_pair(u.y, thr2);
+                    h2 |= outlier_pair(u.z, thr2);
+                    h3 |= outlier_pair(u.w, thr2);
                 }
             // element 2i is the low half of word i, 2i+1 the high half
             const uint32_t f = (h0 & 1u) | ((h0 >> 15) & 2u) | ((h1 & 1u) << 2) | ((h1 >> 13) & 8u) |

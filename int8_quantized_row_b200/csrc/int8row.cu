@@ -319,11 +319,15 @@ cudaError_t launch_dependent(void (*kernel)(Params...), dim3 grid, dim3 block, s
 }
 
 // The row quantiser: G compaction blocks, then one block per row, launched as
-// a programmatic dependent of the outlier scan.
+// a programmatic dependent of the outlier scan (or, finding the mask itself,
+// as the call's first kernel: an ordinary launch).
 template <int kThreads, typename... Args>
-cudaError_t launch_rows(cudaStream_t s, int T, int G, size_t smem, Args &&...args) {
-    return launch_dependent(quantize_rows_kernel<kThreads>, dim3(G + T), dim3(kThreads), smem, s, 1,
-                            std::forward<Args>(args)...);
+cudaError_t launch_rows(cudaStream_t s, int T, int G, size_t smem, bool dependent, Args &&...args) {
+    if (dependent)
+        return launch_dependent(quantize_rows_kernel<kThreads>, dim3(G + T), dim3(kThreads), smem, s, 1,
+                                std::forward<Args>(args)...);
+    quantize_rows_kernel<kThreads><<<dim3(G + T), dim3(kThreads), smem, s>>>(std::forward<Args>(args)...);
+    return cudaGetLastError();
 }
 
 // Grid of the row-band outlier scan: bands of 2048 columns, row blocks of at
@@ -358,6 +362,36 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     const int mode = g_activation_fused.load(std::memory_order_relaxed);
     const bool size_ok = mode == 2 ? T >= 1 : ((mode == 1 || mode == 3) && T >= kFusedMinRows && T <= decode::MAX_T);
     const bool fused = grid_ctr && size_ok && dev->fused_ok && fused_smem_bytes(fR, K) <= kFusedSmemMax;
+    // Below kFusedMinRows rows (modes 1 and 3) the row quantiser finds the mask
+    // itself: every block reads the few rows of X (at most kSelfMaskElems
+    // elements, from L2 after the first), one launch in all.
+    const bool self_mask = !fused && (mode == 1 || mode == 3) && T >= 1 && T < kFusedMinRows &&
+                           static_cast<long long>(T) * K <= kSelfMaskElems;
+    if (self_mask) {
+        const int rt = row_threads(K);
+        const int o_rows = W16o ? outlier_rows(T, K, W16 == nullptr) : 0;
+        const int G = W16o ? std::min(o_rows, 128) : 0;
+        const size_t smem = quantize_smem_bytes(K);
+        const uint32_t thr = half_threshold_bits(alpha);
+        const uint32_t thr2 = thr | (thr << 16);
+        const uint32_t *no_parts = nullptr;
+        cudaError_t e;
+        if (rt == 64)
+            e = launch_rows<64>(s, T, G, smem, false, X, T, K, no_parts, 0, sX, Xq, Xo, mask, idx, count, W16, Wq,
+                                sW, N, W16o, o_rows, G, thr2, static_cast<int4 *>(zero), zero_bytes / 16);
+        else if (rt == 128)
+            e = launch_rows<128>(s, T, G, smem, false, X, T, K, no_parts, 0, sX, Xq, Xo, mask, idx, count, W16, Wq,
+                                 sW, N, W16o, o_rows, G, thr2, static_cast<int4 *>(zero), zero_bytes / 16);
+        else
+            e = launch_rows<256>(s, T, G, smem, false, X, T, K, no_parts, 0, sX, Xq, Xo, mask, idx, count, W16, Wq,
+                                 sW, N, W16o, o_rows, G, thr2, static_cast<int4 *>(zero), zero_bytes / 16);
+        if (e != cudaSuccess) {
+            tl_last_cuda_error = static_cast<int>(e);
+            return I8R_ECUDA;
+        }
+        I8R_LAUNCHED();
+        return I8R_OK;
+    }
     clear_mask_kernel<<<1, 256, 0, s>>>(mask, nwords, fused ? grid_ctr : nullptr);
     I8R_LAUNCHED();
     if (fused) {
@@ -417,15 +451,16 @@ i8r_status launch_activation(const DeviceInfo *dev, const __half *X, int T, int 
     const size_t smem = quantize_smem_bytes(K);
     const uint32_t *m = mask;
     uint32_t *no_mask_out = nullptr;
+    int4 *no_zero = nullptr;
     if (rt == 64)
-        e = launch_rows<64>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
-                            W16o, o_rows, G);
+        e = launch_rows<64>(s, T, G, smem, true, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
+                            W16o, o_rows, G, 0u, no_zero, size_t{0});
     else if (rt == 128)
-        e = launch_rows<128>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
-                             W16o, o_rows, G);
+        e = launch_rows<128>(s, T, G, smem, true, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW,
+                             N, W16o, o_rows, G, 0u, no_zero, size_t{0});
     else
-        e = launch_rows<256>(s, T, G, smem, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW, N,
-                             W16o, o_rows, G);
+        e = launch_rows<256>(s, T, G, smem, true, X, T, K, m, 1, sX, Xq, Xo, no_mask_out, idx, count, W16, Wq, sW,
+                             N, W16o, o_rows, G, 0u, no_zero, size_t{0});
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;

@@ -426,13 +426,46 @@ __device__ __forceinline__ uint32_t pack4_s8(int q0, int q1, int q2, int q3) {
     return __byte_perm(p01, p23, 0x5410u);
 }
 
+// |x| >= alpha on a pair of fp16 values, 0xFFFF per half where it holds:
+// the magnitude bits (bits & 0x7FFF) at least those of the smallest fp16
+// >= alpha (thr2, both halves) -- magnitude bit patterns order like the values
+// -- and at most those of infinity, so that NaN, like the float compare
+// fabsf(x) >= alpha, is no outlier.
+__device__ __forceinline__ uint32_t outlier_pair(uint32_t u, uint32_t thr2) {
+    const uint32_t a = u & 0x7FFF7FFFu;
+    return __vcmpgeu2(a, thr2) & __vcmpleu2(a, 0x7C007C00u);
+}
+
+// The outlier bits of 32 columns (word w) over T rows (outlier_pair).
+__device__ __forceinline__ uint32_t outlier_word(const __half *__restrict__ X, int T, int K, int w, uint32_t thr2) {
+    uint32_t m = 0;
+    for (int r = 0; r < T; ++r) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(X + static_cast<size_t>(r) * K + w * 32);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if (w * 32 + q * 8 >= K) break;                 // K % 32 == 16: the last word has two chunks
+            const uint4 u = __ldg(src + q);
+            const uint32_t h0 = outlier_pair(u.x, thr2), h1 = outlier_pair(u.y, thr2);
+            const uint32_t h2 = outlier_pair(u.z, thr2), h3 = outlier_pair(u.w, thr2);
+            const uint32_t f = (h0 & 1u) | ((h0 >> 15) & 2u) | ((h1 & 1u) << 2) | ((h1 >> 13) & 8u) |
+                               ((h2 & 1u) << 4) | ((h2 >> 11) & 32u) | ((h3 & 1u) << 6) | ((h3 >> 9) & 128u);
+            m |= f << (8 * q);
+        }
+    }
+    return m;
+}
+
+// With parts == nullptr (batches of a few rows) every block finds the outlier
+// mask itself from X (thr2, as outlier_word), so the call needs neither the
+// mask clear nor the outlier scan: one launch, and it also clears `zero`
+// (zero16 16-byte words, grid-strided) on the way.
 template <int kRowThreads>
 __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     const __half *__restrict__ X, int T, int K, const uint32_t *__restrict__ parts, int nparts,
     float *__restrict__ sX, int8_t *__restrict__ Xq, __half *__restrict__ Xo, uint32_t *__restrict__ mask_out,
     int32_t *__restrict__ idx_out, int32_t *__restrict__ count_out, const __half *__restrict__ W16,
     const int8_t *__restrict__ Wq, const float *__restrict__ sW, int N, __half *__restrict__ W16o, int o_rows,
-    int G) {
+    int G, uint32_t thr2, int4 *__restrict__ zero, size_t zero16) {
     constexpr int kWarps = kRowThreads / 32;
     extern __shared__ uint32_t qs[];
     __shared__ float red[kWarps];
@@ -457,11 +490,20 @@ __global__ void __launch_bounds__(kRowThreads) quantize_rows_kernel(
     }
     griddep_wait();                     // the outlier scan's partial masks are complete
 
-    // the mask (OR of the parts), then each word's count of earlier outliers
-    for (int w = tid; w < nwords; w += kRowThreads) {
-        uint32_t m = parts[w];
-        for (int q = 1; q < nparts; ++q) m |= parts[static_cast<size_t>(q) * nwords + w];
-        smask[w] = m;
+    // the mask (OR of the parts, or found here), then each word's count of earlier outliers
+    if (parts) {
+        for (int w = tid; w < nwords; w += kRowThreads) {
+            uint32_t m = parts[w];
+            for (int q = 1; q < nparts; ++q) m |= parts[static_cast<size_t>(q) * nwords + w];
+            smask[w] = m;
+        }
+    } else {
+        for (int w = tid; w < nwords; w += kRowThreads) smask[w] = outlier_word(X, T, K, w, thr2);
+        if (zero) {
+            const size_t nthreads = static_cast<size_t>(gridDim.x) * kRowThreads;
+            for (size_t i = static_cast<size_t>(blockIdx.x) * kRowThreads + tid; i < zero16; i += nthreads)
+                zero[i] = make_int4(0, 0, 0, 0);
+        }
     }
     __syncthreads();
     const int per = (nwords + kRowThreads - 1) / kRowThreads;

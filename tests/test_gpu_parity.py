@@ -126,16 +126,26 @@ FUSED_CASES = ACT_CASES + [
     (64, 1024, [], 1.0 / 3.0),
     (64, 1024, [], 3.1),
     (32, 2048, [], 2.0 ** -20),
+    # batches under 8 rows: by default the row quantiser finds the mask itself
+    (1, 32768, [7, 32000], 6.0),              # T*K at the one-launch bound
+    (1, 16400, [5, 16399], 6.0),              # K % 32 == 16: a half word at the end
+    (7, 1040, [], 0.0),                       # every column an outlier
+    (6, 1024, [], 1.0 / 3.0),
+    (2, 2048, [], 2.0 ** -20),
+    (1, 49152, [7, 40000], 6.0),              # the 175B fc2 width, past the bound: scan + quantiser
+    (3, 16400, [9], 6.0),
 ]
 
 
 @pytest.mark.parametrize("T,K,cols,alpha", FUSED_CASES)
 def test_fused_activation_equals_two_kernel_path(orc, T, K, cols, alpha):
-    """Both activation paths, the one-kernel path (X held in shared memory,
-    grid barrier, fp16 bit-pattern threshold) and the outlier scan followed by
-    the row quantiser, each give the oracle's mask, index list, count, row
-    scales, codes and gathered outlier columns bit for bit, including at
-    thresholds fp16 cannot hold."""
+    """Every activation path -- the cooperative one-kernel path (X held in
+    shared memory, grid barrier, fp16 bit-pattern threshold), the default (for
+    batches under 8 rows the row quantiser finding the mask itself, with the
+    same bit-pattern threshold) and the outlier scan followed by the row
+    quantiser -- gives the oracle's mask, index list, count, row scales, codes
+    and gathered outlier columns bit for bit, including at thresholds fp16
+    cannot hold."""
     rng = np.random.default_rng(T * 7 + K)
     X = outlier_x(rng, T, K, cols)
     if T > 2:
@@ -150,7 +160,7 @@ def test_fused_activation_equals_two_kernel_path(orc, T, K, cols, alpha):
     pad = min((cnt_o + 63) // 64 * 64, K)
     Xd = to_dev(X)
     try:
-        for fused in (2, 0):            # the one-kernel path wherever X fits, then the two kernels
+        for fused in (2, 1, 0):         # cooperative wherever X fits, the default, the two kernels
             i8.int8_debug_set_activation_path(fused)
             out = {k: to_host(v).copy() for k, v in i8.int8_quantize_activation(Xd, alpha).items()}
             what = f"path {fused}"
@@ -194,6 +204,52 @@ def test_refused_cooperative_launch_falls_back_to_two_kernels(orc, T, K):
     finally:
         i8.int8_debug_set_activation_path(1)
     assert launches == {1: 2, 3: 3}     # clear + fused kernel; clear + scan + quantiser
+
+
+@pytest.mark.parametrize("T,K", [(3, 1040), (16, 1024)])
+def test_nan_and_inf_in_x_take_the_oracles_outlier_decision(orc, T, K):
+    """|x| >= alpha is false for NaN and true for infinity on every path (the
+    bit-pattern compares exclude NaN as the float compare does), so the
+    outlier set is the oracle's."""
+    rng = np.random.default_rng(T * K)
+    X = outlier_x(rng, T, K, [4])
+    X[0, 10] = np.float16(np.nan)
+    X[T - 1, 11] = -np.float16(np.nan)
+    X[1, 12] = np.float16(np.inf)
+    X[0, 13] = -np.float16(np.inf)
+    mask_o, idx_o = orc.outlier_columns(X, 6.0)
+    assert list(idx_o) == [4, 12, 13]
+    Xd = to_dev(X)
+    try:
+        for mode in (2, 1, 0):
+            i8.int8_debug_set_activation_path(mode)
+            out = {k: to_host(v).copy() for k, v in i8.int8_quantize_activation(Xd, 6.0).items()}
+            cnt = int(out["count"][0])
+            assert cnt == len(idx_o) and np.array_equal(out["idx"][:cnt], idx_o), f"path {mode}"
+            words = out["mask"].view(np.uint32)
+            bits = (words[np.arange(K) // 32] >> (np.arange(K) % 32)) & 1
+            assert np.array_equal(bits.astype(bool), mask_o), f"path {mode}"
+    finally:
+        i8.int8_debug_set_activation_path(1)
+
+
+@pytest.mark.parametrize("T,K,launches", [(1, 12288, 1), (2, 12288, 1), (3, 12288, 3), (7, 1040, 1)])
+def test_small_batches_quantise_in_one_launch(orc, T, K, launches):
+    """Under 8 rows and T*K <= 32768 the default activation side is one launch
+    (the row quantiser finds the mask); past that bound it is the mask clear,
+    the scan and the quantiser."""
+    rng = np.random.default_rng(T + K)
+    X = outlier_x(rng, T, K, [2, K - 1])
+    mask_o, idx_o = orc.outlier_columns(X, 6.0)
+    Xq_o, sX_o = orc.quantize_rows(X, mask_o)
+    Xd = to_dev(X)
+    n0 = i8.int8_kernel_launch_count()
+    out = {k: to_host(v).copy() for k, v in i8.int8_quantize_activation(Xd, 6.0).items()}
+    assert i8.int8_kernel_launch_count() - n0 == launches
+    cnt = int(out["count"][0])
+    assert cnt == len(idx_o) and np.array_equal(out["idx"][:cnt], idx_o)
+    assert np.array_equal(out["sX"][:T], sX_o) and np.array_equal(out["Xq"][:T], Xq_o)
+    assert device_status_clean()
 
 
 def test_activation_t0_is_noop():

@@ -238,9 +238,12 @@ i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K,
  * int4_dequantize_weight: W4, S4 -> W16d [K,N] fp16, the decoded weight W~
  *   (for checking the codec; the product decodes on the fly).
  * int4_linear: Y [T,N] fp16 = X [T,K] fp16 times W~, for 1 <= T <= 64 rows
- *   (T = 0 is a no-op; larger T returns I8R_ERANGE).  The weight is streamed
- *   at 0.5625 bytes per weight, decoded on the fly into the tensor cores'
- *   operand memory.  Workspace of at least int4_linear_workspace_size(T, K, N)
+ *   (T = 0 is a no-op; larger T returns I8R_ERANGE), with fp32 sums of the
+ *   exact fp16 products.  The weight is streamed at 0.5625 bytes per weight
+ *   and decoded on the fly: for T <= 2 on the CUDA cores (one mixed-precision
+ *   fused multiply-add per weight and row), otherwise into the tensor cores'
+ *   operand memory.  X 16-byte aligned.  Workspace of at least
+ *   int4_linear_workspace_size(T, K, N)
  *   bytes, 256-byte aligned (fp32 partial sums of tiles split over the SMs);
  *   its contents on entry are ignored.  Two calls sharing a workspace must
  *   not overlap on the GPU.  Sizes out of these rules return 0 from the size
@@ -260,6 +263,13 @@ size_t int4_linear_workspace_size(int T, int K, int N);
 
 i8r_status int4_linear(const void *X, int T, int K, const uint8_t *W4, const void *S4, int N, void *Y,
                        void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* int4_debug_set_product_path: 0 (the default) runs int4_linear's product on
+ * the CUDA cores for T <= 2 and on the tensor cores otherwise, 1 always on the
+ * tensor cores, 2 on the CUDA cores whenever T <= 4.  The two give the same
+ * sums up to the order of fp32 additions; the switch (process-wide) exists so
+ * that tests and measurements can compare them. */
+void int4_debug_set_product_path(int mode);
 
 /* ---------------------------------------------------------------------------
  * Outlier statistics: the outlier feature dimensions of X and the share of

@@ -19,7 +19,7 @@ __all__ = [
     "int8_selftest_wait_timeout",
     "int8_time_next_gemm", "int8_kernel_launch_count", "LIB_PATH",
     "int4_packed_code_bytes", "int4_packed_scale_bytes", "int4_quantize_weight_groupwise",
-    "int4_dequantize_weight", "int4_linear_workspace_size", "int4_linear",
+    "int4_dequantize_weight", "int4_linear_workspace_size", "int4_linear", "int4_debug_set_product_path",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libint8row.so")
@@ -66,6 +66,8 @@ def lib():
     so.int8_mixed_linear_chain.argtypes = [_I, _P, _P, _Z, _P]
     so.int8_debug_set_activation_path.argtypes = [_I]
     so.int8_debug_set_activation_path.restype = None
+    so.int4_debug_set_product_path.argtypes = [_I]
+    so.int4_debug_set_product_path.restype = None
     so.int8_outlier_stats_workspace_size.argtypes = [_I]
     so.int8_outlier_stats_workspace_size.restype = _Z
     so.int8_outlier_stats.argtypes = [_P, _I, _I, _F, _P, _P, _P, _P, _P, _Z, _P]
@@ -251,6 +253,12 @@ def int8_debug_set_activation_path(mode):
     """1 (default): the one cooperative activation kernel for 8 <= T <= 128 when X fits in
     shared memory; 2: that kernel whenever X fits; 0: scan + quantiser."""
     lib().int8_debug_set_activation_path(int(mode))
+
+
+def int4_debug_set_product_path(mode):
+    """0 (default): int4_linear's product on the CUDA cores for T <= 2, else the tensor
+    cores; 1: always the tensor cores; 2: the CUDA cores whenever T <= 4."""
+    lib().int4_debug_set_product_path(int(mode))
 
 
 def int8_quantize_activation(X, alpha=6.0, with_xo=True, stream=None):

@@ -63,6 +63,8 @@ constexpr int CODE_BYTES = BN * BK / 2;     // 32 KB of packed codes per stage
 constexpr int SCALE_BYTES = BN * 16;        // 4 KB: four (s, lo) pairs per column
 constexpr int MAX_T = 64;
 constexpr int MAX_CTAS = 256;               // partial-sum slots are sized for up to this many CTAs
+constexpr int COUNTERS_PER_TILE = 8;        // split-tile counters: the tensor kernel uses 4 (one per quadrant),
+                                            // the CUDA-core kernel 8 (one per 32-column group)
 constexpr int MAX_STAGES = 6;
 constexpr int SUB = 2;                      // tensor-memory hand-offs of A per stage
 constexpr int KSUB = BK / SUB;              // K per hand-off
@@ -467,7 +469,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 return p.part + ((static_cast<size_t>(c) * 2 + slot_of(c)) * p.TP + t) * BN + hh * BMH + q * 32 + lane;
             };
             int mode = 0;                                   // 0: whole tile, 1: last piece, 2: store partial
-            int *counter = p.counters + tile * 4 + q;
+            int *counter = p.counters + tile * COUNTERS_PER_TILE + q;
             if (c1 > c0) {
                 int last_piece = 0;
                 if (lane == 0) last_piece = atomicAdd(counter, 0) == c1 - c0;
@@ -532,6 +534,258 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after_sync();
         tmem_dealloc(tmem, TMEM_COLS);
     }
+}
+
+// ------------------------------------------------------------------ product, few rows
+// For one or two rows of X the CUDA cores do better than the tensor path
+// above: per weight the work is the decode (13 instructions per 8 codes, the
+// same decode_word, so the same fp16 W~) and one mixed-precision fused
+// multiply-add per row (fma.rn.f32.f16: the fp16 product is exact in fp32,
+// one rounding per add, as in the tensor core's fp32 accumulation), where the
+// tensor path is bound by issuing MMAs.  The kernel is bound by instruction
+// issue (about 160 warp instructions per 1024 weights at T = 1), so each
+// further row costs about a third more; the host takes it for T <= 2.
+//   A stage is one (tile, 256 of K) unit as above: its packed codes and
+//   scales and the T rows of X over those 256 of K (bulk copies of 512 bytes),
+//   filled by one producer warp.  Sixteen compute warps: warp group g (0..7)
+//   takes columns 32g .. 32g+31 of the tile, one per lane, and half h of the
+//   stage's K (chunks 4h .. 4h+3, groups 2h and 2h+1).  Each lane keeps four
+//   fp32 sums per row (by pair parity and position, a fixed order).  At the
+//   end of a tile's run the h = 1 warps hand their sums to the h = 0 warps
+//   through shared memory (mbarriers, bounded waits), which add them and
+//   write Y, or for a tile split over CTAs store the piece in the CTA's slot
+//   and count it; the piece that completes the count adds the pieces in CTA
+//   order.
+constexpr int SMALL_T = 4;                  // instances exist for T = 1 .. SMALL_T
+constexpr int SMALL_WARPS = 16;
+constexpr int SMALL_THREADS = 32 * (1 + SMALL_WARPS);
+constexpr int SMALL_MAX_STAGES = 6;
+constexpr int SMALL_SMEM_BUDGET = 220 * 1024;
+constexpr int X_SLICE_BYTES = BK * 2;       // one row of X over a stage's K
+
+struct SmallBarriers {
+    uint64_t full[SMALL_MAX_STAGES];
+    uint64_t empty[SMALL_MAX_STAGES];
+    uint64_t red_full;
+    uint64_t red_empty;
+    int abort;
+};
+
+__host__ __device__ inline int small_stage_bytes(int T) { return CODE_BYTES + SCALE_BYTES + T * X_SLICE_BYTES; }
+__host__ __device__ inline size_t small_fixed_bytes(int T) {
+    return 128 + static_cast<size_t>(T) * BN * 4 + sizeof(SmallBarriers);
+}
+__host__ __device__ inline int small_stages(int T) {
+    const int s = static_cast<int>((SMALL_SMEM_BUDGET - small_fixed_bytes(T)) / small_stage_bytes(T));
+    return s < SMALL_MAX_STAGES ? s : SMALL_MAX_STAGES;
+}
+__host__ __device__ inline size_t small_smem_bytes(int T) {
+    return small_fixed_bytes(T) + static_cast<size_t>(small_stages(T)) * small_stage_bytes(T);
+}
+
+// c0 += lo(w) * lo(x), c1 += hi(w) * hi(x): fp16 operands, fp32 sums.
+__device__ __forceinline__ void fma_f16x2_f32(uint32_t w, uint32_t x, float &c0, float &c1) {
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %2;\n\t"
+        "mov.b32 {xl, xh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, wl, xl, %0;\n\t"
+        "fma.rn.f32.f16 %1, wh, xh, %1;\n\t}"
+        : "+f"(c0), "+f"(c1)
+        : "r"(w), "r"(x));
+}
+
+// One compute warp's share of a stage: column r of the tile, chunks 4H .. 4H+3
+// (groups 2H and 2H+1), every row of X; H is a constant so that the chunk,
+// scale and X offsets are immediates.
+template <int TT, int H>
+__device__ __forceinline__ void small_stage_math(const uint8_t *st, int r, float (&acc)[TT][4]) {
+    constexpr int XOFF = CODE_BYTES + SCALE_BYTES;
+    const uint2 sl = *reinterpret_cast<const uint2 *>(st + CODE_BYTES + r * 16 + H * 8);   // groups 2H, 2H+1
+    const uint8_t *col = st + r * 128;
+    const int sw = r & 7;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * H + cc;                           // chunk of the stage: codes 32c .. 32c+31
+        const __half2 sl2 = u32_as_h2(cc < 2 ? sl.x : sl.y);
+        const __half2 s2 = __half2half2(__low2half(sl2)), lo2 = __half2half2(__high2half(sl2));
+        const uint4 cw4 = *reinterpret_cast<const uint4 *>(col + ((c ^ sw) << 4));
+        uint32_t v[16];                                     // v[4i+j]: codes 8i+2j, 8i+2j+1 of the chunk
+        decode_word(cw4.x, s2, lo2, v);
+        decode_word(cw4.y, s2, lo2, v + 4);
+        decode_word(cw4.z, s2, lo2, v + 8);
+        decode_word(cw4.w, s2, lo2, v + 12);
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+            // x over the chunk's 32 codes: 64 bytes of row t's slice
+            const uint4 *xp = reinterpret_cast<const uint4 *>(st + XOFF + t * X_SLICE_BYTES + c * 64);
+            const uint4 x0 = xp[0], x1 = xp[1], x2 = xp[2], x3 = xp[3];
+            const uint32_t xv[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                     x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+                fma_f16x2_f32(v[e], xv[e], acc[t][0], acc[t][1]);
+                fma_f16x2_f32(v[e + 1], xv[e + 1], acc[t][2], acc[t][3]);
+            }
+        }
+    }
+}
+
+template <int TT>
+__global__ void __launch_bounds__(SMALL_THREADS, 1)
+    gemm_int4_small_kernel(const __half *__restrict__ X, const Params p) {
+    constexpr int XOFF = CODE_BYTES + SCALE_BYTES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+    float *red = reinterpret_cast<float *>(smem + static_cast<size_t>(p.stages) * p.stage_bytes);   // [TT][BN]
+    SmallBarriers *bars = reinterpret_cast<SmallBarriers *>(red + TT * BN);
+    volatile int *abort = &bars->abort;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&bars->full[s], 1);
+            mbar_init(&bars->empty[s], SMALL_WARPS);
+        }
+        mbar_init(&bars->red_full, SMALL_WARPS / 2);     // the h = 1 warps have stored their sums
+        mbar_init(&bars->red_empty, SMALL_WARPS / 2);    // the h = 0 warps have read them
+        bars->abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    const long long u0 = unit_begin(p.total_units, blockIdx.x, gridDim.x);
+    const long long u1 = unit_begin(p.total_units, blockIdx.x + 1, gridDim.x);
+    const int KT = p.KB;
+    const uint32_t tx = static_cast<uint32_t>(p.stage_bytes);
+
+    // the weight blocks of the first stages do not depend on earlier kernels
+    const int pre = static_cast<int>(min(static_cast<long long>(p.stages), u1 - u0));
+    if (warp == 0 && lane == 0) {
+        for (int i = 0; i < pre; ++i) {
+            const long long u = u0 + i;
+            const size_t blk = static_cast<size_t>(u / KT) * KT + static_cast<size_t>(u % KT);
+            uint8_t *st = smem + static_cast<size_t>(i) * p.stage_bytes;
+            mbar_arrive_expect_tx(&bars->full[i], tx);
+            bulk_load(st, p.W4 + blk * CODE_BYTES, CODE_BYTES, &bars->full[i]);
+            bulk_load(st + CODE_BYTES, p.S4 + blk * SCALE_BYTES, SCALE_BYTES, &bars->full[i]);
+        }
+    }
+    griddep_wait();                                         // X and the cleared counters
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        int pending[SMALL_MAX_STAGES];
+        for (int s = 0; s < SMALL_MAX_STAGES; ++s) pending[s] = -1;
+        int stage = 0, n = 0;
+        uint32_t phase = 0;
+        const bool ok = walk(p, u0, u1, [&](int tile, int kb, bool, bool) -> bool {
+            uint8_t *st = smem + static_cast<size_t>(stage) * p.stage_bytes;
+            uint64_t *fb = &bars->full[stage];
+            if (n >= pre) {
+                if (!warp_wait(&bars->empty[stage], phase ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+                if (lane == 0) {
+                    const size_t blk = static_cast<size_t>(tile) * KT + kb;
+                    mbar_arrive_expect_tx(fb, tx);
+                    bulk_load(st, p.W4 + blk * CODE_BYTES, CODE_BYTES, fb);
+                    bulk_load(st + CODE_BYTES, p.S4 + blk * SCALE_BYTES, SCALE_BYTES, fb);
+                }
+            }
+            if (lane == 0) {
+#pragma unroll
+                for (int t = 0; t < TT; ++t)
+                    bulk_load(st + XOFF + t * X_SLICE_BYTES, X + static_cast<size_t>(t) * p.K + static_cast<size_t>(kb) * BK,
+                              X_SLICE_BYTES, fb);
+                pending[stage] = static_cast<int>(phase);
+            }
+            ++n;
+            __syncwarp();
+            if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+            return true;
+        });
+        if (!ok && lane == 0) {
+            volatile int never = 0;
+            for (int s = 0; s < p.stages; ++s)
+                if (pending[s] >= 0) mbar_wait(&bars->full[s], static_cast<uint32_t>(pending[s]), &never, 0);
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- compute
+    const int cw = warp - 1;
+    const int h = cw >> 3, grp = cw & 7;
+    const int r = grp * 32 + lane;                          // column of the tile
+    float acc[TT][4];
+    int stage = 0, seg = 0;
+    uint32_t phase = 0;
+    walk(p, u0, u1, [&](int tile, int, bool first, bool last) -> bool {
+        if (first) {
+#pragma unroll
+            for (int t = 0; t < TT; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+        }
+        if (!warp_wait(&bars->full[stage], phase, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+        const uint8_t *st = smem + static_cast<size_t>(stage) * p.stage_bytes;
+        if (h == 0)
+            small_stage_math<TT, 0>(st, r, acc);
+        else
+            small_stage_math<TT, 1>(st, r, acc);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->empty[stage]);    // this warp's shared-memory reads are done
+        if (++stage == p.stages) { stage = 0; phase ^= 1u; }
+        if (!last) return true;
+
+        // the end of this CTA's run of the tile: the two halves of K meet
+        float y[TT];
+#pragma unroll
+        for (int t = 0; t < TT; ++t) y[t] = (acc[t][0] + acc[t][1]) + (acc[t][2] + acc[t][3]);
+        const uint32_t rph = static_cast<uint32_t>(seg & 1);
+        ++seg;
+        if (h == 1) {
+            if (!warp_wait(&bars->red_empty, rph ^ 1u, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+#pragma unroll
+            for (int t = 0; t < TT; ++t) red[t * BN + r] = y[t];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->red_full);
+            return true;
+        }
+        if (!warp_wait(&bars->red_full, rph, abort, I8R_DEV_PIPELINE_TIMEOUT)) return false;
+#pragma unroll
+        for (int t = 0; t < TT; ++t) y[t] += red[t * BN + r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->red_empty);
+
+        const long long tile_u0 = static_cast<long long>(tile) * p.KB;
+        const int c0 = unit_owner(p.total_units, tile_u0, gridDim.x);
+        const int c1 = unit_owner(p.total_units, tile_u0 + p.KB - 1, gridDim.x);
+        const int col = tile * BN + r;
+        if (c1 == c0) {
+            if (col < p.N)
+#pragma unroll
+                for (int t = 0; t < TT; ++t) p.Y[static_cast<size_t>(t) * p.N + col] = __float2half_rn(y[t]);
+            return true;
+        }
+        // the tile is c0's last run and the first of the others: slots 1 and 0
+        auto part_at = [&](int c, int t) {
+            return p.part + ((static_cast<size_t>(c) * 2 + (c == c0 ? 1 : 0)) * p.TP + t) * BN + r;
+        };
+#pragma unroll
+        for (int t = 0; t < TT; ++t) __stcg(part_at(blockIdx.x, t), y[t]);
+        __threadfence();
+        __syncwarp();
+        int done = 0;
+        if (lane == 0) done = atomicAdd(p.counters + tile * COUNTERS_PER_TILE + grp, 1) == c1 - c0;
+        if (__shfl_sync(0xFFFFFFFFu, done, 0)) {
+            __threadfence();
+            if (col < p.N)
+#pragma unroll
+                for (int t = 0; t < TT; ++t) {
+                    float sum = 0.0f;
+                    for (int c = c0; c <= c1; ++c) sum += __ldcg(part_at(c, t));
+                    p.Y[static_cast<size_t>(t) * p.N + col] = __float2half_rn(sum);
+                }
+        }
+        return true;
+    });
 }
 
 }  // namespace w4

@@ -63,6 +63,12 @@ struct DeviceInfo {
 // kernel whenever X fits, 0 always the scan + quantiser pair, 3 as 1 but with
 // the cooperative launch treated as refused (the fallback to the pair runs).
 std::atomic<int> g_activation_fused{1};
+// Which 4-bit product runs (int4_debug_set_product_path): 0 (default) the
+// CUDA-core kernel for T <= kInt4SmallRows, the tensor-core kernel above;
+// 1 always the tensor-core kernel; 2 the CUDA-core kernel whenever
+// T <= w4::SMALL_T.
+std::atomic<int> g_int4_path{0};
+constexpr int kInt4SmallRows = 2;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -112,6 +118,21 @@ CUcontext current_context() {
 // context, so the setup is done again whenever the calling thread's current
 // context is not the one it was done in (after cudaDeviceReset, or under a
 // context the caller made current).
+template <int TT>
+cudaError_t set_int4_small_attribute() {
+    return cudaFuncSetAttribute(w4::gemm_int4_small_kernel<TT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(w4::small_smem_bytes(TT)));
+}
+
+// Shared memory beyond 48 KB for every instance of the CUDA-core 4-bit product.
+i8r_status set_int4_small_attributes() {
+    I8R_CUDA(set_int4_small_attribute<1>());
+    I8R_CUDA(set_int4_small_attribute<2>());
+    I8R_CUDA(set_int4_small_attribute<3>());
+    I8R_CUDA(set_int4_small_attribute<4>());
+    return I8R_OK;
+}
+
 i8r_status device_setup(const DeviceInfo **out) {
     int dev = 0;
     I8R_CUDA(cudaGetDevice(&dev));
@@ -151,6 +172,7 @@ i8r_status device_setup(const DeviceInfo **out) {
                                           static_cast<int>(decode::SMEM_MAX)));
             I8R_CUDA(cudaFuncSetAttribute(w4::gemm_int4_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(w4::SMEM_BUDGET + 4096)));
+            I8R_TRY(set_int4_small_attributes());
             I8R_CUDA(cudaFuncSetAttribute(activation_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           static_cast<int>(kFusedSmemMax)));
             int per_sm = 0;
@@ -624,6 +646,17 @@ i8r_status launch_decode(const DeviceInfo *dev, const int8_t *Xq, int T, int K, 
     return I8R_OK;
 }
 
+// The CUDA-core 4-bit product's instances, T = 1 .. w4::SMALL_T rows.
+cudaError_t launch_int4_small(int T, unsigned grid, const __half *X, const w4::Params &p, cudaStream_t s) {
+    const dim3 g(grid), b(w4::SMALL_THREADS);
+    switch (T) {
+        case 1: return launch_dependent(w4::gemm_int4_small_kernel<1>, g, b, w4::small_smem_bytes(1), s, 1, X, p);
+        case 2: return launch_dependent(w4::gemm_int4_small_kernel<2>, g, b, w4::small_smem_bytes(2), s, 1, X, p);
+        case 3: return launch_dependent(w4::gemm_int4_small_kernel<3>, g, b, w4::small_smem_bytes(3), s, 1, X, p);
+        default: return launch_dependent(w4::gemm_int4_small_kernel<4>, g, b, w4::small_smem_bytes(4), s, 1, X, p);
+    }
+}
+
 // The group-wise 4-bit codec: shape rules and the product's workspace.
 i8r_status check_int4_shape(int K, int N) {
     if (K < 0 || N < 0) return I8R_EINVAL;
@@ -641,7 +674,7 @@ Int4Workspace int4_ws_layout(int T, int N) {
     const int TP = (T + 15) / 16 * 16;
     w.part = 0;
     w.counters = align_up(static_cast<size_t>(w4::MAX_CTAS) * 2 * TP * w4::BN * 4);
-    w.total = align_up(w.counters + static_cast<size_t>(w4::padded_n(N) / w4::BN) * 4 * 4);
+    w.total = align_up(w.counters + static_cast<size_t>(w4::padded_n(N) / w4::BN) * w4::COUNTERS_PER_TILE * 4);
     return w;
 }
 
@@ -843,6 +876,8 @@ size_t int8_mixed_linear_noalloc_max_workspace(void) { return kNoAllocScratchByt
 
 void int8_debug_set_activation_path(int mode) { g_activation_fused.store(mode < 0 ? 0 : (mode > 3 ? 3 : mode)); }
 
+void int4_debug_set_product_path(int mode) { g_int4_path.store(mode < 0 ? 0 : (mode > 2 ? 2 : mode)); }
+
 i8r_status int8_mixed_linear_noalloc(const void *X, int T, int K, const int8_t *Wq, const float *sW,
                                      const void *W16, int N, float alpha, void *Y, cudaStream_t stream) {
     I8R_TRY(check_shape(T, K, N, true));
@@ -1024,16 +1059,28 @@ i8r_status int4_linear(const void *X, int T, int K, const uint8_t *W4, const voi
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     p.part = reinterpret_cast<float *>(ws + w.part);
     p.counters = reinterpret_cast<int *>(ws + w.counters);
-    CUtensorMap map_x;
-    I8R_TRY(make_map(&map_x, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, p.TP, 64));
-    const int ncount = p.num_tiles * 4;
-    w4::int4_clear_kernel<<<(ncount + 255) / 256, 256, 0, stream>>>(p.counters, ncount);
-    I8R_LAUNCHED();
+    const int ncount = p.num_tiles * w4::COUNTERS_PER_TILE;
     const long long g = std::min<long long>(p.total_units, std::min(dev->sms, w4::MAX_CTAS));
-    record_before(stream);
-    cudaError_t e = launch_dependent(w4::gemm_int4_decode_kernel, dim3(static_cast<unsigned>(g)),
-                                     dim3(w4::THREADS), w4::smem_bytes(p.stages, p.stage_bytes), stream, 1,
-                                     map_x, p);
+    const int path = g_int4_path.load(std::memory_order_relaxed);
+    const bool small = path == 2 ? T <= w4::SMALL_T : (path == 0 && T <= kInt4SmallRows);
+    cudaError_t e;
+    if (small) {
+        // the CUDA-core product: a stage is the codes, the scales and T slices of X
+        p.stage_bytes = w4::small_stage_bytes(T);
+        p.stages = w4::small_stages(T);
+        w4::int4_clear_kernel<<<(ncount + 255) / 256, 256, 0, stream>>>(p.counters, ncount);
+        I8R_LAUNCHED();
+        record_before(stream);
+        e = launch_int4_small(T, static_cast<unsigned>(g), static_cast<const __half *>(X), p, stream);
+    } else {
+        CUtensorMap map_x;
+        I8R_TRY(make_map(&map_x, X, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, T, K, p.TP, 64));
+        w4::int4_clear_kernel<<<(ncount + 255) / 256, 256, 0, stream>>>(p.counters, ncount);
+        I8R_LAUNCHED();
+        record_before(stream);
+        e = launch_dependent(w4::gemm_int4_decode_kernel, dim3(static_cast<unsigned>(g)), dim3(w4::THREADS),
+                             w4::smem_bytes(p.stages, p.stage_bytes), stream, 1, map_x, p);
+    }
     if (e != cudaSuccess) {
         tl_last_cuda_error = static_cast<int>(e);
         return I8R_ECUDA;

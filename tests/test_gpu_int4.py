@@ -95,6 +95,74 @@ def test_int4_linear_matches_oracle(orc, T, K, N):
     assert device_status_clean()
 
 
+SMALL_CASES = [
+    # T, K, N: the CUDA-core product (T <= 4), each checked on both products
+    (1, 256, 16),
+    (2, 512, 272),          # ragged N
+    (3, 1024, 1024),
+    (4, 2048, 528),
+    (1, 12288, 2048),       # tiles split over several CTAs
+    (4, 4096, 12288),
+    (2, 49152, 256),        # one tile over every CTA
+]
+
+
+@pytest.mark.parametrize("T,K,N", SMALL_CASES)
+def test_int4_cuda_core_and_tensor_products_match_oracle(orc, T, K, N):
+    """Both products (int4_debug_set_product_path 2: CUDA cores, 1: tensor
+    cores) against the oracle, and against each other: the same decoded
+    weights and exact fp16 products, fp32 sums in different orders."""
+    rng = np.random.default_rng(T * 131 + K + N)
+    X = rng.standard_normal((T, K)).astype(np.float16)
+    W = _weights(rng, K, N)
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev(W))
+    Xd = to_dev(X)
+    codes_o, s_o, lo_o = orc.int4_quantize_groupwise(W)
+    Y_o, _ = orc.int4_linear(X, codes_o, s_o, lo_o)
+    out = {}
+    try:
+        for mode in (2, 1):
+            i8.int4_debug_set_product_path(mode)
+            out[mode] = to_host(i8.int4_linear(Xd, W4, S4, N))
+            assert_y_close(out[mode], Y_o, f"int4 path {mode} T={T} K={K} N={N}")
+            assert device_status_clean()
+    finally:
+        i8.int4_debug_set_product_path(0)
+    assert_y_close(out[2], out[1].astype(np.float64), f"int4 paths T={T} K={K} N={N}")
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+def test_int4_cuda_core_product_exact_integers(T):
+    """Integer activations and exact 4-bit grids on the CUDA-core product:
+    every product and partial sum is exact in fp32, so Y is exact."""
+    rng = np.random.default_rng(70 + T)
+    K, N = 2048, 768
+    Q = rng.integers(0, 16, (K, N))
+    Q[0::64] = 0
+    Q[1::64] = 15
+    W = (Q - 7).astype(np.float16)
+    X = rng.integers(-2, 3, (T, K)).astype(np.float16)
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev(W))
+    try:
+        i8.int4_debug_set_product_path(2)
+        Y = to_host(i8.int4_linear(to_dev(X), W4, S4, N)).astype(np.int64)
+    finally:
+        i8.int4_debug_set_product_path(0)
+    exact = X.astype(np.int64) @ (Q - 7)
+    assert np.abs(exact).max() <= 2048
+    assert np.array_equal(Y, exact)
+
+
+def test_int4_cuda_core_product_is_deterministic():
+    rng = np.random.default_rng(12)
+    T, K, N = 2, 12288, 4096                 # tiles split over CTAs: pieces added in CTA order
+    X = to_dev(rng.standard_normal((T, K)).astype(np.float16))
+    W4, S4 = i8.int4_quantize_weight_groupwise(to_dev((rng.standard_normal((K, N)) * 0.01).astype(np.float16)))
+    a = to_host(i8.int4_linear(X, W4, S4, N))
+    b = to_host(i8.int4_linear(X, W4, S4, N))
+    assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
+
+
 def test_int4_linear_exact_integers(orc):
     """Integer activations and weights on exact 4-bit grids: every product and
     partial sum is exact in fp32, so Y is the exact integer product."""
@@ -131,14 +199,16 @@ def test_int4_linear_t0_and_limits():
         i8.int4_linear(torch.zeros((65, 256), dtype=torch.float16, device="cuda"), W4, S4, 16)
 
 
-def test_int4_full_size_fc1_decode(orc):
-    """The 175B fc1 shape at T=16 (K=12288, N=49152; 302 MB of packed codes), in
-    the launch configuration the sweep times: every group's (s, lo) bit for bit,
-    and Y on sampled rows within the tolerance."""
+@pytest.mark.parametrize("T", [1, 16])
+def test_int4_full_size_fc1_decode(orc, T):
+    """The 175B fc1 shape (K=12288, N=49152; 302 MB of packed codes) at T=1 (the
+    CUDA-core product) and T=16 (the tensor cores), in the launch configuration
+    the sweep times: every group's (s, lo) bit for bit, and Y on sampled rows
+    within the tolerance."""
     from int8_quantized_row_b200 import workloads as wl
-    T, K, N = 16, 12288, 49152
+    K, N = 12288, 49152
     W = wl.make_w(K, N, 0.01)
-    X = wl.make_x(T, K, 0, seed=16)
+    X = wl.make_x(T, K, 0, seed=T)
     W4, S4 = i8.int4_quantize_weight_groupwise(to_dev(W))
     Y = to_host(i8.int4_linear(to_dev(X), W4, S4, N))
     codes_o, s_o, lo_o = orc.int4_quantize_groupwise(W)
@@ -146,7 +216,7 @@ def test_int4_full_size_fc1_decode(orc):
     sl = to_host(S4).reshape(NP // 256, KT, 256, 4, 2, 2).view("<u2")[..., 0].transpose(1, 3, 0, 2, 4).reshape(K // 64, NP, 2)
     assert np.array_equal(sl[:, :N, 0], s_o.view(np.uint16))
     assert np.array_equal(sl[:, :N, 1], lo_o.view(np.uint16))
-    rows = np.array([0, 7, 15], np.int32)
+    rows = np.array(sorted({0, T // 2, T - 1}), np.int32)
     Y_o, _ = orc.int4_linear(X, codes_o, s_o, lo_o, rows=rows)
-    assert_y_close(Y[rows], Y_o, "int4 fc1 T=16 full size")
+    assert_y_close(Y[rows], Y_o, f"int4 fc1 T={T} full size")
     assert device_status_clean()

@@ -163,11 +163,12 @@ def test_int4_cuda_core_product_is_deterministic():
     assert np.array_equal(a.view(np.uint16), b.view(np.uint16))
 
 
-def test_int4_linear_exact_integers(orc):
+@pytest.mark.parametrize("T", [16, 64])
+def test_int4_linear_exact_integers(orc, T):
     """Integer activations and weights on exact 4-bit grids: every product and
     partial sum is exact in fp32, so Y is the exact integer product."""
-    rng = np.random.default_rng(7)
-    T, K, N = 16, 1024, 512
+    rng = np.random.default_rng(7 + T)
+    K, N = 1024, 512
     Q = rng.integers(0, 16, (K, N))
     Q[0::64] = 0
     Q[1::64] = 15

@@ -283,6 +283,49 @@ def test_int8_gemm_bit_exact(T, K, N):
     assert device_status_clean()
 
 
+K_MAX = 133136      # the largest multiple of 16 with K * 127^2 < 2^31 (int32 accumulation exact)
+
+
+@pytest.mark.parametrize("T", [2, 130])
+def test_int8_gemm_at_the_largest_k(T):
+    """K = 133136, with a row of 127 codes against a column of 127 codes: the
+    accumulator K * 127^2 = 2147350544 is within 2^17 of INT32_MAX.  Decode
+    (T = 2) and prefill (T = 130) kernels, checked bit for bit against int64
+    sums on a few columns (all of them at T = 2)."""
+    K, N = K_MAX, 256
+    assert K * 127 * 127 < 2 ** 31 and K % 16 == 0
+    rng = np.random.default_rng(T + 1)
+    A = rng.integers(-127, 128, (T, K)).astype(np.int8)
+    B = rng.integers(-127, 128, (K, N)).astype(np.int8)
+    A[0, :] = 127
+    B[:, 0] = 127
+    A[T - 1, :] = -127                           # the most negative accumulator
+    acc = to_host(i8.int8_gemm_i8_s32(to_dev(A), to_dev(B))).astype(np.int64)
+    cols = np.arange(N) if T <= 16 else np.array([0, 1, 128, 255])
+    ref = A.astype(np.int64) @ B[:, cols].astype(np.int64)
+    assert ref[0, 0] == K * 127 * 127 and ref[T - 1, 0] == -K * 127 * 127
+    assert np.array_equal(acc[:, cols], ref)
+    assert device_status_clean()
+
+
+def test_mixed_linear_at_the_largest_k(orc):
+    """The whole layer at K = 133136 against the oracle (decode shape, outlier
+    columns spread over the whole K)."""
+    T, K, N = 2, K_MAX, 256
+    rng = np.random.default_rng(2)
+    X = outlier_x(rng, T, K, [0, 70000, K - 1])
+    W = (rng.standard_normal((K, N)) * 0.01).astype(np.float16)
+    Wq_o, sW_o = orc.quantize_weight_colwise(W)
+    Wd = to_dev(W)
+    Wq, sW = i8.int8_quantize_weight_colwise(Wd)
+    assert np.array_equal(to_host(Wq), Wq_o) and np.array_equal(to_host(sW), sW_o)
+    Y = to_host(i8.int8_mixed_linear(to_dev(X), Wq, sW, Wd, 6.0))
+    Y_o, _, _, cnt = orc.mixed_linear(X, Wq_o, sW_o, W, 6.0)
+    assert cnt == 3
+    assert_y_close(Y, Y_o, f"K={K}")
+    assert device_status_clean()
+
+
 def test_int8_gemm_against_oracle_accumulators(orc):
     rng = np.random.default_rng(99)
     X = outlier_x(rng, 200, 1024, [3, 500])

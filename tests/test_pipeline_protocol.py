@@ -1,0 +1,293 @@
+"""The mbarrier hand-off protocols of the 4-bit product kernels, model-checked
+on the CPU under random interleavings.
+
+A GPU run only samples the interleavings its warps happen to take.  Here
+each role of a kernel (producer, compute or decoder warps, MMA issuer,
+epilogue) is a Python generator that issues the same barrier operations as
+the kernel in the same order.  The barriers follow the mbarrier rules: a
+phase completes when its pending arrivals and its transaction bytes both
+reach zero; a parity wait succeeds once the phase of that parity has
+completed.  Bulk copies and MMAs complete asynchronously, at random later
+points.  Each shared buffer holds a tag of what was last written to it; every
+read checks that the tag is the one the reader expects, so a refill that
+overtakes a reader, or a reader that runs ahead of its data, fails.  Runs
+that stop with roles still waiting are deadlocks.
+
+The schedules are those of the kernels: stream-K ranges of (tile, k-block)
+units over the CTAs, walked as runs of one tile (first and last flags); the
+split of one CTA's range is what matters, so one CTA is modelled.  Planted
+protocol mistakes (an empty barrier that counts one consumer too few, a
+hand-off without its wait) must be caught, which shows that the checks can
+fail.
+"""
+import random
+
+import pytest
+
+
+class Barrier:
+    def __init__(self, count, name):
+        self.count, self.pending, self.tx, self.phase, self.name = count, count, 0, 0, name
+
+    def arrive(self, tx=0):
+        self.tx += tx
+        self.pending -= 1
+        if self.pending < 0:
+            raise Stale(f"{self.name}: more arrivals than its count")
+        self._settle()
+
+    def complete_tx(self, nbytes):
+        self.tx -= nbytes
+        self._settle()
+
+    def _settle(self):
+        if self.pending == 0 and self.tx == 0:
+            self.phase ^= 1
+            self.pending = self.count
+
+    def passed(self, parity):
+        # the phase with this parity has completed (a fresh barrier has "completed" parity 1)
+        return self.phase != parity
+
+
+class Stale(AssertionError):
+    pass
+
+
+def run(roles, seed, max_steps=200000):
+    """Interleave the generators at random; asynchronous completions are
+    extra runnable events.  Raises Stale on a wrong read, RuntimeError on a
+    deadlock."""
+    rng = random.Random(seed)
+    mem = {}
+    events = []                                   # callables: bulk-copy completions, in any order
+    commits = {}                                  # role -> its MMA commits, completing in issue order
+    live = {i: (g, None) for i, g in enumerate(roles)}
+    for i in list(live):
+        live[i] = (live[i][0], next(live[i][0], None))
+    for _ in range(max_steps):
+        ready = [i for i, (g, op) in live.items() if op is not None and (op[0] != "wait" or op[1].passed(op[2]))]
+        choices = ([("role", i) for i in ready] + [("event", j) for j in range(len(events))]
+                   + [("commit", i) for i, q in commits.items() if q])
+        if not choices:
+            if all(op is None for _, op in live.values()):
+                return
+            waiting = [f"{op[1].name}@{op[2]}" for _, op in live.values() if op is not None]
+            raise RuntimeError("deadlock: roles wait on " + ", ".join(waiting))
+        kind, k = rng.choice(choices)
+        if kind == "event":
+            events.pop(k)(mem)
+            continue
+        if kind == "commit":
+            commits[k].pop(0)(mem)
+            continue
+        g, op = live[k]
+        res = None
+        if op[0] == "arrive":                     # ("arrive", bar[, tx])
+            op[1].arrive(op[2] if len(op) > 2 else 0)
+        elif op[0] == "copy":                     # ("copy", bar, nbytes, key, tag): completes later
+            _, bar, nbytes, key, tag = op
+            events.append(lambda m, bar=bar, nbytes=nbytes, key=key, tag=tag: (m.__setitem__(key, tag),
+                                                                               bar.complete_tx(nbytes)))
+        elif op[0] == "commit":
+            # ("commit", bar, [reads]): the MMAs issued since the last commit read
+            # their operands, then the barrier gets an arrival.  A commit tracks
+            # every earlier MMA of the issuing thread, so one role's commits
+            # complete in the order they were issued.
+            _, bar, reads = op
+
+            def done(m, bar=bar, reads=reads):
+                for key, tag in reads:
+                    if m.get(key) != tag:
+                        raise Stale(f"MMA read {key}: {m.get(key)} instead of {tag}")
+                bar.arrive()
+            commits.setdefault(k, []).append(done)
+        elif op[0] == "write":
+            mem[op[1]] = op[2]
+        elif op[0] == "read":
+            if mem.get(op[1]) != op[2]:
+                raise Stale(f"read {op[1]}: {mem.get(op[1])} instead of {op[2]}")
+        elif op[0] != "wait":
+            raise ValueError(op)
+        live[k] = (g, g.send(res) if res is not None else next(g, None))
+    raise RuntimeError("step limit")
+
+
+def units_of(total, ctas, c, KB):
+    """CTA c's stream-K range as (tile, kb, first, last) steps."""
+    u0, u1 = total * c // ctas, total * (c + 1) // ctas
+    out, u = [], u0
+    while u < u1:
+        tile = u // KB
+        end = min(u1, (tile + 1) * KB)
+        for v in range(u, end):
+            out.append((tile, v - tile * KB, v == u, v == end - 1))
+        u = end
+    return out
+
+
+# ---------------------------------------------------------------- the CUDA-core product
+
+def small_kernel_roles(steps, stages, groups, empty_short=0, skip_red_empty=False, early_refill=False):
+    """Producer + compute warps (2 halves x `groups` column groups) of
+    gemm_int4_small_kernel.  empty_short, skip_red_empty and early_refill
+    plant mistakes."""
+    full = [Barrier(1, f"full{s}") for s in range(stages)]
+    empty = [Barrier(2 * groups - empty_short, f"empty{s}") for s in range(stages)]
+    red_full, red_empty = Barrier(groups, "red_full"), Barrier(groups, "red_empty")
+
+    def producer():
+        for n, (tile, kb, _, _) in enumerate(steps):
+            s, ph = n % stages, (n // stages) & 1
+            if n >= stages and not (early_refill and n == stages):
+                yield ("wait", empty[s], ph ^ 1)
+            yield ("arrive", full[s], 2)          # arrive.expect_tx: codes+scales, then X
+            yield ("copy", full[s], 1, ("w", s), n)
+            yield ("copy", full[s], 1, ("x", s), n)
+
+    def compute(h, grp):
+        seg = 0
+        for n, (tile, kb, first, last) in enumerate(steps):
+            s, ph = n % stages, (n // stages) & 1
+            yield ("wait", full[s], ph)
+            yield ("read", ("w", s), n)
+            yield ("read", ("x", s), n)
+            yield ("arrive", empty[s])
+            if last:
+                rph = seg & 1
+                if h == 1:
+                    if not skip_red_empty:
+                        yield ("wait", red_empty, rph ^ 1)
+                    yield ("write", ("red", grp), seg)
+                    yield ("arrive", red_full)
+                else:
+                    yield ("wait", red_full, rph)
+                    yield ("read", ("red", grp), seg)
+                    yield ("arrive", red_empty)
+                seg += 1
+
+    return [producer()] + [compute(h, g) for h in (0, 1) for g in range(groups)]
+
+
+SCHEDULES = [
+    # total units, CTAs, CTA modelled, k-blocks per tile, stages
+    (12, 1, 0, 4, 2),       # three whole tiles
+    (50, 7, 3, 6, 3),       # pieces of tiles at both ends
+    (40, 3, 1, 40, 2),      # one tile over several CTAs
+    (9, 9, 4, 1, 2),        # one unit: first and last at once
+    (60, 4, 2, 3, 5),       # short tiles, deep ring
+]
+
+
+@pytest.mark.parametrize("total,ctas,c,KB,stages", SCHEDULES)
+def test_small_kernel_protocol(total, ctas, c, KB, stages):
+    steps = units_of(total, ctas, c, KB)
+    for seed in range(150):
+        run(small_kernel_roles(steps, stages, groups=2), seed)
+
+
+CAUGHT = (Stale, RuntimeError)                    # a wrong read, or a deadlock
+
+
+def test_small_kernel_protocol_catches_planted_mistakes():
+    steps = units_of(60, 2, 0, 5)
+    with pytest.raises(CAUGHT):                   # a refill that does not wait for every compute warp
+        for seed in range(300):
+            run(small_kernel_roles(steps, 2, groups=2, empty_short=1), seed)
+    with pytest.raises(Stale):                    # the first reuse of a stage without its empty wait
+        for seed in range(300):
+            run(small_kernel_roles(steps, 2, groups=2, early_refill=True), seed)
+    with pytest.raises(CAUGHT):                   # the second half overwriting sums not yet read
+        for seed in range(300):
+            run(small_kernel_roles(units_of(60, 1, 0, 1), 2, groups=2, skip_red_empty=True), seed)
+
+
+# ---------------------------------------------------------------- the tensor-core product
+
+def tensor_kernel_roles(steps, stages, na, decoders=2, issuers=2, sub=2, empty_short=0):
+    """Producer, decoder warps, MMA issuers and epilogue warps of
+    gemm_int4_decode_kernel: decoders fill a ring of `na` tensor-memory A
+    buffers (`sub` per stage); each issuer's MMAs read A and X and commit to
+    the A buffer's and the stage's empty barriers (asynchronously, when the
+    MMAs complete), and to an accumulator's full barrier at a tile run's end;
+    the epilogue drains the accumulator (two in turn)."""
+    full = [Barrier(1, f"full{s}") for s in range(stages)]
+    empty = [Barrier(decoders + issuers - empty_short, f"empty{s}") for s in range(stages)]
+    a_full = [Barrier(decoders, f"a_full{b}") for b in range(na)]
+    a_empty = [Barrier(issuers, f"a_empty{b}") for b in range(na)]
+    t_full = [Barrier(issuers, f"tmem_full{d}") for d in range(2)]
+    t_empty = [Barrier(1, f"tmem_empty{d}") for d in range(2)]
+
+    def producer():
+        for n, _ in enumerate(steps):
+            s, ph = n % stages, (n // stages) & 1
+            if n >= stages:
+                yield ("wait", empty[s], ph ^ 1)
+            yield ("arrive", full[s], 2)
+            yield ("copy", full[s], 1, ("codes", s), n)
+            yield ("copy", full[s], 1, ("x", s), n)
+
+    def decoder(w):
+        a, aph = 0, 0
+        for n, _ in enumerate(steps):
+            s, ph = n % stages, (n // stages) & 1
+            yield ("wait", full[s], ph)
+            yield ("read", ("codes", s), n)
+            yield ("arrive", empty[s])
+            for b in range(sub):
+                yield ("wait", a_empty[a], aph ^ 1)
+                yield ("write", ("A", a, w), (n, b))
+                yield ("arrive", a_full[a])
+                a += 1
+                if a == na:
+                    a, aph = 0, aph ^ 1
+
+    def issuer(i):
+        a, aph, seg, tph = 0, 0, 0, 0
+        for n, (_, _, first, last) in enumerate(steps):
+            s, ph = n % stages, (n // stages) & 1
+            d = seg & 1
+            if first:
+                yield ("wait", t_empty[d], ((tph >> d) & 1) ^ 1)
+            yield ("wait", full[s], ph)
+            for b in range(sub):
+                yield ("wait", a_full[a], aph)
+                reads = [(("A", a, w), (n, b)) for w in range(decoders)] + [(("x", s), n)]
+                yield ("commit", a_empty[a], reads)
+                a += 1
+                if a == na:
+                    a, aph = 0, aph ^ 1
+            yield ("commit", empty[s], [(("x", s), n)])
+            if last:
+                yield ("commit", t_full[d], [])
+                tph ^= 1 << d
+                seg += 1
+
+    def epilogue():
+        seg, tph = 0, 0
+        for n, (_, _, _, last) in enumerate(steps):
+            if not last:
+                continue
+            d = seg & 1
+            yield ("wait", t_full[d], (tph >> d) & 1)
+            yield ("arrive", t_empty[d])
+            tph ^= 1 << d
+            seg += 1
+
+    return ([producer()] + [decoder(w) for w in range(decoders)] + [issuer(i) for i in range(issuers)]
+            + [epilogue()])
+
+
+@pytest.mark.parametrize("total,ctas,c,KB,stages", SCHEDULES)
+@pytest.mark.parametrize("na", [2, 3])
+def test_tensor_kernel_protocol(total, ctas, c, KB, stages, na):
+    steps = units_of(total, ctas, c, KB)
+    for seed in range(60):
+        run(tensor_kernel_roles(steps, stages, na), seed)
+
+
+def test_tensor_kernel_protocol_catches_a_premature_refill():
+    steps = units_of(40, 1, 0, 4)
+    with pytest.raises(CAUGHT):
+        for seed in range(300):
+            run(tensor_kernel_roles(steps, 2, 2, empty_short=1), seed)

@@ -90,16 +90,19 @@ def run(roles, seed, max_steps=200000):
             events.append(lambda m, bar=bar, nbytes=nbytes, key=key, tag=tag: (m.__setitem__(key, tag),
                                                                                bar.complete_tx(nbytes)))
         elif op[0] == "commit":
-            # ("commit", bar, [reads]): the MMAs issued since the last commit read
-            # their operands, then the barrier gets an arrival.  A commit tracks
-            # every earlier MMA of the issuing thread, so one role's commits
-            # complete in the order they were issued.
-            _, bar, reads = op
+            # ("commit", bar, [reads], [writes]): the MMAs issued since the last
+            # commit read their operands and write their accumulators, then the
+            # barrier gets an arrival.  A commit tracks every earlier MMA of the
+            # issuing thread, so one role's commits complete in issue order.
+            bar, reads = op[1], op[2]
+            writes = op[3] if len(op) > 3 else []
 
-            def done(m, bar=bar, reads=reads):
+            def done(m, bar=bar, reads=reads, writes=writes):
                 for key, tag in reads:
                     if m.get(key) != tag:
                         raise Stale(f"MMA read {key}: {m.get(key)} instead of {tag}")
+                for key, tag in writes:
+                    m[key] = tag
                 bar.arrive()
             commits.setdefault(k, []).append(done)
         elif op[0] == "write":
@@ -291,3 +294,124 @@ def test_tensor_kernel_protocol_catches_a_premature_refill():
     with pytest.raises(CAUGHT):
         for seed in range(300):
             run(tensor_kernel_roles(steps, 2, 2, empty_short=1), seed)
+
+
+# ---------------------------------------------------------------- the int8 decode GEMM
+
+def decode_visits(total, ctas, c, KB, nob):
+    """walk_stages of gemm_decode_kernel for CTA c: a run that starts a tile
+    opens with the tile's nob outlier stages (kind 1, a segment of their own),
+    then the run's weight stages (kind 0, one segment)."""
+    out = []
+    for tile, kb, first, last in units_of(total, ctas, c, KB):
+        if kb == 0 and first:
+            out += [(1, tile, b, b == 0, b == nob - 1) for b in range(nob)]
+        out.append((0, tile, kb, first, last))
+    return out
+
+
+def decode_kernel_roles(visits, stages, nbuf, pre, two_producers=False):
+    """Producer, MMA issuer and four epilogue warps of gemm_decode_kernel:
+    one ring of stages for weight and outlier stages alike; the first `pre`
+    weight stages are armed and requested before the programmatic wait, their
+    X tiles after it; accumulator buffers seg % nbuf, each drained by the
+    epilogue before the MMAs of a later segment reuse it.  two_producers
+    plants the earlier design in which a second warp filled the outlier
+    stages and skipped the weight slots."""
+    full = [Barrier(1, f"full{s}") for s in range(stages)]
+    empty = [Barrier(1, f"empty{s}") for s in range(stages)]
+    t_full = [Barrier(1, f"tmem_full{b}") for b in range(nbuf)]
+    t_empty = [Barrier(4, f"tmem_empty{b}") for b in range(nbuf)]
+
+    # the first `pre` visits are weight stages in slots 0 .. pre-1 (the kernel
+    # requests none early when its range may open with outlier stages)
+    assert all(visits[i][0] == 0 for i in range(min(pre, len(visits))))
+
+    def producer(kinds):
+        if 0 in kinds:
+            for i in range(pre):                       # before griddepcontrol.wait
+                yield ("arrive", full[i], 2)
+                yield ("copy", full[i], 1, ("w", i), i)
+        stage, phase, n = 0, 0, 0
+        for v, (kind, tile, j, _, _) in enumerate(visits):
+            if kind in kinds:
+                if kind == 0 and n < pre:
+                    yield ("copy", full[stage], 1, ("x", stage), v)
+                else:
+                    yield ("wait", empty[stage], phase ^ 1)
+                    yield ("arrive", full[stage], 2)
+                    yield ("copy", full[stage], 1, ("w", stage), v)
+                    yield ("copy", full[stage], 1, ("x", stage), v)
+            if kind == 0:
+                n += 1
+            stage += 1
+            if stage == stages:
+                stage, phase = 0, phase ^ 1
+
+    def issuer():
+        stage, phase, seg, tph = 0, 0, 0, 0
+        for v, (kind, tile, j, first, last) in enumerate(visits):
+            buf = seg % nbuf
+            if first:
+                yield ("wait", t_empty[buf], ((tph >> buf) & 1) ^ 1)
+            yield ("wait", full[stage], phase)
+            yield ("commit", empty[stage], [(("w", stage), v), (("x", stage), v)], [(("D", buf), ("partial", seg))])
+            if last:
+                yield ("commit", t_full[buf], [], [(("D", buf), ("done", seg))])
+                tph ^= 1 << buf
+                seg += 1
+            stage += 1
+            if stage == stages:
+                stage, phase = 0, phase ^ 1
+
+    def epilogue():
+        seg, tph = 0, 0
+        for kind, tile, j, first, last in visits:
+            if not last:
+                continue
+            buf = seg % nbuf
+            yield ("wait", t_full[buf], (tph >> buf) & 1)
+            yield ("read", ("D", buf), ("done", seg))
+            yield ("arrive", t_empty[buf])
+            tph ^= 1 << buf
+            seg += 1
+
+    producers = [producer({0}), producer({1})] if two_producers else [producer({0, 1})]
+    return producers + [issuer()] + [epilogue() for _ in range(4)]
+
+
+DECODE_SCHEDULES = [
+    # total units, CTAs, CTA modelled, k-blocks per tile, outlier stages, ring stages, buffers
+    (24, 2, 0, 6, 2, 3, 2),     # starts two tiles: outlier segments, no early requests
+    (24, 5, 2, 6, 3, 2, 4),     # starts mid-tile, then a tile with outliers
+    (40, 1, 0, 5, 1, 5, 3),     # ring wraps many times around segments of different kinds
+    (30, 3, 1, 30, 4, 2, 2),    # one tile over several CTAs, this CTA's piece mid-tile
+    (18, 1, 0, 3, 0, 4, 4),     # no outliers
+]
+
+
+def _pre(visits, stages, KB, total, ctas, c):
+    u0 = total * c // ctas
+    if visits and visits[0][0] == 1:
+        return 0
+    first_seg = min(total * (c + 1) // ctas, (u0 // KB + 1) * KB) - u0
+    return min(stages, first_seg)
+
+
+@pytest.mark.parametrize("total,ctas,c,KB,nob,stages,nbuf", DECODE_SCHEDULES)
+def test_decode_kernel_protocol(total, ctas, c, KB, nob, stages, nbuf):
+    visits = decode_visits(total, ctas, c, KB, nob)
+    pre = _pre(visits, stages, KB, total, ctas, c)
+    for seed in range(150):
+        run(decode_kernel_roles(visits, stages, nbuf, pre), seed)
+
+
+def test_decode_kernel_protocol_catches_the_two_producer_design():
+    """The design that faulted on the GPU: weight and outlier stages of one ring
+    filled by two warps, each skipping the other's slots.  A parity wait cannot
+    tell a phase from the one two laps later, so the outlier producer can pass
+    the consumer and overwrite a live stage."""
+    visits = decode_visits(60, 1, 0, 4, 3)
+    with pytest.raises(CAUGHT):
+        for seed in range(400):
+            run(decode_kernel_roles(visits, 2, 2, 0, two_producers=True), seed)

@@ -1,4 +1,4 @@
-"""The mbarrier hand-off protocols of the 4-bit product kernels, model-checked
+"""The mbarrier hand-off protocols of the GEMM kernels, model-checked
 on the CPU under random interleavings.
 
 A GPU run only samples the interleavings its warps happen to take.  Here
@@ -415,3 +415,121 @@ def test_decode_kernel_protocol_catches_the_two_producer_design():
     with pytest.raises(CAUGHT):
         for seed in range(400):
             run(decode_kernel_roles(visits, 2, 2, 0, two_producers=True), seed)
+
+
+# ---------------------------------------------------------------- the int8 prefill GEMM (CTA pairs)
+
+def prefill_visits(tiles, KB, nob, defer=4):
+    """walk_schedule of gemm_prefill_pair_kernel for one cluster, `tiles`
+    tiles in turn (it = 0, 1, ...): each tile's K-blocks, and a tile's
+    outlier stages deferred into the next tile's after `defer` K-blocks (the
+    last tile's at the end)."""
+    defer = min(KB, defer)
+    out, prev = [], -1
+    for it in range(tiles):
+        for kb in range(KB):
+            out.append((0, it, kb))
+            if kb + 1 == defer and prev >= 0:
+                out += [(1, prev, ob) for ob in range(nob)]
+                prev = -1
+        prev = it
+    if prev >= 0:
+        out += [(1, prev, ob) for ob in range(nob)]
+    return out
+
+
+def prefill_kernel_roles(visits, tiles, KB, nob, stages, skip_conv_wait=False, skip_empty_wait=False):
+    """The two CTAs' producers, the leader's MMA issuer and the 2 x 4 epilogue
+    warps of gemm_prefill_pair_kernel.  Both producers' copies complete on the
+    leader's full barrier (armed by the leader with both CTAs' bytes); the
+    MMAs commit to both CTAs' empty, int_full and final_full barriers; the
+    epilogue warps of both CTAs arrive on the leader's acc_conv and acc_empty
+    (8 arrivals).  The accumulator of tile `it` is buffer it % 2; with
+    outliers the epilogue rewrites it in place (int32 -> scaled fp32) before
+    the deferred outlier MMAs accumulate onto it.  skip_conv_wait plants an
+    outlier MMA that does not wait for the conversion, skip_empty_wait a tile
+    that does not wait for its accumulator to be drained."""
+    full = [Barrier(1, f"full{s}") for s in range(stages)]
+    empty = [[Barrier(1, f"empty{r}.{s}") for s in range(stages)] for r in range(2)]
+    int_full = [[Barrier(1, f"int_full{r}.{b}") for b in range(2)] for r in range(2)]
+    fin_full = [[Barrier(1, f"final_full{r}.{b}") for b in range(2)] for r in range(2)]
+    acc_conv = [Barrier(8, f"acc_conv{b}") for b in range(2)]
+    acc_empty = [Barrier(8, f"acc_empty{b}") for b in range(2)]
+    D = [(r, b, q) for r in range(2) for b in range(2) for q in range(4)]
+
+    def producer(rank):
+        for v, _ in enumerate(visits):
+            s, ph = v % stages, (v // stages) & 1
+            if v >= stages:
+                yield ("wait", empty[rank][s], ph ^ 1)
+            if rank == 0:
+                yield ("arrive", full[s], 2)
+            yield ("copy", full[s], 1, ("half", rank, s), v)
+
+    def issuer():
+        for v, (kind, it, blk) in enumerate(visits):
+            s, ph = v % stages, (v // stages) & 1
+            buf, use = it & 1, (it >> 1) & 1
+            if kind == 0 and blk == 0 and not skip_empty_wait:
+                yield ("wait", acc_empty[buf], use ^ 1)
+            if kind == 1 and blk == 0 and not skip_conv_wait:
+                yield ("wait", acc_conv[buf], use)
+            yield ("wait", full[s], ph)
+            reads = [(("half", r, s), v) for r in range(2)]
+            if kind == 0:
+                writes = [(("D",) + d, ("int", it)) for d in D if d[1] == buf]
+            else:
+                reads += [(("D",) + d, ("conv", it) if blk == 0 else ("outl", it)) for d in D if d[1] == buf]
+                writes = [(("D",) + d, ("outl", it)) for d in D if d[1] == buf]
+            for r in range(2):
+                yield ("commit", empty[r][s], reads if r == 0 else [], writes if r == 0 else [])
+            if kind == 0 and blk == KB - 1:
+                for r in range(2):
+                    yield ("commit", int_full[r][buf], [])
+            if kind == 1 and blk == nob - 1:
+                for r in range(2):
+                    yield ("commit", fin_full[r][buf], [])
+
+    def epilogue(rank, q):
+        for it in range(tiles):
+            buf, use = it & 1, (it >> 1) & 1
+            key = ("D", rank, buf, q)
+            yield ("wait", int_full[rank][buf], use)
+            yield ("read", key, ("int", it))
+            if nob:
+                yield ("write", key, ("conv", it))
+                yield ("arrive", acc_conv[buf])
+                yield ("wait", fin_full[rank][buf], use)
+                yield ("read", key, ("outl", it))
+            yield ("arrive", acc_empty[buf])
+
+    return ([producer(0), producer(1), issuer()]
+            + [epilogue(r, q) for r in range(2) for q in range(4)])
+
+
+PREFILL_SCHEDULES = [
+    # tiles of this cluster, K-blocks per tile, outlier stages, ring stages (3 in the kernel)
+    (5, 6, 2, 3),
+    (4, 2, 3, 3),      # fewer K-blocks than the deferral: outlier stages after the next tile's last
+    (6, 5, 0, 3),      # no outliers
+    (1, 4, 1, 3),      # one tile: its outlier stages at the end
+    (7, 8, 4, 2),
+]
+
+
+@pytest.mark.parametrize("tiles,KB,nob,stages", PREFILL_SCHEDULES)
+def test_prefill_kernel_protocol(tiles, KB, nob, stages):
+    visits = prefill_visits(tiles, KB, nob)
+    for seed in range(100):
+        run(prefill_kernel_roles(visits, tiles, KB, nob, stages), seed)
+
+
+def test_prefill_kernel_protocol_catches_planted_mistakes():
+    visits = prefill_visits(4, 3, 2)
+    with pytest.raises(Stale):                    # outlier MMAs onto an unconverted accumulator
+        for seed in range(300):
+            run(prefill_kernel_roles(visits, 4, 3, 2, 3, skip_conv_wait=True), seed)
+    visits = prefill_visits(5, 2, 0)
+    with pytest.raises(Stale):                    # a tile's MMAs over an accumulator not yet drained
+        for seed in range(300):
+            run(prefill_kernel_roles(visits, 5, 2, 0, 3, skip_empty_wait=True), seed)

@@ -524,6 +524,24 @@ def pin_int4_nearest_level(o):
                 assert d <= best + s * Fraction(1, 2 ** 20), (g, n, i)
 
 
+def pin_int4_ties_round_away_from_zero(o):
+    """Exact halfway weights: a group spanning 0 .. 15 has step s = 1 (exact in
+    binary16, reciprocal exact in fp32) and base 0, so w = k + 1/2 gives
+    (w - lo) / s = k + 1/2 exactly, and the codec's rounding (half away from
+    zero, the same rule as the int8 codes) must give k + 1.  Scaled by 2^-4
+    (s = 1/16) the same holds.  Ties to even would give k for even k."""
+    for scale in (1.0, 1.0 / 16.0):
+        col = np.zeros(64, np.float64)
+        col[0], col[1] = 0.0, 15.0                     # the group's minimum and maximum
+        halves = np.arange(15) + 0.5                   # 0.5, 1.5, ..., 14.5
+        col[2:17] = halves
+        W = (col * scale).astype(np.float16).reshape(64, 1)
+        assert np.array_equal(W.astype(np.float64).ravel(), col * scale)     # all exact in binary16
+        codes, step, lo = o.int4_quantize_groupwise(np.repeat(W, 16, axis=1), 64)
+        assert float(step[0, 0]) == scale and float(lo[0, 0]) == 0.0
+        assert np.array_equal(codes[2:17, 0].astype(np.int64), np.arange(15) + 1), codes[2:17, 0]
+
+
 def pin_int4_invariants(o):
     """A constant group has step 0 and decodes exactly; scaling a column by 2^j
     (no binary16 overflow or underflow) leaves its codes unchanged and scales step,

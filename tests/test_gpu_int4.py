@@ -26,6 +26,12 @@ def _weights(rng, K, N, sigma=0.02):
     W[64:128, 1] = 0                                     # an all-zero group
     W[0:64, 2] = np.where(np.arange(64) % 2 == 0, np.float16(0.0), np.float16(-0.0))   # signed zeros
     W[128:192, 3] = (rng.standard_normal(64) * 40).astype(np.float16)                 # a wide group
+    if N > 4:
+        # exact halfway points: step 1/16, base 0, w - lo = (k + 1/2) * s
+        tie = np.zeros(64)
+        tie[1] = 15.0
+        tie[2:17] = np.arange(15) + 0.5
+        W[0:64, 4] = (tie / 16.0).astype(np.float16)
     return W
 
 

@@ -47,6 +47,17 @@ MUTANTS = {
     "int4_decode_drops_lo": ("+ (double)orc_half_to_float(lo[gi]);", "+ 0.0;"),
     "int4_product_wrong_row": ("const uint16_t *wrow = Wd + (size_t)k * N;",
                                "const uint16_t *wrow = Wd + (size_t)(k ^ 1) * N;"),
+    # sign and extremum slips
+    "outlier_test_signed": ("if (fabsf(orc_half_to_float(X[(size_t)t * K + k])) >= alpha)\n                is_outlier[k] = 1;",
+                            "if (orc_half_to_float(X[(size_t)t * K + k]) >= alpha)\n                is_outlier[k] = 1;"),
+    "row_scale_signed_max": ("float a = fabsf(orc_half_to_float(xrow[k]));", "float a = orc_half_to_float(xrow[k]);"),
+    "int4_lo_first_not_min": ("if (w < lo) lo = w;", "if (k == g * G) lo = w;"),
+    # the 4-bit codec's rounding steps
+    "int4_code_ties_to_even": ("float r = orc_rhaz(d * inv);", "float r = nearbyintf(d * inv);"),
+    "int4_codes_from_unrounded_step": ("float s = orc_half_to_float(s16);", "float s = range / 15.0f;"),
+    "int4_decode_two_roundings": ("double v = (double)codes[(size_t)k * N + n] * (double)orc_half_to_float(scale[gi])",
+                                  "double v = (double)orc_half_to_float(orc_double_to_half((double)codes[(size_t)k * N + n]"
+                                  " * (double)orc_half_to_float(scale[gi])))"),
 }
 
 

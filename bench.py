@@ -305,11 +305,37 @@ def max_over_ranks(pg, value, device):
 
 # ------------------------------------------------------------------ CPU oracle timing
 
-def cpu_threads():
+def host_cores():
     try:
         return len(os.sched_getaffinity(0))
     except AttributeError:
         return os.cpu_count() or 1
+
+
+def _libgomp():
+    import ctypes
+    try:
+        return ctypes.CDLL("libgomp.so.1")
+    except OSError:
+        return None
+
+
+def cpu_threads():
+    """Threads the oracle's OpenMP loops run with (OMP_NUM_THREADS, which
+    torchrun sets to 1 per rank, else every core this process may use)."""
+    gomp = _libgomp()
+    if gomp is not None:
+        return int(gomp.omp_get_max_threads())
+    env = os.environ.get("OMP_NUM_THREADS", "").split(",")[0].strip()
+    return int(env) if env.isdigit() and int(env) > 0 else host_cores()
+
+
+def use_all_cores():
+    """Let the oracle's OpenMP loops on this thread use every core this
+    process may use (the reference arm runs on rank 0 alone)."""
+    gomp = _libgomp()
+    if gomp is not None:
+        gomp.omp_set_num_threads(host_cores())
 
 
 def oracle_sample(cfg, X, W, target_s=15.0, orc_state=None, variant="w16"):
@@ -388,6 +414,7 @@ def reference_line(args, name, cfg, world, seconds):
 def run_reference(args, world, rank):
     if rank != 0:
         return
+    use_all_cores()                         # the other ranks do no work
     cfgs = all_configs()
     decode = args.decode_workload != "none"
     line = reference_line(args, args.workload, cfgs[args.workload], world, 80.0 if decode else 100.0)

@@ -150,3 +150,18 @@ def test_traffic_is_keyed_on_the_kernel_sources(tmp_path, monkeypatch):
     rec["captures"]["w"]["source_sha"] = "stale"
     (tmp_path / "ncu_traffic.json").write_text(json.dumps(rec))
     assert bench.ncu_traffic("w", "gemm_decode_kernel") is None
+
+
+def test_oracle_thread_count_follows_openmp():
+    """`cores` in the CPU baseline is the thread count the oracle's OpenMP loops
+    run with: OMP_NUM_THREADS when set (torchrun sets 1 per rank), and every
+    core of the process once the reference arm raises it on rank 0."""
+    import subprocess
+    import sys
+    code = ("import bench, oracle; oracle.default(); a = bench.cpu_threads(); bench.use_all_cores(); "
+            "print(a, bench.cpu_threads(), bench.host_cores())")
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    out = subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True,
+                         check=True).stdout.split()
+    before, after, host = map(int, out)
+    assert before == 1 and after == host >= 1

@@ -543,7 +543,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 // multiply-add per row (fma.rn.f32.f16: the fp16 product is exact in fp32,
 // one rounding per add, as in the tensor core's fp32 accumulation), where the
 // tensor path is bound by issuing MMAs.  The kernel is bound by instruction
-// issue (about 160 warp instructions per 1024 weights at T = 1), so each
+// issue (about 140 warp instructions per 1024 weights at T = 1), so each
 // further row costs about a third more; the host takes it for T <= 2.
 //   A stage is one (tile, 256 of K) unit as above: its packed codes and
 //   scales and the T rows of X over those 256 of K (bulk copies of 512 bytes),

@@ -533,3 +533,73 @@ def test_prefill_kernel_protocol_catches_planted_mistakes():
     with pytest.raises(Stale):                    # a tile's MMAs over an accumulator not yet drained
         for seed in range(300):
             run(prefill_kernel_roles(visits, 5, 2, 0, 3, skip_empty_wait=True), seed)
+
+
+# ---------------------------------------------------------------- the cooperative activation kernel
+
+def grid_barrier_run(blocks, failing, seed, fail_after_arrive=False):
+    """The grid barrier of activation_fused_kernel, one step per memory
+    operation.  Block b ORs its rows' bit into the mask if its row copies
+    arrived (all but `failing`); a block whose copies never arrived sets the
+    fail word; every block then adds itself to the counter and waits (bounded)
+    for all.  A block that goes on (counter complete, fail word clear) reads
+    the mask, which must hold the bits of every block.  Returns the blocks
+    that went on and the blocks whose wait gave up."""
+    rng = random.Random(seed)
+    mem = {"mask": 0, "ctr": 0, "fail": 0}
+
+    def block(b):
+        ok = b not in failing
+        if ok:
+            mem["mask"] |= 1 << b
+            yield
+        if not ok and not fail_after_arrive:
+            mem["fail"] = 1
+            yield
+        mem["ctr"] += 1
+        yield
+        if not ok and fail_after_arrive:
+            mem["fail"] = 1
+            yield
+        for _ in range(50):                           # the bounded wait
+            if mem["ctr"] >= blocks:
+                break
+            yield
+        else:
+            return ("gave_up", b)
+        yield
+        if ok and mem["fail"] == 0:
+            if mem["mask"] != (1 << blocks) - 1:
+                raise Stale(f"block {b} went on with mask {mem['mask']:b}")
+            return ("went_on", b)
+        return ("stopped", b)
+
+    gens = {b: block(b) for b in range(blocks)}
+    result = {}
+    while gens:
+        b = rng.choice(list(gens))
+        try:
+            next(gens[b])
+        except StopIteration as e:
+            result[b] = e.value
+            del gens[b]
+    return result
+
+
+@pytest.mark.parametrize("blocks,failing", [(6, set()), (6, {2}), (5, {0, 4}), (8, {7})])
+def test_grid_barrier_never_goes_on_with_an_incomplete_mask(blocks, failing):
+    for seed in range(400):
+        out = grid_barrier_run(blocks, failing, seed)
+        went = [b for b, (what, _) in out.items() if what == "went_on"]
+        if failing:
+            assert not went                            # the fail word stops every block
+        else:
+            assert all(what in ("went_on", "gave_up") for what, _ in out.values())
+
+
+def test_grid_barrier_model_catches_a_late_fail_word():
+    """Setting the fail word after arriving (the earlier ordering) lets a fast
+    block pass the barrier with a mask that lacks the failed block's rows."""
+    with pytest.raises(Stale):
+        for seed in range(400):
+            grid_barrier_run(6, {3}, seed, fail_after_arrive=True)
